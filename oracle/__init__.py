@@ -1,0 +1,10 @@
+"""CPU oracle (test infrastructure only; see ``oracle.paged_attention``)."""
+from .paged_attention import (  # noqa: F401
+    gather_sequence_kv,
+    paged_kv_append,
+    paged_tree_attention,
+    softmax_attend,
+    visible_positions,
+    widen_to_f64,
+    within_tolerance,
+)

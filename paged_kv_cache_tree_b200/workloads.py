@@ -1,0 +1,285 @@
+"""Seeded synthetic inputs for paged tree-attention verify and paged KV-append.
+
+This module only draws inputs; it holds none of the attention or append arithmetic, and it is the one
+piece of code that both the CPU oracle's tests and the CUDA path's tests/bench share.
+
+Shapes follow the workloads the TACO-LLM pages talk about: Llama-3.1-70B-like attention heads
+(64 query / 8 KV heads, head_dim 128) verifying lookahead candidates, arranged as a chain or as a
+forest-derived token tree, over a paged KV cache whose fixed-size blocks are reached through a block
+table ("大模型倍速推理引擎 TACO-LLM 的设计与实践", 53ai.com workshop page, sections
+"4. 支持 Paged Attention" and "优化方案设计思路"). The pages print no dataset; every value is
+drawn here from a seeded CPU ``torch.Generator``.
+
+Recipe (one generator per workload, seed = 1000 + k for the k-th named workload), in draw order:
+  1. context lengths L_b (uniform integers, inclusive bounds; they count the candidates too);
+  2. a random permutation of the physical block pool; sequence b takes the next ceil(L_b/bs) pool
+     entries, in order, as its block table (unused table entries are -1);
+  3. tree parents per sequence: a chain has parent[i] = i-1 (no draws); a forest draws parent[i]
+     uniformly from {-1, 0, ..., i-1};
+  4. q, then the K cache, then the V cache, then k_new, then v_new, all ~N(0,1) rounded to the dtype.
+Pool size is ceil(1.1 * sum_b ceil(L_b/bs)) blocks unless a workload fixes it. Memory the verify must
+never read (unmapped pool blocks, slots >= L_b of a sequence's last block, query rows of padding
+candidates) is filled with NaN for parity runs (``fill="nan"``) or zeros for timed runs.
+
+Candidate i of sequence b sits at logical position P_b + i with P_b = L_b - n_b. With
+``candidates_in_cache=True`` the cache already holds k_new/v_new there (the state after a
+paged KV-append); otherwise those slots are poisoned too and an append must fill them.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional, Sequence, Union
+
+import torch
+
+# name -> spec; index k (1-based) gives the seed 1000 + k.
+WORKLOADS = {
+    "tiny": dict(k=1, dtype="fp16", B=2, Hq=4, Hkv=2, D=64, bs=16, C=4, tree="chain",
+                 ctx=("fixed", [37, 100]), num_blocks=40),
+    "decode": dict(k=2, dtype="bf16", B=64, Hq=32, Hkv=8, D=128, bs=16, C=1, tree="chain",
+                   ctx=("uniform", 512, 4096)),
+    "chain": dict(k=3, dtype="bf16", B=32, Hq=64, Hkv=8, D=128, bs=16, C=8, tree="chain",
+                  ctx=("uniform", 1024, 8192)),
+    "tree": dict(k=4, dtype="bf16", B=16, Hq=64, Hkv=8, D=128, bs=32, C=16, tree="forest",
+                 ctx=("uniform", 2048, 16384)),
+    "long": dict(k=5, dtype="bf16", B=4, Hq=64, Hkv=8, D=128, bs=64, C=4, tree="chain",
+                 ctx=("uniform", 32768, 131072)),
+}
+
+WORKLOAD_DESCRIPTIONS = {
+    "tiny": "tiny paged tree-attention: B2, 4q/2kv, D64, fp16, bs16, L={37,100}, 40 blocks, C=4 chain",
+    "decode": "plain paged decode: B64, 32q/8kv, D128, bf16, bs16, L~U[512,4096], C=1",
+    "chain": "lookahead chain verify: B32, 64q/8kv, D128, bf16, bs16, L~U[1024,8192], C=8 chain",
+    "tree": "tree verify: B16, 64q/8kv, D128, bf16, bs32, L~U[2048,16384], C=16 random forest",
+    "long": "long-sequence verify: B4, 64q/8kv, D128, bf16, bs64, L~U[32768,131072], C=4 chain",
+}
+
+TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+_CHUNK = 1 << 24  # elements per randn call, so that huge caches are drawn without a giant fp32 temp
+
+
+@dataclasses.dataclass
+class Workload:
+    """Host (CPU) tensors of one verify step. Shapes use B, C, Hq, Hkv, D, bs, NB, maxblk."""
+
+    name: str
+    dtype: str                    # "bf16" | "fp16"
+    B: int
+    C: int
+    Hq: int
+    Hkv: int
+    D: int
+    bs: int
+    num_blocks: int
+    max_blocks: int
+    scale: float
+    context_lens: torch.Tensor    # int32 [B]      L_b, candidates included
+    num_candidates: torch.Tensor  # int32 [B]      n_b <= min(C, L_b)
+    parents: torch.Tensor         # int32 [B, C]   parent index or -1
+    tree_mask: torch.Tensor       # int32 [B, C]   uint32 bit pattern: bit j = row i may see candidate j
+    block_tables: torch.Tensor    # int32 [B, maxblk], -1 where unmapped
+    slot_offsets: torch.Tensor    # int32 [B, C]   P_b + i for i < n_b, else -1
+    q: torch.Tensor               # [B, C, Hq, D]
+    k_cache: torch.Tensor         # [NB, Hkv, bs, D]
+    v_cache: torch.Tensor         # [NB, Hkv, bs, D]
+    k_new: torch.Tensor           # [B, C, Hkv, D]
+    v_new: torch.Tensor           # [B, C, Hkv, D]
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    def kv_bytes(self) -> int:
+        """K+V bytes the verify must read: sum_b L_b * Hkv * D * elt * 2."""
+        return int(self.context_lens.long().sum()) * self.Hkv * self.D * 2 * 2
+
+    def qo_bytes(self) -> int:
+        """Q + O bytes: 2 * B * C * Hq * D * elt."""
+        return 2 * self.B * self.C * self.Hq * self.D * 2
+
+    def append_bytes(self) -> int:
+        """K/V-append bytes moved: (read + write) of every appended row of K and V."""
+        rows = int(self.num_candidates.long().sum())
+        return 2 * 2 * rows * self.Hkv * self.D * 2
+
+    def candidate_tokens(self) -> int:
+        return int(self.num_candidates.long().sum())
+
+    def to(self, device) -> "Workload":
+        out = dataclasses.replace(self)
+        for f in dataclasses.fields(self):
+            v = getattr(self, f.name)
+            if isinstance(v, torch.Tensor):
+                setattr(out, f.name, v.to(device))
+        return out
+
+
+def _randn(n: int, g: torch.Generator, dtype: torch.dtype) -> torch.Tensor:
+    out = torch.empty(n, dtype=dtype)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        out[s:e] = torch.randn(e - s, generator=g).to(dtype)
+    return out
+
+
+def chain_parents(C: int) -> list:
+    return [i - 1 for i in range(C)]
+
+
+def masks_from_parents(parents: Sequence[int], n: int) -> list:
+    """Ancestor-or-self bit sets (bit j = candidate j) for rows i < n; rows i >= n get 0."""
+    masks = []
+    for i in range(len(parents)):
+        if i >= n:
+            masks.append(0)
+            continue
+        m = 1 << i
+        p = parents[i]
+        if p >= 0:
+            m |= masks[p]
+        masks.append(m)
+    return masks
+
+
+def _to_i32_bits(words: Sequence[int]) -> list:
+    return [w - (1 << 32) if w >= (1 << 31) else w for w in words]
+
+
+def make_workload(
+    spec: Union[str, dict],
+    *,
+    seed: Optional[int] = None,
+    fill: str = "nan",
+    candidates_in_cache: bool = True,
+    context_lens: Optional[Sequence[int]] = None,
+    num_candidates: Optional[Sequence[int]] = None,
+    parents: Optional[Sequence[Sequence[int]]] = None,
+    pool_slack: float = 1.1,
+    extra_table_cols: int = 0,
+) -> Workload:
+    """Draw one workload.
+
+    ``spec`` is a name of ``WORKLOADS`` or a dict with the same keys (dtype, B, Hq, Hkv, D, bs, C,
+    tree in {"chain", "forest"}, ctx = ("fixed", [..]) | ("uniform", lo, hi), optional num_blocks).
+    ``context_lens`` / ``num_candidates`` / ``parents`` override what the spec would draw (the draws
+    still happen, so the stream of later draws does not move).
+    """
+    if isinstance(spec, str):
+        name = spec
+        sp = dict(WORKLOADS[spec])
+    else:
+        sp = dict(spec)
+        name = sp.get("name", "custom")
+    if seed is None:
+        seed = 1000 + int(sp.get("k", 0))
+    if fill not in ("nan", "zero"):
+        raise ValueError("fill must be 'nan' or 'zero'")
+    tdt = TORCH_DTYPES[sp["dtype"]]
+    B, C, Hq, Hkv, D, bs = (int(sp[x]) for x in ("B", "C", "Hq", "Hkv", "D", "bs"))
+    g = torch.Generator().manual_seed(int(seed))
+
+    # 1. context lengths
+    ctx = sp["ctx"]
+    if ctx[0] == "fixed":
+        L = [int(x) for x in ctx[1]]
+    else:
+        L = [int(x) for x in torch.randint(int(ctx[1]), int(ctx[2]) + 1, (B,), generator=g)]
+    if context_lens is not None:
+        L = [int(x) for x in context_lens]
+    assert len(L) == B
+    if num_candidates is None:
+        n = [min(C, Lb) for Lb in L]
+    else:
+        n = [int(x) for x in num_candidates]
+    for b in range(B):
+        if not (0 <= n[b] <= C and n[b] <= L[b]):
+            raise ValueError(f"need 0 <= n_b <= min(C, L_b); got n={n[b]} L={L[b]} C={C}")
+
+    # 2. block pool permutation and block tables
+    nblk = [(Lb + bs - 1) // bs for Lb in L]
+    total = sum(nblk)
+    NB = int(sp.get("num_blocks") or math.ceil(pool_slack * total))
+    NB = max(NB, total, 1)
+    perm = torch.randperm(NB, generator=g)
+    maxblk = max(max(nblk), 1) + int(extra_table_cols)
+    bt = torch.full((B, maxblk), -1, dtype=torch.int32)
+    off = 0
+    for b in range(B):
+        bt[b, : nblk[b]] = perm[off: off + nblk[b]].to(torch.int32)
+        off += nblk[b]
+
+    # 3. tree parents
+    par = []
+    for b in range(B):
+        if sp["tree"] == "chain":
+            pb = chain_parents(C)
+        elif sp["tree"] == "forest":
+            pb = [int(torch.randint(0, i + 1, (1,), generator=g)) - 1 for i in range(C)]
+        else:
+            raise ValueError("tree must be 'chain' or 'forest'")
+        par.append(pb)
+    if parents is not None:
+        par = [list(map(int, p)) for p in parents]
+    masks = [_to_i32_bits(masks_from_parents(par[b], n[b])) for b in range(B)]
+
+    # 4. values
+    q = _randn(B * C * Hq * D, g, tdt).view(B, C, Hq, D)
+    k_cache = _randn(NB * Hkv * bs * D, g, tdt).view(NB, Hkv, bs, D)
+    v_cache = _randn(NB * Hkv * bs * D, g, tdt).view(NB, Hkv, bs, D)
+    k_new = _randn(B * C * Hkv * D, g, tdt).view(B, C, Hkv, D)
+    v_new = _randn(B * C * Hkv * D, g, tdt).view(B, C, Hkv, D)
+
+    poison = float("nan") if fill == "nan" else 0.0
+    used = torch.zeros(NB, dtype=torch.bool)
+    for b in range(B):
+        blocks = bt[b, : nblk[b]].long()
+        used[blocks] = True
+        P = L[b] - n[b]
+        if nblk[b] > 0:
+            last = int(bt[b, nblk[b] - 1])
+            tail = L[b] - (nblk[b] - 1) * bs          # valid slots in the last block
+            k_cache[last, :, tail:, :] = poison
+            v_cache[last, :, tail:, :] = poison
+        for i in range(n[b]):
+            p = P + i
+            blk = int(bt[b, p // bs])
+            if candidates_in_cache:
+                k_cache[blk, :, p % bs, :] = k_new[b, i]
+                v_cache[blk, :, p % bs, :] = v_new[b, i]
+            else:
+                k_cache[blk, :, p % bs, :] = poison
+                v_cache[blk, :, p % bs, :] = poison
+        q[b, n[b]:] = poison
+        k_new[b, n[b]:] = poison
+        v_new[b, n[b]:] = poison
+    k_cache[~used] = poison
+    v_cache[~used] = poison
+
+    slots = torch.full((B, C), -1, dtype=torch.int32)
+    for b in range(B):
+        P = L[b] - n[b]
+        for i in range(n[b]):
+            slots[b, i] = P + i
+
+    return Workload(
+        name=name, dtype=sp["dtype"], B=B, C=C, Hq=Hq, Hkv=Hkv, D=D, bs=bs, num_blocks=NB,
+        max_blocks=maxblk, scale=1.0 / math.sqrt(D),
+        context_lens=torch.tensor(L, dtype=torch.int32),
+        num_candidates=torch.tensor(n, dtype=torch.int32),
+        parents=torch.tensor(par, dtype=torch.int32).view(B, C),
+        tree_mask=torch.tensor(masks, dtype=torch.int32).view(B, C),
+        block_tables=bt, slot_offsets=slots, q=q, k_cache=k_cache, v_cache=v_cache,
+        k_new=k_new, v_new=v_new,
+    )
+
+
+def to_numpy_bits(t: torch.Tensor):
+    """Raw 16-bit patterns of a bf16/fp16 tensor as a numpy uint16 array (no value conversion)."""
+    return t.contiguous().view(torch.int16).numpy().view("uint16")
+
+
+def as_uint32(t: torch.Tensor):
+    """int32 tensor holding uint32 bit patterns -> numpy uint32 array."""
+    return t.contiguous().numpy().view("uint32")
