@@ -1,0 +1,137 @@
+/*
+ * libtaco_attn: paged tree-attention verify and paged KV-append for NVIDIA B200 (sm_100a).
+ *
+ * The operations come from public TACO-LLM pages:
+ *  - paging: "大模型倍速推理引擎 TACO-LLM 的设计与实践" (53ai.com workshop page), section
+ *    "4. 支持 Paged Attention": a sequence's KV cache is cut into blocks of a fixed number of tokens,
+ *    and consecutive logical blocks map to non-contiguous physical blocks through a block table;
+ *    blocks are filled as new tokens are produced.
+ *  - verification and tree attention: same page, sections "TACO-LLM 如何解决大模型推理瓶颈?",
+ *    "优化方案设计思路" and "优化策略总结" item 1: the target model checks a batch of candidate tokens
+ *    in one parallel pass, and candidates sharing a prefix share its computation (each candidate sees
+ *    the committed prefix and its own ancestors).
+ *  - TurboAttention: same page, the kernel bullets under "整体方案分为两大部分" (paged + flash-style
+ *    fused softmax; several candidates turn vector-matrix into matrix-matrix work for tensor cores),
+ *    and the 618zxw.cn article, section "長シーケンス推論最適化におけるTurboAttention".
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device, owned by the caller, and must
+ *    stay valid until the work enqueued on `stream` has finished. Nothing is copied to or from host.
+ *  - Calls only enqueue work on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ *    return; they do not synchronise.
+ *  - Every array is dense, row-major, innermost dimension last. 16-bit float tensors must start on a
+ *    16-byte boundary.
+ *  - Host-side validation runs before any launch; a non-OK status means nothing was enqueued, and
+ *    taco_attn_last_error() gives a message (thread-local).
+ *  - Values inside device arrays (block ids, lengths, slots) are checked on the device: an
+ *    out-of-range value sets a bit in a per-device error word and the offending access is skipped
+ *    (it never faults or traps). taco_attn_check_device() reads and clears that word.
+ *
+ * Shapes: B batch, C max candidates per sequence (1..32), Hq / Hkv query / KV heads (Hq % Hkv == 0,
+ * G = Hq / Hkv), D head dim (64 or 128), bs block size (power of two, 8..256), NB physical blocks,
+ * maxblk block-table columns.
+ */
+#ifndef TACO_ATTN_H
+#define TACO_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t taco_status;
+#define TACO_OK 0
+#define TACO_ERR_INVALID_ARG 1   /* null pointer, bad size, misaligned pointer */
+#define TACO_ERR_UNSUPPORTED 2   /* a size this build has no kernel for (D, bs, C) */
+#define TACO_ERR_CUDA 3          /* a CUDA runtime call or launch failed */
+#define TACO_ERR_DEVICE_CHECK 4  /* taco_attn_check_device found a device-side range error */
+
+#define TACO_DTYPE_F16 0
+#define TACO_DTYPE_BF16 1
+
+/* Device error word bits (taco_attn_check_device). */
+#define TACO_DEVERR_BLOCK_ID 0x1u       /* block table entry outside [0, NB) */
+#define TACO_DEVERR_CONTEXT_LEN 0x2u    /* context_lens[b] outside [0, maxblk * bs] */
+#define TACO_DEVERR_NUM_CAND 0x4u       /* num_candidates[b] outside [0, min(C, context_lens[b])] */
+#define TACO_DEVERR_SLOT 0x8u           /* slot_offsets[b][i] >= maxblk * bs */
+#define TACO_DEVERR_WAIT_TIMEOUT 0x10u  /* a pipeline wait gave up (the kernel returned early) */
+
+/*
+ * paged_tree_attention: masked softmax attention of every candidate query over its sequence's
+ * paged keys (the TurboAttention verify pass).
+ *
+ *   q               [B, C, Hq, D]   dtype; row (b, i, h) is candidate i of sequence b, query head h
+ *   k_cache,v_cache [NB, Hkv, bs, D] dtype; (block, kv head, slot, dim)
+ *   block_tables    int32 [B, maxblk]; logical block j of sequence b is physical block
+ *                   block_tables[b*maxblk + j] (entries past ceil(L_b/bs) are never read)
+ *   context_lens    int32 [B]; L_b = number of keys of sequence b, its n_b candidates included; the
+ *                   candidates' K/V sit at logical positions P_b .. L_b-1, P_b = L_b - n_b (written
+ *                   before this call, e.g. by paged_kv_append)
+ *   num_candidates  int32 [B]; n_b, 0 <= n_b <= min(C, L_b)
+ *   tree_mask_bits  uint32 [B, C]; bit j of word (b, i): candidate i may attend to candidate j.
+ *                   Bits j >= n_b are ignored. Any pattern is allowed (a chain is 2^(i+1)-1, a tree
+ *                   is the ancestor-or-self set).
+ *   scale           multiplies q.k before the softmax (usually 1/sqrt(D))
+ *   out             [B, C, Hq, D] dtype, written completely: row (b, i, h) with i < n_b is
+ *                   sum_p softmax_p(scale q.k_p) v_p over the visible positions p (the prefix
+ *                   0..P_b-1 plus the candidates its mask word selects); rows i >= n_b and rows that
+ *                   see no key are zeros. Must not alias any input.
+ *   query head h reads KV head h / G.
+ * Softmax state (max, sum) and the output accumulator are fp32; the result is rounded once to
+ * `dtype` (round to nearest even). The library keeps a per-device workspace for split-KV partial
+ * results; the first call on a device (or one that needs a larger workspace) allocates it with
+ * cudaMalloc and therefore synchronises the device.
+ */
+taco_status paged_tree_attention(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* block_tables, const int32_t* context_lens,
+                                 const int32_t* num_candidates, const uint32_t* tree_mask_bits,
+                                 float scale, void* out,
+                                 int32_t dtype, int32_t batch, int32_t max_candidates,
+                                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                 void* stream);
+
+/*
+ * paged_kv_append: write the candidates' new K/V rows into their cache slots through the block
+ * table (paging section cited above: blocks are filled as tokens are generated).
+ *
+ *   k_new, v_new    [B, C, Hkv, D] dtype
+ *   block_tables    int32 [B, maxblk]
+ *   slot_offsets    int32 [B, C]; logical position s of row (b, i); s < 0 means "skip this row".
+ *                   Row (b, i, h) is copied bit-for-bit to cache[block_tables[b][s / bs], h, s % bs, :].
+ *                   Slots within one call must be distinct (otherwise which row lands is undefined).
+ *   k_cache,v_cache [NB, Hkv, bs, D] dtype, updated in place; no other byte changes.
+ */
+taco_status paged_kv_append(const void* k_new, const void* v_new, const int32_t* block_tables,
+                            const int32_t* slot_offsets, void* k_cache, void* v_cache,
+                            int32_t dtype, int32_t batch, int32_t max_candidates,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int32_t num_blocks, int32_t max_blocks_per_seq, void* stream);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* taco_attn_last_error(void);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's error word. Returns TACO_OK if it
+ * was zero, TACO_ERR_DEVICE_CHECK otherwise (the bits are in the message and in *bits_out when
+ * bits_out is not NULL). After a wait timeout it also clears the split-KV arrival counters.
+ */
+taco_status taco_attn_check_device(void* stream, uint32_t* bits_out);
+
+/* Free the per-device workspaces (call only when no work using them is in flight). */
+void taco_attn_release_workspace(void);
+
+/* Tuning / test knobs (process-wide). */
+#define TACO_OPT_GRID_CTAS 1   /* verify grid size in CTAs; 0 = automatic (2 per SM). */
+#define TACO_OPT_KERNEL 2      /* 0 = automatic, 1 = mma.sync path, 2 = tcgen05 path (where built) */
+taco_status taco_attn_set_option(int32_t key, int64_t value);
+
+/* ABI version of this header (bumped on any signature change). */
+int32_t taco_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TACO_ATTN_H */

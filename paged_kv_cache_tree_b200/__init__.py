@@ -1,0 +1,17 @@
+"""B200-native paged tree-attention verify and paged KV-append (libtaco_attn + a thin binding).
+
+The compute path is the C-ABI library ``libtaco_attn.so`` built from ``csrc/`` for sm_100a; the
+functions below only marshal torch tensors into its pointers and sizes.
+"""
+from ._lib import (  # noqa: F401
+    TACO_OPT_GRID_CTAS,
+    TACO_OPT_KERNEL,
+    TacoError,
+    check_device,
+    load,
+    paged_kv_append,
+    paged_tree_attention,
+    release_workspace,
+    set_option,
+    version,
+)

@@ -1,0 +1,180 @@
+"""ctypes binding of libtaco_attn (argument marshalling only).
+
+Every function here takes torch tensors for device memory and a CUDA stream, turns them into the
+pointers and sizes of the C ABI in ``include/taco_attn.h`` and calls it. No arithmetic of the method
+happens here, and there is no fallback: if the shared library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtaco_attn.so")
+
+TACO_OK = 0
+TACO_ERR_INVALID_ARG = 1
+TACO_ERR_UNSUPPORTED = 2
+TACO_ERR_CUDA = 3
+TACO_ERR_DEVICE_CHECK = 4
+
+TACO_DTYPE_F16 = 0
+TACO_DTYPE_BF16 = 1
+
+TACO_OPT_GRID_CTAS = 1
+TACO_OPT_KERNEL = 2
+
+EXPORTED = (
+    "paged_tree_attention",
+    "paged_kv_append",
+    "taco_attn_last_error",
+    "taco_attn_check_device",
+    "taco_attn_release_workspace",
+    "taco_attn_set_option",
+    "taco_attn_version",
+)
+
+_lib = None
+
+
+class TacoError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"libtaco_attn status {status}: {message}")
+        self.status = status
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree library (built by ``paged_kv_cache_tree_b200.build_lib``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_tree_b200.build_lib`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    lib.paged_tree_attention.argtypes = [vp] * 7 + [f32, vp] + [i32] * 9 + [vp]
+    lib.paged_tree_attention.restype = i32
+    lib.paged_kv_append.argtypes = [vp] * 6 + [i32] * 8 + [vp]
+    lib.paged_kv_append.restype = i32
+    lib.taco_attn_last_error.argtypes = []
+    lib.taco_attn_last_error.restype = ctypes.c_char_p
+    lib.taco_attn_check_device.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.taco_attn_check_device.restype = i32
+    lib.taco_attn_release_workspace.argtypes = []
+    lib.taco_attn_release_workspace.restype = None
+    lib.taco_attn_set_option.argtypes = [i32, ctypes.c_int64]
+    lib.taco_attn_set_option.restype = i32
+    lib.taco_attn_version.argtypes = []
+    lib.taco_attn_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != TACO_OK:
+        msg = load().taco_attn_last_error().decode(errors="replace")
+        raise TacoError(status, msg)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return TACO_DTYPE_BF16
+    if t.dtype == torch.float16:
+        return TACO_DTYPE_F16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected bfloat16 or float16")
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream], device: torch.device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return int(s.cuda_stream)
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtype=None, ndim=None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {t.dim()}")
+
+
+def paged_tree_attention(q, k_cache, v_cache, block_tables, context_lens, num_candidates, tree_mask_bits,
+                         scale: float, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """q [B,C,Hq,D]; k/v_cache [NB,Hkv,bs,D]; block_tables int32 [B,maxblk]; context_lens and
+    num_candidates int32 [B]; tree_mask_bits int32/uint32 [B,C] (bit patterns). Returns ``out``."""
+    _need_cuda("q", q, (torch.bfloat16, torch.float16), 4)
+    _need_cuda("k_cache", k_cache, q.dtype, 4)
+    _need_cuda("v_cache", v_cache, q.dtype, 4)
+    _need_cuda("block_tables", block_tables, torch.int32, 2)
+    _need_cuda("context_lens", context_lens, torch.int32, 1)
+    _need_cuda("num_candidates", num_candidates, torch.int32, 1)
+    _need_cuda("tree_mask_bits", tree_mask_bits, (torch.int32, torch.uint32), 2)
+    B, C, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache / v_cache shape mismatch with q")
+    if block_tables.shape[0] != B or context_lens.shape[0] != B or num_candidates.shape[0] != B:
+        raise ValueError("batch dimension mismatch")
+    if tuple(tree_mask_bits.shape) != (B, C):
+        raise ValueError("tree_mask_bits must be [B, C]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need_cuda("out", out, q.dtype, 4)
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must have q's shape")
+    lib = load()
+    _check(lib.paged_tree_attention(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), context_lens.data_ptr(),
+        num_candidates.data_ptr(), tree_mask_bits.data_ptr(), float(scale), out.data_ptr(),
+        _dtype_code(q), B, C, Hq, Hkv, D, bs, NB, block_tables.shape[1],
+        _stream_handle(stream, q.device)))
+    return out
+
+
+def paged_kv_append(k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, stream=None) -> None:
+    """k_new, v_new [B,C,Hkv,D]; slot_offsets int32 [B,C] (-1 = skip); caches updated in place."""
+    _need_cuda("k_new", k_new, (torch.bfloat16, torch.float16), 4)
+    _need_cuda("v_new", v_new, k_new.dtype, 4)
+    _need_cuda("block_tables", block_tables, torch.int32, 2)
+    _need_cuda("slot_offsets", slot_offsets, torch.int32, 2)
+    _need_cuda("k_cache", k_cache, k_new.dtype, 4)
+    _need_cuda("v_cache", v_cache, k_new.dtype, 4)
+    B, C, Hkv, D = k_new.shape
+    NB, Hkv2, bs, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(v_new.shape) != tuple(k_new.shape):
+        raise ValueError("shape mismatch between new rows and caches")
+    if tuple(slot_offsets.shape) != (B, C) or block_tables.shape[0] != B:
+        raise ValueError("slot_offsets must be [B, C] and block_tables [B, maxblk]")
+    lib = load()
+    _check(lib.paged_kv_append(
+        k_new.data_ptr(), v_new.data_ptr(), block_tables.data_ptr(), slot_offsets.data_ptr(),
+        k_cache.data_ptr(), v_cache.data_ptr(), _dtype_code(k_new), B, C, Hkv, D, bs, NB,
+        block_tables.shape[1], _stream_handle(stream, k_new.device)))
+
+
+def check_device(stream=None, device=None) -> int:
+    """Synchronise the stream and return the device error bits (raises TacoError if any are set)."""
+    lib = load()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    bits = ctypes.c_uint32(0)
+    st = lib.taco_attn_check_device(_stream_handle(stream, dev), ctypes.byref(bits))
+    _check(st)
+    return int(bits.value)
+
+
+def set_option(key: int, value: int) -> None:
+    _check(load().taco_attn_set_option(int(key), int(value)))
+
+
+def release_workspace() -> None:
+    load().taco_attn_release_workspace()
+
+
+def version() -> int:
+    return int(load().taco_attn_version())

@@ -1,0 +1,329 @@
+// Host side of libtaco_attn: argument validation, per-device workspace, TMA descriptors and
+// kernel dispatch behind the C ABI declared in taco_attn.h.
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "device_common.cuh"
+#include "launchers.h"
+#include "taco_attn.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kAbiVersion = 1;
+
+thread_local std::string g_last_error;
+
+taco_status fail(taco_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+taco_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(TACO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Workspace of one device: [error word | counters | partial lse | partial O].
+struct Workspace {
+  uint8_t* base = nullptr;
+  size_t bytes = 0;
+  uint32_t* error_word = nullptr;
+  uint32_t* counters = nullptr;
+  size_t counters_cap = 0;
+  float* part_lse = nullptr;
+  size_t lse_cap = 0;  // floats
+  float* part_o = nullptr;
+  size_t o_cap = 0;    // floats
+  int sm_count = 0;
+};
+
+std::mutex g_mu;
+Workspace g_ws[kMaxDevices];
+int64_t g_opt_grid = 0;
+int64_t g_opt_kernel = 0;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Make sure device `dev`'s workspace has room; returns a status. Caller holds g_mu.
+taco_status ensure_workspace(int dev, size_t counters, size_t lse_floats, size_t o_floats) {
+  Workspace& w = g_ws[dev];
+  if (w.sm_count == 0) {
+    cudaError_t e = cudaDeviceGetAttribute(&w.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  }
+  if (w.base && counters <= w.counters_cap && lse_floats <= w.lse_cap && o_floats <= w.o_cap) return TACO_OK;
+  // grow (keeping at least the old capacities); the old buffer may still be in use by queued
+  // work, so wait for the device before freeing it
+  counters = std::max(counters, w.counters_cap);
+  lse_floats = std::max(lse_floats, w.lse_cap);
+  o_floats = std::max(o_floats, w.o_cap);
+  const size_t off_counters = 256;
+  const size_t off_lse = off_counters + round_up(counters * 4, 256);
+  const size_t off_o = off_lse + round_up(lse_floats * 4, 256);
+  const size_t total = off_o + round_up(o_floats * 4, 256);
+  uint32_t old_err = 0;
+  if (w.base) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize (workspace grow)");
+    cudaMemcpy(&old_err, w.error_word, 4, cudaMemcpyDeviceToHost);
+    cudaFree(w.base);
+    w = Workspace{nullptr, 0, nullptr, nullptr, 0, nullptr, 0, nullptr, 0, w.sm_count};
+  }
+  void* p = nullptr;
+  cudaError_t e = cudaMalloc(&p, total);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc (workspace)");
+  e = cudaMemset(p, 0, off_lse);  // error word and counters start at zero
+  if (e != cudaSuccess) {
+    cudaFree(p);
+    return cuda_fail(e, "cudaMemset (workspace)");
+  }
+  if (old_err) cudaMemcpy(p, &old_err, 4, cudaMemcpyHostToDevice);
+  w.base = static_cast<uint8_t*>(p);
+  w.bytes = total;
+  w.error_word = reinterpret_cast<uint32_t*>(w.base);
+  w.counters = reinterpret_cast<uint32_t*>(w.base + off_counters);
+  w.counters_cap = counters;
+  w.part_lse = reinterpret_cast<float*>(w.base + off_lse);
+  w.lse_cap = lse_floats;
+  w.part_o = reinterpret_cast<float*>(w.base + off_o);
+  w.o_cap = o_floats;
+  return TACO_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* sym = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &sym, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(sym);
+  });
+  return fn;
+}
+
+// [NB * Hkv * bs rows, D columns] view of a cache; box = 64 columns (one 128-byte swizzle row) x
+// rows_per_chunk rows.
+taco_status make_cache_map(CUtensorMap* map, const void* base, int dtype, int D, int64_t rows, int rows_per_chunk) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(rows_per_chunk)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dtype == TACO_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return TACO_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+taco_status check_common(int32_t dtype, int32_t batch, int32_t max_candidates, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t block_size, int32_t num_blocks, int32_t max_blocks) {
+  if (dtype != TACO_DTYPE_F16 && dtype != TACO_DTYPE_BF16) return fail(TACO_ERR_INVALID_ARG, "dtype must be F16 (0) or BF16 (1)");
+  if (batch < 0) return fail(TACO_ERR_INVALID_ARG, "batch must be >= 0");
+  if (max_candidates < 1) return fail(TACO_ERR_INVALID_ARG, "max_candidates must be >= 1");
+  if (max_candidates > 32) return fail(TACO_ERR_UNSUPPORTED, "max_candidates must be <= 32 (one 32-bit mask word per row)");
+  if (num_kv_heads < 1) return fail(TACO_ERR_INVALID_ARG, "num_kv_heads must be >= 1");
+  if (head_dim != 64 && head_dim != 128) return fail(TACO_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (!is_pow2(block_size) || block_size < 8 || block_size > 256)
+    return fail(TACO_ERR_UNSUPPORTED, "block_size must be a power of two in [8, 256]");
+  if (num_blocks < 1) return fail(TACO_ERR_INVALID_ARG, "num_blocks must be >= 1");
+  if (max_blocks < 1) return fail(TACO_ERR_INVALID_ARG, "max_blocks_per_seq must be >= 1");
+  if (static_cast<int64_t>(num_blocks) * num_kv_heads * block_size > INT32_MAX)
+    return fail(TACO_ERR_UNSUPPORTED, "num_blocks * num_kv_heads * block_size must fit in int32");
+  if (static_cast<int64_t>(max_blocks) * block_size > INT32_MAX)
+    return fail(TACO_ERR_UNSUPPORTED, "max_blocks_per_seq * block_size must fit in int32");
+  return TACO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t taco_attn_version(void) { return kAbiVersion; }
+
+const char* taco_attn_last_error(void) { return g_last_error.c_str(); }
+
+taco_status taco_attn_set_option(int32_t key, int64_t value) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (key == TACO_OPT_GRID_CTAS) {
+    if (value < 0 || value > (1 << 20)) return fail(TACO_ERR_INVALID_ARG, "grid size out of range");
+    g_opt_grid = value;
+    return TACO_OK;
+  }
+  if (key == TACO_OPT_KERNEL) {
+    if (value < 0 || value > 2) return fail(TACO_ERR_INVALID_ARG, "kernel choice must be 0, 1 or 2");
+    g_opt_kernel = value;
+    return TACO_OK;
+  }
+  return fail(TACO_ERR_INVALID_ARG, "unknown option key %d", key);
+}
+
+taco_status paged_tree_attention(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* block_tables, const int32_t* context_lens,
+                                 const int32_t* num_candidates, const uint32_t* tree_mask_bits, float scale,
+                                 void* out, int32_t dtype, int32_t batch, int32_t max_candidates,
+                                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
+  taco_status st = check_common(dtype, batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks,
+                                max_blocks_per_seq);
+  if (st != TACO_OK) return st;
+  if (num_q_heads < 1 || num_q_heads % num_kv_heads != 0)
+    return fail(TACO_ERR_INVALID_ARG, "num_q_heads must be a positive multiple of num_kv_heads");
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !num_candidates || !tree_mask_bits || !out)
+    return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return fail(TACO_ERR_INVALID_ARG, "q, k_cache, v_cache and out must be 16-byte aligned");
+  if (!(scale == scale)) return fail(TACO_ERR_INVALID_ARG, "scale is NaN");
+  if (batch == 0) return TACO_OK;
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(TACO_ERR_UNSUPPORTED, "device index %d too large", dev);
+
+  const int G = num_q_heads / num_kv_heads;
+  const int packed = G * max_candidates;
+  const int rows = taco::mma_rows_per_unit(packed);
+  const int row_groups = (packed + rows - 1) / rows;
+  const int64_t units = static_cast<int64_t>(batch) * num_kv_heads * row_groups;
+
+  std::lock_guard<std::mutex> lk(g_mu);
+  int grid = static_cast<int>(g_opt_grid);
+  if (grid == 0) {
+    if (g_ws[dev].sm_count == 0) {
+      e = cudaDeviceGetAttribute(&g_ws[dev].sm_count, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    }
+    grid = 2 * g_ws[dev].sm_count;
+  }
+  const size_t slots = 2 * static_cast<size_t>(grid);
+  st = ensure_workspace(dev, static_cast<size_t>(units), slots * rows, slots * rows * head_dim);
+  if (st != TACO_OK) return st;
+  Workspace& w = g_ws[dev];
+
+  const int rpc = block_size < taco::kTileKeys ? block_size : taco::kTileKeys;
+  const int64_t cache_rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
+  CUtensorMap tk, tv;
+  st = make_cache_map(&tk, k_cache, dtype, head_dim, cache_rows, rpc);
+  if (st != TACO_OK) return st;
+  st = make_cache_map(&tv, v_cache, dtype, head_dim, cache_rows, rpc);
+  if (st != TACO_OK) return st;
+
+  taco::VerifyParams p{};
+  p.q = q;
+  p.out = out;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.num_candidates = num_candidates;
+  p.tree_mask_bits = tree_mask_bits;
+  p.part_o = w.part_o;
+  p.part_lse = w.part_lse;
+  p.counters = w.counters;
+  p.error_word = w.error_word;
+  p.scale_log2 = scale * taco::kLog2e;
+  p.B = batch;
+  p.C = max_candidates;
+  p.Hq = num_q_heads;
+  p.Hkv = num_kv_heads;
+  p.G = G;
+  p.D = head_dim;
+  p.bs = block_size;
+  p.num_blocks = num_blocks;
+  p.max_blocks = max_blocks_per_seq;
+  p.rows_per_unit = rows;
+  p.row_groups = row_groups;
+
+  e = taco::launch_verify_mma(tk, tv, p, dtype, grid, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "verify kernel launch");
+  return TACO_OK;
+}
+
+taco_status paged_kv_append(const void* k_new, const void* v_new, const int32_t* block_tables,
+                            const int32_t* slot_offsets, void* k_cache, void* v_cache, int32_t dtype,
+                            int32_t batch, int32_t max_candidates, int32_t num_kv_heads, int32_t head_dim,
+                            int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
+  taco_status st = check_common(dtype, batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks,
+                                max_blocks_per_seq);
+  if (st != TACO_OK) return st;
+  if (!k_new || !v_new || !block_tables || !slot_offsets || !k_cache || !v_cache)
+    return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(TACO_ERR_INVALID_ARG, "k_new, v_new, k_cache and v_cache must be 16-byte aligned");
+  if (batch == 0) return TACO_OK;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(TACO_ERR_UNSUPPORTED, "device index %d too large", dev);
+  uint32_t* err = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    st = ensure_workspace(dev, 0, 0, 0);
+    if (st != TACO_OK) return st;
+    err = g_ws[dev].error_word;
+  }
+  taco::AppendArgs a{k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, err,
+                     batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq};
+  e = taco::launch_append(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+  return TACO_OK;
+}
+
+taco_status taco_attn_check_device(void* stream, uint32_t* bits_out) {
+  if (bits_out) *bits_out = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(TACO_ERR_UNSUPPORTED, "device index %d too large", dev);
+  e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[dev];
+  if (!w.base) return TACO_OK;
+  uint32_t bits = 0;
+  e = cudaMemcpy(&bits, w.error_word, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy (error word)");
+  if (bits_out) *bits_out = bits;
+  if (bits == 0) return TACO_OK;
+  cudaMemset(w.error_word, 0, 4);
+  if (bits & TACO_DEVERR_WAIT_TIMEOUT) cudaMemset(w.counters, 0, w.counters_cap * 4);
+  return fail(TACO_ERR_DEVICE_CHECK, "device range check failed: bits 0x%x%s%s%s%s%s", bits,
+              (bits & TACO_DEVERR_BLOCK_ID) ? " [block id out of range]" : "",
+              (bits & TACO_DEVERR_CONTEXT_LEN) ? " [context length out of range]" : "",
+              (bits & TACO_DEVERR_NUM_CAND) ? " [candidate count out of range]" : "",
+              (bits & TACO_DEVERR_SLOT) ? " [slot out of range]" : "",
+              (bits & TACO_DEVERR_WAIT_TIMEOUT) ? " [pipeline wait timed out]" : "");
+}
+
+void taco_attn_release_workspace(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (int d = 0; d < kMaxDevices; ++d) {
+    if (!g_ws[d].base) continue;
+    cudaSetDevice(d);
+    cudaFree(g_ws[d].base);
+    g_ws[d] = Workspace{};
+  }
+  cudaSetDevice(cur);
+}
+
+}  // extern "C"

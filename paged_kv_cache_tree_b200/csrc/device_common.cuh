@@ -1,0 +1,261 @@
+// Device-side building blocks shared by the verify and append kernels: shared-memory mbarriers,
+// TMA tile loads, ldmatrix / mma.sync wrappers, bounded waits and the split-KV work schedule.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "taco_attn.h"
+
+namespace taco {
+
+constexpr int kTileKeys = 64;                 // keys per pipeline stage
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a pipeline wait gives up after 2 s
+
+struct VerifyParams {
+  const void* q;
+  void* out;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* num_candidates;
+  const uint32_t* tree_mask_bits;
+  float* part_o;         // [slots, rows_per_unit, D] fp32 split-KV partial outputs (normalised)
+  float* part_lse;       // [slots, rows_per_unit] base-2 log-sum-exp of each partial
+  uint32_t* counters;    // [units] arrivals of split units (zero between calls)
+  uint32_t* error_word;  // device error bits
+  float scale_log2;      // scale * log2(e)
+  int B, C, Hq, Hkv, G, D, bs, num_blocks, max_blocks;
+  int rows_per_unit;     // packed query rows handled by one unit (row group)
+  int row_groups;        // ceil(G * C / rows_per_unit)
+};
+
+// ---------------------------------------------------------------------------------------------
+// small PTX wrappers
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Wait for the phase with the given parity to complete. Gives up after kWaitLimitNs, sets the
+// timeout bit in the error word and returns false (the caller then leaves its loop).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* error_word) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1; it < (1u << 30); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) break;
+  }
+  atomicOr(error_word, TACO_DEVERR_WAIT_TIMEOUT);
+  return false;
+}
+
+// 2-D TMA tile load global -> shared, completion counted in bytes on `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int32_t x, int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+template <typename T>
+struct MmaOp;
+
+template <>
+struct MmaOp<__nv_bfloat16> {
+  __device__ __forceinline__ static void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+
+template <>
+struct MmaOp<__half> {
+  __device__ __forceinline__ static void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+
+// ---------------------------------------------------------------------------------------------
+// split-KV work schedule ("stream-K" over key tiles)
+//
+// Work unit u = (b, kv head g, row group rg), ordered u = (b * Hkv + g) * RG + rg. Unit u holds
+// T_b = max(1, ceil(L_b / kTileKeys)) key tiles (an empty sequence still gets one tile, which
+// writes its zero rows). All units' tiles are concatenated into one range [0, W); CTA c of the nC
+// working CTAs takes tiles [c*W/nC, (c+1)*W/nC). A unit that falls into several CTAs' ranges is
+// split: each piece writes a partial (normalised output + log-sum-exp), and the CTA that arrives
+// last on the unit's counter combines them. Since each CTA's range is contiguous, only its first
+// and last piece can be partial, so CTA c owns two partial slots: 2c (its first piece) and 2c+1.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ int clamp_context(const VerifyParams& p, int b, bool report) {
+  int L = __ldg(p.context_lens + b);
+  const int cap = p.max_blocks * p.bs;
+  if (L < 0 || L > cap) {
+    if (report) atomicOr(p.error_word, TACO_DEVERR_CONTEXT_LEN);
+    L = L < 0 ? 0 : cap;
+  }
+  return L;
+}
+
+__device__ __forceinline__ int clamp_candidates(const VerifyParams& p, int b, int L, bool report) {
+  int n = __ldg(p.num_candidates + b);
+  const int cap = L < p.C ? L : p.C;
+  if (n < 0 || n > cap) {
+    if (report) atomicOr(p.error_word, TACO_DEVERR_NUM_CAND);
+    n = n < 0 ? 0 : cap;
+  }
+  return n;
+}
+
+__device__ __forceinline__ int tiles_of(int L) { return L <= 0 ? 1 : (L + kTileKeys - 1) / kTileKeys; }
+
+// first CTA (of nC over W tiles) whose range contains tile t
+__device__ __forceinline__ int cta_of_tile(int64_t t, int64_t W, int64_t nC) {
+  return static_cast<int>(((t + 1) * nC - 1) / W);
+}
+
+struct SchedStart {
+  int64_t W;        // total tiles
+  int nC;           // working CTAs
+  int64_t lo, hi;   // this CTA's tile range
+  int b;            // sequence of the first unit
+  int64_t base_b;   // first tile of sequence b's units
+};
+
+// Computed by one full warp; every lane returns the same values.
+__device__ __forceinline__ SchedStart schedule_start(const VerifyParams& p, int cta, int grid) {
+  const int lane = threadIdx.x & 31;
+  const int HR = p.Hkv * p.row_groups;
+  int64_t W = 0;
+  for (int b = lane; b < p.B; b += 32) W += static_cast<int64_t>(tiles_of(clamp_context(p, b, false))) * HR;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+  SchedStart s;
+  s.W = W;
+  s.nC = static_cast<int>(W < grid ? W : grid);
+  s.lo = s.hi = 0;
+  s.b = 0;
+  s.base_b = 0;
+  if (cta >= s.nC) return s;
+  s.lo = static_cast<int64_t>(cta) * W / s.nC;
+  s.hi = static_cast<int64_t>(cta + 1) * W / s.nC;
+  // find the sequence whose unit range contains tile lo: scan in chunks of 32 sequences
+  int64_t run = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    int64_t mine = b < p.B ? static_cast<int64_t>(tiles_of(clamp_context(p, b, false))) * HR : 0;
+    int64_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int64_t excl = run + incl - mine;
+    const bool here = b < p.B && excl <= s.lo && s.lo < run + incl;
+    const uint32_t ball = __ballot_sync(0xffffffffu, here);
+    if (ball) {
+      const int src = __ffs(ball) - 1;
+      s.b = b0 + src;
+      s.base_b = __shfl_sync(0xffffffffu, excl, src);
+      return s;
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return s;  // not reached for lo < W
+}
+
+}  // namespace taco

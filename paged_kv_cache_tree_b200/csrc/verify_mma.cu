@@ -1,0 +1,52 @@
+// Instantiations and launcher of the mma.sync verify kernel.
+#include "launchers.h"
+#include "verify_mma.cuh"
+
+namespace taco {
+
+int mma_rows_per_unit(int packed_rows) {
+  if (packed_rows <= 16) return 16;
+  if (packed_rows <= 32) return 32;
+  return 64;
+}
+
+int mma_smem_bytes(int D, int rows_per_unit) {
+  const int mt = rows_per_unit / 16;
+  if (D == 128) {
+    return mt == 1 ? MmaCfg<128, 1>::kSmemBytes : mt == 2 ? MmaCfg<128, 2>::kSmemBytes : MmaCfg<128, 4>::kSmemBytes;
+  }
+  return mt == 1 ? MmaCfg<64, 1>::kSmemBytes : mt == 2 ? MmaCfg<64, 2>::kSmemBytes : MmaCfg<64, 4>::kSmemBytes;
+}
+
+template <typename T, int D, int MT>
+static cudaError_t launch_one(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p, int grid,
+                              cudaStream_t stream) {
+  using Cfg = MmaCfg<D, MT>;
+  auto kern = verify_mma_kernel<T, D, MT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tk, tv, p);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_typed(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p, int grid,
+                                cudaStream_t stream) {
+  const int mt = p.rows_per_unit / 16;
+  if (p.D == 128) {
+    if (mt == 1) return launch_one<T, 128, 1>(tk, tv, p, grid, stream);
+    if (mt == 2) return launch_one<T, 128, 2>(tk, tv, p, grid, stream);
+    return launch_one<T, 128, 4>(tk, tv, p, grid, stream);
+  }
+  if (mt == 1) return launch_one<T, 64, 1>(tk, tv, p, grid, stream);
+  if (mt == 2) return launch_one<T, 64, 2>(tk, tv, p, grid, stream);
+  return launch_one<T, 64, 4>(tk, tv, p, grid, stream);
+}
+
+cudaError_t launch_verify_mma(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p, int dtype,
+                              int grid, cudaStream_t stream) {
+  if (dtype == TACO_DTYPE_BF16) return launch_typed<__nv_bfloat16>(tk, tv, p, grid, stream);
+  return launch_typed<__half>(tk, tv, p, grid, stream);
+}
+
+}  // namespace taco

@@ -1,0 +1,513 @@
+// Verify kernel for narrow packed query tiles (G * C up to 64 rows per unit): the warp-level
+// mma.sync path.
+//
+// One CTA = 4 consumer warps + 1 producer warp, two CTAs per SM, persistent over a stream-K range of
+// key tiles (device_common.cuh). The producer warp walks the block table and streams each tile's
+// K and V chunks (one chunk = min(bs, 64) consecutive slots of one physical block and one KV head,
+// contiguous in the [NB, Hkv, bs, D] cache) into a ring of shared-memory stages with TMA, 128-byte
+// swizzled so that ldmatrix reads are conflict-free. Consumer warps own 16 packed query rows each
+// (rows r = i * G + h' of candidate i and head g*G + h') and, when fewer than 4 row tiles exist,
+// split the tile's keys between them; S = Q K^T and O += P V run on mma.sync m16n8k16 with fp32
+// accumulators, and the softmax is the flash-style online form in base 2 (fp32 running max / sum).
+// The tree mask only enters the tiles that reach the candidates' positions.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace taco {
+
+template <int D, int MT>
+struct MmaCfg {
+  static constexpr int kConsumerWarps = 4;
+  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+  static constexpr int KG = kConsumerWarps / MT;              // key groups
+  static constexpr int kKeysPerWarp = kTileKeys / KG;         // 16, 32 or 64
+  static constexpr int kRows = 16 * MT;                       // packed rows per unit
+  static constexpr int kPanels = D / 64;                      // 128-byte-wide column panels
+  static constexpr int kPanelBytes = kTileKeys * 128;
+  static constexpr int kTensorBytes = kPanels * kPanelBytes;  // one of K or V per stage
+  static constexpr int kStageBytes = 2 * kTensorBytes;
+  static constexpr int kStages = (D == 128) ? 3 : 6;
+  static constexpr int kScratchFloats = 16 * D + 64;          // cross-warp O and l
+  static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes +
+                                    kScratchFloats * 4 + 64 * 4 /*m publish*/ +
+                                    2 * kStages * 8 /*barriers*/ + 64 /*schedule*/;
+};
+
+struct SchedShared {
+  long long W, lo, hi, base_b;
+  int nC, b, merge_flag, abort_flag;
+};
+
+template <typename T, int D, int MT>
+__global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
+    verify_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                      const __grid_constant__ CUtensorMap tmap_v, const VerifyParams p) {
+  using Cfg = MmaCfg<D, MT>;
+  using Op = MmaOp<T>;
+  constexpr int KG = Cfg::KG;
+  constexpr int KW = Cfg::kKeysPerWarp;
+  constexpr int NT = KW / 8;          // 8-key n-tiles per warp and tile
+  constexpr int DT = D / 8;           // 8-wide d tiles of the output
+  constexpr int KSTEPS = D / 16;      // k steps of Q K^T
+  constexpr int ROWS = Cfg::kRows;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  float* scratch = reinterpret_cast<float*>(smem + Cfg::kStages * Cfg::kStageBytes);
+  float* scratch_l = scratch + 16 * D;
+  float* m_pub = scratch + Cfg::kScratchFloats;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(m_pub + 64);
+  uint64_t* empty_bar = full_bar + Cfg::kStages;
+  SchedShared* sched = reinterpret_cast<SchedShared*>(empty_bar + Cfg::kStages);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int HR = p.Hkv * p.row_groups;
+
+  if (tid == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(smem_addr(full_bar + s), 1);
+      mbar_init(smem_addr(empty_bar + s), Cfg::kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  if (warp == Cfg::kConsumerWarps) {
+    SchedStart s = schedule_start(p, blockIdx.x, gridDim.x);
+    if (lane == 0) {
+      sched->W = s.W;
+      sched->lo = s.lo;
+      sched->hi = s.hi;
+      sched->base_b = s.base_b;
+      sched->nC = s.nC;
+      sched->b = s.b;
+      sched->merge_flag = 0;
+      sched->abort_flag = 0;
+    }
+  }
+  __syncthreads();
+  const int64_t W = sched->W;
+  const int nC = sched->nC;
+  if (static_cast<int>(blockIdx.x) >= nC) return;
+  const int64_t lo = sched->lo, hi = sched->hi;
+  volatile int* abort_flag = &sched->abort_flag;
+
+  if (warp == Cfg::kConsumerWarps) {
+    // ------------------------------------------------------------------ producer warp
+    prefetch_tensormap(&tmap_k);
+    prefetch_tensormap(&tmap_v);
+    const uint64_t policy = policy_evict_first();
+    const int rpc = p.bs < kTileKeys ? p.bs : kTileKeys;   // rows per chunk
+    const int chunks_per_tile = kTileKeys / rpc;
+    const uint32_t chunk_bytes = static_cast<uint32_t>(rpc) * 128u;
+    int stage = 0;
+    uint32_t phase = 0;
+    int b = sched->b;
+    int64_t base_b = sched->base_b;
+    int L = clamp_context(p, b, true);
+    int Tb = tiles_of(L);
+    int64_t t = lo;
+    int j = static_cast<int>((t - base_b) / Tb);
+    int tile = static_cast<int>((t - base_b) % Tb);
+    while (t < hi) {
+      const int g = j / p.row_groups;
+      const int tend = static_cast<int>(Tb < tile + (hi - t) ? Tb : tile + (hi - t));
+      const int nblk = (L + p.bs - 1) / p.bs;
+      const int32_t* bt_row = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+      int win = -1000000;
+      int32_t win_val = -1;
+      for (int tl = tile; tl < tend; ++tl) {
+        const int key0 = tl * kTileKeys;
+        int nvalid = L > key0 ? (L - key0 + rpc - 1) / rpc : 0;
+        if (nvalid > chunks_per_tile) nvalid = chunks_per_tile;
+        // block ids of this tile's chunks (window of 32 logical blocks held one per lane)
+        const int lb_first = key0 / p.bs;
+        if (nvalid > 0 && (lb_first < win || (key0 + (nvalid - 1) * rpc) / p.bs >= win + 32)) {
+          win = lb_first;
+          const int lb = win + lane;
+          win_val = lb < nblk ? __ldg(bt_row + lb) : -1;
+        }
+        int my_lb = (key0 + lane * rpc) / p.bs;
+        int32_t blk = __shfl_sync(0xffffffffu, win_val, (my_lb - win) & 31);
+        bool ok = lane < nvalid;
+        if (ok && (blk < 0 || blk >= p.num_blocks)) {
+          atomicOr(p.error_word, TACO_DEVERR_BLOCK_ID);
+          ok = false;
+        }
+        const uint32_t okmask = __ballot_sync(0xffffffffu, ok);
+        const uint32_t bytes = __popc(okmask) * chunk_bytes * Cfg::kPanels * 2u;
+        bool go = true;
+        if (lane == 0) {
+          go = (*abort_flag == 0) && mbar_wait(smem_addr(empty_bar + stage), phase ^ 1u, p.error_word);
+          if (!go) *abort_flag = 1;
+          mbar_arrive_expect_tx(smem_addr(full_bar + stage), go ? bytes : 0u);
+        }
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (go && ok) {
+          const uint32_t kdst = smem_addr(stages + stage * Cfg::kStageBytes) + lane * chunk_bytes;
+          const uint32_t vdst = kdst + Cfg::kTensorBytes;
+          const int row = (blk * p.Hkv + g) * p.bs + (key0 + lane * rpc) % p.bs;
+          const uint32_t fb = smem_addr(full_bar + stage);
+#pragma unroll
+          for (int pn = 0; pn < Cfg::kPanels; ++pn) {
+            tma_load_2d(kdst + pn * Cfg::kPanelBytes, &tmap_k, fb, pn * 64, row, policy);
+            tma_load_2d(vdst + pn * Cfg::kPanelBytes, &tmap_v, fb, pn * 64, row, policy);
+          }
+        }
+        __syncwarp();
+        if (++stage == Cfg::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      t += tend - tile;
+      tile = 0;
+      if (++j == HR) {
+        j = 0;
+        base_b += static_cast<int64_t>(Tb) * HR;
+        if (++b < p.B) {
+          L = clamp_context(p, b, true);
+          Tb = tiles_of(L);
+        }
+      }
+    }
+    // make sure no copy of ours is still landing when the CTA exits
+    if (lane == 0) {
+      for (int s = 0; s < Cfg::kStages; ++s) {
+        // the most recent use of stage s completed phase (uses-1); waiting for its parity is
+        // immediate when it has landed (or when the stage was never used)
+        int uses_parity_phase = (s < stage) ? phase : (phase ^ 1u);
+        mbar_wait(smem_addr(full_bar + s), static_cast<uint32_t>(uses_parity_phase), p.error_word);
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------------- consumer warps
+  const int mt = warp % MT;
+  const int kg = warp / MT;
+  const int gq = lane >> 2;
+  const int tq = lane & 3;
+  int stage = 0;
+  uint32_t phase = 0;
+  int b = sched->b;
+  int64_t base_b = sched->base_b;
+  int L = clamp_context(p, b, false);
+  int Tb = tiles_of(L);
+  int64_t t = lo;
+  int j = static_cast<int>((t - base_b) / Tb);
+  int tile = static_cast<int>((t - base_b) % Tb);
+  bool first_segment = true;
+
+  while (t < hi) {
+    const int g = j / p.row_groups;
+    const int rg = j % p.row_groups;
+    const int tbegin = tile;
+    const int tend = static_cast<int>(Tb < tile + (hi - t) ? Tb : tile + (hi - t));
+    const int n = clamp_candidates(p, b, L, first_segment && warp == 0 && lane == 0 && tile == 0);
+    const int P = L - n;
+    const uint32_t nmask = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+
+    // this thread's two packed rows
+    int Rrow[2];
+    bool rvalid[2];
+    uint32_t mw[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      Rrow[h] = rg * ROWS + mt * 16 + gq + 8 * h;
+      rvalid[h] = Rrow[h] < p.G * n;
+      mw[h] = rvalid[h] ? (__ldg(p.tree_mask_bits + static_cast<int64_t>(b) * p.C + Rrow[h] / p.G) & nmask) : 0u;
+    }
+    // Q fragments (A operand of m16n8k16): rows gq / gq+8, columns 2*tq.. of each 16-wide k step
+    uint32_t qf[KSTEPS][4];
+    {
+      const uint32_t* qrow[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = Rrow[h] / p.G, hh = Rrow[h] % p.G;
+        qrow[h] = reinterpret_cast<const uint32_t*>(static_cast<const T*>(p.q) +
+                                                    ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D);
+      }
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        qf[kk][0] = rvalid[0] ? __ldg(qrow[0] + kk * 8 + tq) : 0u;
+        qf[kk][1] = rvalid[1] ? __ldg(qrow[1] + kk * 8 + tq) : 0u;
+        qf[kk][2] = rvalid[0] ? __ldg(qrow[0] + kk * 8 + 4 + tq) : 0u;
+        qf[kk][3] = rvalid[1] ? __ldg(qrow[1] + kk * 8 + 4 + tq) : 0u;
+      }
+    }
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    float o[DT][4];
+#pragma unroll
+    for (int dt = 0; dt < DT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+
+    for (int tl = tbegin; tl < tend; ++tl) {
+      const int key0 = tl * kTileKeys;
+      bool ready = false;
+      if (*abort_flag == 0) {
+        ready = mbar_wait(smem_addr(full_bar + stage), phase, p.error_word);
+        if (!ready) *abort_flag = 1;
+      }
+      const uint32_t kbase = smem_addr(stages + stage * Cfg::kStageBytes);
+      const uint32_t vbase = kbase + Cfg::kTensorBytes;
+      const int wkey0 = kg * KW;   // first tile-relative key of this warp
+      if (ready && key0 + kTileKeys > L) {
+        // keys >= L in this tile: their V rows may be stale or NaN-poisoned; zero this warp's
+        int zr0 = L - key0 - wkey0;
+        if (zr0 < 0) zr0 = 0;
+        uint8_t* vgen = stages + stage * Cfg::kStageBytes + Cfg::kTensorBytes;
+        for (int idx = lane; idx < (KW - zr0) * Cfg::kPanels * 8; idx += 32) {
+          const int r = wkey0 + zr0 + idx / (Cfg::kPanels * 8);
+          const int rem = idx % (Cfg::kPanels * 8);
+          *reinterpret_cast<uint4*>(vgen + (rem / 8) * Cfg::kPanelBytes + r * 128 + (rem % 8) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (ready) {
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+#pragma unroll
+          for (int np = 0; np < NT / 2; ++np) {
+            const int key = wkey0 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
+            const int d = kk * 16 + ((lane >> 3) & 1) * 8;
+            const int c = (d & 63) >> 3;
+            const uint32_t addr = kbase + (d >> 6) * Cfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(addr, b0, b1, b2, b3);
+            Op::run(s[2 * np], qf[kk], b0, b1);
+            Op::run(s[2 * np + 1], qf[kk], b2, b3);
+          }
+        }
+        // scale, mask, online softmax
+        const bool need_mask = key0 + kTileKeys > P;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v = s[nt][e] * p.scale_log2;
+            if (need_mask) {
+              const int key = key0 + wkey0 + nt * 8 + 2 * tq + (e & 1);
+              const int h = e >> 1;
+              bool vis = key < P || (key < L && ((mw[h] >> ((key - P) & 31)) & 1u));
+              v = vis ? v : -INFINITY;
+            }
+            s[nt][e] = v;
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mx = fmaxf(mx, fmaxf(s[nt][2 * h], s[nt][2 * h + 1]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          const float m_new = fmaxf(m_run[h], mx);
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+          const float alpha = fast_exp2(m_run[h] - m_use);
+          m_run[h] = m_new;
+          float rs = 0.f;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const float p0 = fast_exp2(s[nt][2 * h] - m_use);
+            const float p1 = fast_exp2(s[nt][2 * h + 1] - m_use);
+            s[nt][2 * h] = p0;
+            s[nt][2 * h + 1] = p1;
+            rs += p0 + p1;
+          }
+          l_run[h] = l_run[h] * alpha + rs;
+#pragma unroll
+          for (int dt = 0; dt < DT; ++dt) {
+            o[dt][2 * h] *= alpha;
+            o[dt][2 * h + 1] *= alpha;
+          }
+        }
+        // O += P V
+#pragma unroll
+        for (int ks = 0; ks < KW / 16; ++ks) {
+          uint32_t a[4];
+          a[0] = Op::pack(s[2 * ks][0], s[2 * ks][1]);
+          a[1] = Op::pack(s[2 * ks][2], s[2 * ks][3]);
+          a[2] = Op::pack(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+          a[3] = Op::pack(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+#pragma unroll
+          for (int dp = 0; dp < D / 16; ++dp) {
+            const int key = wkey0 + ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int d = dp * 16 + (lane >> 4) * 8;
+            const int c = (d & 63) >> 3;
+            const uint32_t addr = vbase + (d >> 6) * Cfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_trans(addr, b0, b1, b2, b3);
+            Op::run(o[2 * dp], a, b0, b1);
+            Op::run(o[2 * dp + 1], a, b2, b3);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(empty_bar + stage));
+      if (++stage == Cfg::kStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+
+    // ---------------------------------------------------------------- segment epilogue
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
+      l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
+    }
+    if constexpr (KG > 1) {
+      if (tq == 0) {
+        m_pub[warp * 16 + gq] = m_run[0];
+        m_pub[warp * 16 + gq + 8] = m_run[1];
+      }
+      named_bar_sync(1, 128);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float mstar = -INFINITY;
+#pragma unroll
+        for (int k2 = 0; k2 < KG; ++k2) mstar = fmaxf(mstar, m_pub[(mt + k2 * MT) * 16 + gq + 8 * h]);
+        const float f = (m_run[h] == -INFINITY) ? 0.f : fast_exp2(m_run[h] - mstar);
+        l_run[h] *= f;
+#pragma unroll
+        for (int dt = 0; dt < DT; ++dt) {
+          o[dt][2 * h] *= f;
+          o[dt][2 * h + 1] *= f;
+        }
+        m_run[h] = mstar;
+      }
+      // deterministic sequential sum of the key groups' partial O through one scratch tile
+      for (int mr = 0; mr < MT; ++mr) {
+        for (int kr = 0; kr < KG; ++kr) {
+          if (mt == mr && kg == kr) {
+            if (kr > 0) {
+#pragma unroll
+              for (int dt = 0; dt < DT; ++dt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[dt][e] += scratch[(dt * 4 + e) * 32 + lane];
+              l_run[0] += scratch_l[lane];
+              l_run[1] += scratch_l[32 + lane];
+            }
+            if (kr < KG - 1) {
+#pragma unroll
+              for (int dt = 0; dt < DT; ++dt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) scratch[(dt * 4 + e) * 32 + lane] = o[dt][e];
+              scratch_l[lane] = l_run[0];
+              scratch_l[32 + lane] = l_run[1];
+            }
+          }
+          named_bar_sync(1, 128);
+        }
+      }
+    }
+    const bool owner = (kg == KG - 1);
+    const bool whole_unit = (tbegin == 0 && tend == Tb);
+    const int64_t unit_base = base_b + static_cast<int64_t>(j) * Tb;
+    const int slot = 2 * static_cast<int>(blockIdx.x) + (first_segment ? 0 : 1);
+    if (owner) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int R = Rrow[h];
+        const float inv = l_run[h] > 0.f ? 1.f / l_run[h] : 0.f;
+        if (whole_unit) {
+          if (R < p.G * p.C) {
+            const int i = R / p.G, hh = R % p.G;
+            T* dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D;
+#pragma unroll
+            for (int dt = 0; dt < DT; ++dt)
+              *reinterpret_cast<uint32_t*>(dst + dt * 8 + 2 * tq) =
+                  rvalid[h] ? Op::pack(o[dt][2 * h] * inv, o[dt][2 * h + 1] * inv) : 0u;
+          }
+        } else {
+          const int r = mt * 16 + gq + 8 * h;
+          float* dst = p.part_o + (static_cast<int64_t>(slot) * ROWS + r) * D;
+#pragma unroll
+          for (int dt = 0; dt < DT; ++dt)
+            __stcg(reinterpret_cast<float2*>(dst + dt * 8 + 2 * tq),
+                   make_float2(o[dt][2 * h] * inv, o[dt][2 * h + 1] * inv));
+          if (tq == 0)
+            __stcg(p.part_lse + static_cast<int64_t>(slot) * ROWS + r,
+                   l_run[h] > 0.f ? m_run[h] + __log2f(l_run[h]) : -INFINITY);
+        }
+      }
+    }
+    if (!whole_unit) {
+      __threadfence();
+      named_bar_sync(1, 128);
+      const int c_first = cta_of_tile(unit_base, W, nC);
+      const int c_last = cta_of_tile(unit_base + Tb - 1, W, nC);
+      const int u = (b * p.Hkv + g) * p.row_groups + rg;
+      if (tid == 0) {
+        const uint32_t prev = atomicAdd(p.counters + u, 1u);
+        const bool last = prev == static_cast<uint32_t>(c_last - c_first);
+        if (last) {
+          p.counters[u] = 0u;
+          __threadfence();
+        }
+        sched->merge_flag = last ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      if (sched->merge_flag) {
+        // combine the unit's partials in CTA order: out = sum_s 2^(lse_s - max) O_s / sum_s 2^(...)
+        const int64_t lo_first = static_cast<int64_t>(c_first) * W / nC;
+        for (int r = warp; r < ROWS; r += 4) {
+          const int R = rg * ROWS + r;
+          if (R >= p.G * p.C) break;
+          const int i = R / p.G, hh = R % p.G;
+          T* dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D;
+          float acc[D / 32];
+#pragma unroll
+          for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+          float wsum = 0.f;
+          if (R < p.G * n) {
+            float lmax = -INFINITY;
+            for (int c = c_first; c <= c_last; ++c) {
+              const int sl = (c == c_first && lo_first < unit_base) ? 2 * c + 1 : 2 * c;
+              lmax = fmaxf(lmax, __ldcg(p.part_lse + static_cast<int64_t>(sl) * ROWS + r));
+            }
+            if (lmax != -INFINITY) {
+              for (int c = c_first; c <= c_last; ++c) {
+                const int sl = (c == c_first && lo_first < unit_base) ? 2 * c + 1 : 2 * c;
+                const float ls = __ldcg(p.part_lse + static_cast<int64_t>(sl) * ROWS + r);
+                const float wgt = ls == -INFINITY ? 0.f : exp2f(ls - lmax);
+                wsum += wgt;
+                const float* src = p.part_o + (static_cast<int64_t>(sl) * ROWS + r) * D + lane * (D / 32);
+#pragma unroll
+                for (int e = 0; e < D / 32; ++e) acc[e] += wgt * __ldcg(src + e);
+              }
+            }
+          }
+          const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+          for (int e = 0; e < D / 32; e += 2)
+            *reinterpret_cast<uint32_t*>(dst + lane * (D / 32) + e) = Op::pack(acc[e] * inv, acc[e + 1] * inv);
+        }
+      }
+      named_bar_sync(1, 128);
+    }
+
+    // next unit
+    first_segment = false;
+    t += tend - tile;
+    tile = 0;
+    if (++j == HR) {
+      j = 0;
+      base_b += static_cast<int64_t>(Tb) * HR;
+      if (++b < p.B) {
+        L = clamp_context(p, b, false);
+        Tb = tiles_of(L);
+      }
+    }
+  }
+}
+
+}  // namespace taco

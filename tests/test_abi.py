@@ -1,0 +1,92 @@
+"""The C-ABI library loads without a GPU, exports every symbol its header declares, and rejects bad
+arguments on the host before touching CUDA (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_tree_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "taco_attn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)) - {"defined", "if", "sizeof"})
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert "paged_tree_attention" in names and "paged_kv_append" in names
+    assert set(names) == set(_lib.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.taco_attn_version() == 1
+
+
+def _attn_args(**over):
+    a = dict(q=16, k=16, v=16, bt=16, ctx=16, nc=16, mask=16, scale=0.125, out=16, dtype=1, B=2, C=4,
+             Hq=8, Hkv=2, D=128, bs=16, NB=40, maxblk=8, stream=None)
+    a.update(over)
+    return [a["q"], a["k"], a["v"], a["bt"], a["ctx"], a["nc"], a["mask"], ctypes.c_float(a["scale"]), a["out"],
+            a["dtype"], a["B"], a["C"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["NB"], a["maxblk"], a["stream"]]
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(out=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(mask=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(dtype=7), _lib.TACO_ERR_INVALID_ARG),
+    (dict(D=96), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(bs=24), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(bs=4), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(C=33), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(C=0), _lib.TACO_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), _lib.TACO_ERR_INVALID_ARG),
+    (dict(B=-1), _lib.TACO_ERR_INVALID_ARG),
+    (dict(NB=0), _lib.TACO_ERR_INVALID_ARG),
+    (dict(maxblk=0), _lib.TACO_ERR_INVALID_ARG),
+    (dict(q=24), _lib.TACO_ERR_INVALID_ARG),        # not 16-byte aligned
+    (dict(scale=float("nan")), _lib.TACO_ERR_INVALID_ARG),
+])
+def test_attention_rejects_bad_arguments_on_host(lib, over, status):
+    assert lib.paged_tree_attention(*_attn_args(**over)) == status
+    assert lib.taco_attn_last_error().decode()
+
+
+def test_attention_empty_batch_is_a_no_op(lib):
+    assert lib.paged_tree_attention(*_attn_args(B=0)) == _lib.TACO_OK
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(kn=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(so=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(D=32), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(bs=1000), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(kc=8), _lib.TACO_ERR_INVALID_ARG),
+])
+def test_append_rejects_bad_arguments_on_host(lib, over, status):
+    a = dict(kn=16, vn=16, bt=16, so=16, kc=16, vc=16, dtype=0, B=2, C=4, Hkv=2, D=64, bs=16, NB=40,
+             maxblk=8, stream=None)
+    a.update(over)
+    args = [a["kn"], a["vn"], a["bt"], a["so"], a["kc"], a["vc"], a["dtype"], a["B"], a["C"], a["Hkv"], a["D"],
+            a["bs"], a["NB"], a["maxblk"], a["stream"]]
+    assert lib.paged_kv_append(*args) == status
+
+
+def test_options(lib):
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_GRID_CTAS, 7) == _lib.TACO_OK
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_GRID_CTAS, 0) == _lib.TACO_OK
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_KERNEL, 5) == _lib.TACO_ERR_INVALID_ARG
+    assert lib.taco_attn_set_option(99, 1) == _lib.TACO_ERR_INVALID_ARG
