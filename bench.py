@@ -1,0 +1,389 @@
+"""Benchmark of one verify step (paged KV-append of the candidates, then paged tree attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line on rank 0. A step is the whole hot path over one batch of seeded synthetic input:
+paged_kv_append writes every candidate's K/V into its cache slot, then paged_tree_attention attends
+all candidates over their paged prefixes. Inputs are resident in HBM when the timed region starts;
+the KV cache (0.6 - 1.5 GB) is larger than the 126 MB L2, so L2 is not flushed between steps.
+
+value        = algorithmic bytes of the step / device time per step, summed over ranks (GB/s):
+               attention reads K and V of every key once plus Q, writes O; append reads and writes
+               each appended K/V row.
+e2e          = the same metric through the public Python API with the step's per-call inputs
+               (q, k_new, v_new, tables, lengths, masks, slots) copied host->device from pinned memory
+               and the output copied back, every step; the KV cache is device-resident state.
+roofline     = the attention kernel alone: its algorithmic bytes / its mean launch time (CUDA events on
+               its stream) against the measured HBM copy bandwidth.
+cpu_baseline = the CPU oracle (fp64 NumPy) timed on a bounded sample of the same workload.
+
+With torchrun (N > 1) every rank runs an independent batch (its own seed) on its own GPU: the path
+needs no exchange between sequences, so there is no collective on the data path ("weak" scaling);
+the only collectives are a barrier and the max-over-ranks of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from paged_kv_cache_tree_b200 import workloads as wl  # noqa: E402
+
+METRIC = "paged tree-attn KV GB/s & % of B200 HBM peak; candidate-tokens/s vs CPU oracle"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DEFAULT_WORKLOAD = "decode"
+KERNEL_SOURCES = ("device_common.cuh", "verify_mma.cuh", "verify_mma.cu", "verify_tc.cuh", "verify_tc.cu")
+
+
+def time_at_roofline(bytes_moved: float, flops: float, bw_gbs: float, tflops: float):
+    """Seconds a step needs at a bandwidth (GB/s, 1e9) and a compute peak (TFLOP/s, 1e12): (io, compute)."""
+    return bytes_moved / (bw_gbs * 1e9), flops / (tflops * 1e12)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        p = os.path.join(ROOT, "paged_kv_cache_tree_b200", "csrc", name)
+        if os.path.exists(p):
+            with open(p, "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from a committed ncu summary, if it matches the current kernel."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("kernel_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={bus}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif args.impl == "ours":
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def step_bytes(w) -> int:
+    return w.kv_bytes() + w.qo_bytes() + w.append_bytes()
+
+
+# --------------------------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, budget_s: float):
+    """Time the oracle (append + attention) on the first sequences of ``w`` until about ``budget_s``.
+
+    Returns (bytes, candidate tokens, seconds, description) of the sample it ran.
+    """
+    import numpy as np
+
+    import oracle
+
+    bits = dict(q=wl.to_numpy_bits(w.q), kc=wl.to_numpy_bits(w.k_cache), vc=wl.to_numpy_bits(w.v_cache),
+                kn=wl.to_numpy_bits(w.k_new), vn=wl.to_numpy_bits(w.v_new))
+    masks = wl.as_uint32(w.tree_mask)
+    bt, ctx, nc, so = w.block_tables.numpy(), w.context_lens.numpy(), w.num_candidates.numpy(), w.slot_offsets.numpy()
+    done_b, spent, nbytes, ncand = 0, 0.0, 0, 0
+    for b in range(w.B):
+        sl = slice(b, b + 1)
+        t0 = time.perf_counter()
+        # the append oracle returns a new cache; give it a cache holding just this sequence's blocks
+        blocks = bt[b, : (int(ctx[b]) + w.bs - 1) // w.bs]
+        sub_bt = np.arange(len(blocks), dtype=np.int32)[None, :]
+        sub_k, sub_v = oracle.paged_kv_append(bits["kn"][sl], bits["vn"][sl], sub_bt, so[sl],
+                                              bits["kc"][blocks], bits["vc"][blocks])
+        oracle.paged_tree_attention(bits["q"][sl], sub_k, sub_v, sub_bt, ctx[sl], nc[sl], masks[sl], w.scale, w.dtype)
+        spent += time.perf_counter() - t0
+        done_b += 1
+        L = int(ctx[b])
+        nbytes += L * w.Hkv * w.D * 4 + 2 * w.C * w.Hq * w.D * 2 + 4 * int(nc[b]) * w.Hkv * w.D * 2
+        ncand += int(nc[b])
+        if spent >= budget_s:
+            break
+    return nbytes, ncand, spent, f"{done_b} of {w.B} sequences (all their KV heads and candidates), append + attention"
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [int(i.get("num_threads", 1)) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+# --------------------------------------------------------------------------------------------- arms
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = wl.make_workload(args.workload, seed=None, fill="zero")
+    # size each step so that warmup + steps fit in about 90 s of CPU time
+    per_step_budget = max(0.02, 90.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, per_step_budget)
+    tot_bytes, tot_cand, tot_s, desc = 0, 0, 0.0, ""
+    for _ in range(args.steps):
+        nb, ncnd, s, desc = oracle_sample(w, per_step_budget)
+        tot_bytes += nb
+        tot_cand += ncnd
+        tot_s += s
+    gbs = tot_bytes / tot_s / 1e9
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.WORKLOAD_DESCRIPTIONS[args.workload], "name": args.workload,
+                   "l2": "not applicable (host)"},
+        "candidate_tokens_per_s": tot_cand / tot_s,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {desc}"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def run_ours(args, world, rank, local):
+    import paged_kv_cache_tree_b200 as taco
+
+    taco.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    w = wl.make_workload(args.workload, seed=1000 + wl.WORKLOADS[args.workload]["k"] + 7919 * rank, fill="zero")
+    d = w.to(dev)
+    out = torch.empty_like(d.q)
+    stream = torch.cuda.current_stream(dev)
+    nbytes = step_bytes(w)
+    attn_bytes = w.kv_bytes() + w.qo_bytes()
+
+    def step(ev_pair=None):
+        taco.paged_kv_append(d.k_new, d.v_new, d.block_tables, d.slot_offsets, d.k_cache, d.v_cache, stream=stream)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        taco.paged_tree_attention(d.q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, d.num_candidates,
+                                  d.tree_mask, w.scale, out=out, stream=stream)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    taco.check_device(stream)
+
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(pairs[k])
+    t_stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    taco.check_device(stream)
+    region_ms = t_start.elapsed_time(t_stop)
+    attn_ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    region_ms = max_over_ranks(region_ms, world)
+    attn_ms = max_over_ranks(attn_ms, world)
+    ms_per_step = region_ms / args.steps
+    value = world * nbytes / (ms_per_step * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    host = {k: getattr(w, k).pin_memory() for k in ("q", "k_new", "v_new", "block_tables", "context_lens",
+                                                     "num_candidates", "tree_mask", "slot_offsets")}
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    out_host = torch.empty(w.q.shape, dtype=w.q.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        taco.paged_kv_append(dev_in["k_new"], dev_in["v_new"], dev_in["block_tables"], dev_in["slot_offsets"],
+                             d.k_cache, d.v_cache, stream=stream)
+        taco.paged_tree_attention(dev_in["q"], d.k_cache, d.v_cache, dev_in["block_tables"], dev_in["context_lens"],
+                                  dev_in["num_candidates"], dev_in["tree_mask"], w.scale, out=out, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    taco.check_device(stream)
+    e2e_value = world * nbytes / (e2e_ms * 1e-3) / 1e9
+
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peaks()
+    achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1) values, seeded block tables)",
+        "config": {"workload": wl.WORKLOAD_DESCRIPTIONS[args.workload], "name": args.workload,
+                   "step_bytes": nbytes, "attention_bytes": attn_bytes, "append_bytes": w.append_bytes(),
+                   "candidate_tokens_per_step": w.candidate_tokens(),
+                   "l2": "inputs larger than L2 (KV cache > 126 MB), no flush", "parallelism": f"dp{world} (independent batches)"},
+        "candidate_tokens_per_s": world * w.candidate_tokens() / (ms_per_step * 1e-3),
+        "hbm_frac_of_measured": value / world / peak,
+        "hbm_frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
+                     "kernel": "paged_tree_attention", "peak_source": f"{peak_kind} hbm_gbs",
+                     "launch_ms": attn_ms},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        nb, ncnd, secs, desc = oracle_sample(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{desc}; {secs:.1f} s", "candidate_tokens_per_s": ncnd / secs}
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+        else:
+            line = run_ours(args, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
