@@ -109,6 +109,34 @@ taco_status paged_kv_append(const void* k_new, const void* v_new, const int32_t*
                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                             int32_t num_blocks, int32_t max_blocks_per_seq, void* stream);
 
+/*
+ * paged_tree_attention_noalloc: the same operation, arguments and results as paged_tree_attention,
+ * for callers that cannot allocate device memory. The pages have no counterpart of this entry point;
+ * it exists because paged_tree_attention grows a workspace with cudaMalloc on first use, which a
+ * caller cannot allow when it runs under a fixed memory-pool budget (e.g. a server that has handed
+ * all free HBM to its KV cache), when an implicit device synchronisation mid-step is not acceptable,
+ * or when allocation after start-up is forbidden.
+ *   - Scratch: a fixed 8 MiB array inside the library's device image (every GPU that loads the
+ *     library holds it until exit); no cudaMalloc, cudaFree or other allocating call is made.
+ *   - Limit: at most 65536 work units (batch * num_kv_heads * row groups of up to 64 packed query
+ *     rows); larger calls return TACO_ERR_UNSUPPORTED with a message and enqueue nothing. The grid is
+ *     capped so that the split-KV partials fit the scratch.
+ *   - All calls on a device share the array and it keeps the last call's contents; each call clears
+ *     what must start at zero on `stream` first. Calls whose work overlaps on the GPU race: order them
+ *     on one stream.
+ *   - The first call on a device looks up the array's address (cudaGetSymbolAddress, that device
+ *     current); make it before any stream capture.
+ *   - Device-side range violations are skipped but are not visible to taco_attn_check_device.
+ */
+taco_status paged_tree_attention_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_tables, const int32_t* context_lens,
+                                         const int32_t* num_candidates, const uint32_t* tree_mask_bits,
+                                         float scale, void* out,
+                                         int32_t dtype, int32_t batch, int32_t max_candidates,
+                                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                         void* stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char* taco_attn_last_error(void);
 

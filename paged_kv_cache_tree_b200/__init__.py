@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     load,
     paged_kv_append,
     paged_tree_attention,
+    paged_tree_attention_noalloc,
     release_workspace,
     set_option,
     version,

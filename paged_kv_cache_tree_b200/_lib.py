@@ -31,6 +31,7 @@ TACO_OPT_KERNEL = 2
 EXPORTED = (
     "paged_tree_attention",
     "paged_kv_append",
+    "paged_tree_attention_noalloc",
     "taco_attn_last_error",
     "taco_attn_check_device",
     "taco_attn_release_workspace",
@@ -58,6 +59,8 @@ def load() -> ctypes.CDLL:
     vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
     lib.paged_tree_attention.argtypes = [vp] * 7 + [f32, vp] + [i32] * 9 + [vp]
     lib.paged_tree_attention.restype = i32
+    lib.paged_tree_attention_noalloc.argtypes = [vp] * 7 + [f32, vp] + [i32] * 9 + [vp]
+    lib.paged_tree_attention_noalloc.restype = i32
     lib.paged_kv_append.argtypes = [vp] * 6 + [i32] * 8 + [vp]
     lib.paged_kv_append.restype = i32
     lib.taco_attn_last_error.argtypes = []
@@ -105,7 +108,8 @@ def _need_cuda(name: str, t: torch.Tensor, dtype=None, ndim=None) -> None:
 
 
 def paged_tree_attention(q, k_cache, v_cache, block_tables, context_lens, num_candidates, tree_mask_bits,
-                         scale: float, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                         scale: float, out: Optional[torch.Tensor] = None, stream=None,
+                         _entry: str = "paged_tree_attention") -> torch.Tensor:
     """q [B,C,Hq,D]; k/v_cache [NB,Hkv,bs,D]; block_tables int32 [B,maxblk]; context_lens and
     num_candidates int32 [B]; tree_mask_bits int32/uint32 [B,C] (bit patterns). Returns ``out``."""
     _need_cuda("q", q, (torch.bfloat16, torch.float16), 4)
@@ -129,12 +133,21 @@ def paged_tree_attention(q, k_cache, v_cache, block_tables, context_lens, num_ca
     if tuple(out.shape) != tuple(q.shape):
         raise ValueError("out must have q's shape")
     lib = load()
-    _check(lib.paged_tree_attention(
+    _check(getattr(lib, _entry)(
         q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), context_lens.data_ptr(),
         num_candidates.data_ptr(), tree_mask_bits.data_ptr(), float(scale), out.data_ptr(),
         _dtype_code(q), B, C, Hq, Hkv, D, bs, NB, block_tables.shape[1],
         _stream_handle(stream, q.device)))
     return out
+
+
+def paged_tree_attention_noalloc(q, k_cache, v_cache, block_tables, context_lens, num_candidates,
+                                 tree_mask_bits, scale: float, out: Optional[torch.Tensor] = None,
+                                 stream=None) -> torch.Tensor:
+    """Same as paged_tree_attention, through the entry point that allocates no device memory (its
+    scratch is a fixed array in the library; see include/taco_attn.h for its limits)."""
+    return paged_tree_attention(q, k_cache, v_cache, block_tables, context_lens, num_candidates, tree_mask_bits,
+                                scale, out=out, stream=stream, _entry="paged_tree_attention_noalloc")
 
 
 def paged_kv_append(k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, stream=None) -> None:

@@ -156,6 +156,10 @@ taco_status check_common(int32_t dtype, int32_t batch, int32_t max_candidates, i
 
 }  // namespace
 
+namespace taco {
+void set_last_error_message(const char* msg) { g_last_error = msg; }
+}  // namespace taco
+
 extern "C" {
 
 int32_t taco_attn_version(void) { return kAbiVersion; }

@@ -29,5 +29,7 @@ int mma_smem_bytes(int D, int rows_per_unit);
 cudaError_t launch_verify_mma(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p,
                               int dtype, int grid, cudaStream_t stream);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+// Store the message taco_attn_last_error() returns on this thread.
+void set_last_error_message(const char* msg);
 
 }  // namespace taco
