@@ -5,6 +5,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -131,6 +132,23 @@ taco_status make_cache_map(CUtensorMap* map, const void* base, int dtype, int D,
   return TACO_OK;
 }
 
+// Query tile view [B*C, Hq, D]; box = 64 columns x G heads x cands_per_group candidates, so one box
+// holds the packed rows r = i * G + h' of one (sequence, KV head, row group).
+taco_status make_query_map(CUtensorMap* map, const void* q, int dtype, int D, int Hq, int64_t bc, int G,
+                           int cands_per_group) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(bc)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hq) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(cands_per_group)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, dtype == TACO_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   3, const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", static_cast<int>(r));
+  return TACO_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -206,31 +224,52 @@ taco_status paged_tree_attention(const void* q, const void* k_cache, const void*
 
   const int G = num_q_heads / num_kv_heads;
   const int packed = G * max_candidates;
-  const int rows = taco::mma_rows_per_unit(packed);
-  const int row_groups = (packed + rows - 1) / rows;
-  const int64_t units = static_cast<int64_t>(batch) * num_kv_heads * row_groups;
 
   std::lock_guard<std::mutex> lk(g_mu);
-  int grid = static_cast<int>(g_opt_grid);
-  if (grid == 0) {
-    if (g_ws[dev].sm_count == 0) {
-      e = cudaDeviceGetAttribute(&g_ws[dev].sm_count, cudaDevAttrMultiProcessorCount, dev);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-    }
-    grid = 2 * g_ws[dev].sm_count;
+  // kernel choice: the tcgen05 path once the packed (GQA group x candidates) tile is wide enough to
+  // keep tensor cores busy; the mma.sync path for narrow tiles
+  const bool tc_possible = G <= 128;
+  bool use_tc = tc_possible && packed >= 48;
+  if (g_opt_kernel == 1) use_tc = false;
+  if (g_opt_kernel == 2) {
+    if (!tc_possible) return fail(TACO_ERR_UNSUPPORTED, "tensor-core path needs num_q_heads / num_kv_heads <= 128");
+    use_tc = true;
   }
+  int rows, row_groups, cands_per_group = 0;
+  if (use_tc) {
+    cands_per_group = std::min(max_candidates, 128 / G);
+    row_groups = (max_candidates + cands_per_group - 1) / cands_per_group;
+    rows = 128;
+  } else {
+    rows = taco::mma_rows_per_unit(packed);
+    row_groups = (packed + rows - 1) / rows;
+  }
+  const int64_t units = static_cast<int64_t>(batch) * num_kv_heads * row_groups;
+
+  if (g_ws[dev].sm_count == 0) {
+    e = cudaDeviceGetAttribute(&g_ws[dev].sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  }
+  int grid = static_cast<int>(g_opt_grid);
+  if (grid == 0) grid = (use_tc ? 1 : 2) * g_ws[dev].sm_count;
   const size_t slots = 2 * static_cast<size_t>(grid);
   st = ensure_workspace(dev, static_cast<size_t>(units), slots * rows, slots * rows * head_dim);
   if (st != TACO_OK) return st;
   Workspace& w = g_ws[dev];
 
-  const int rpc = block_size < taco::kTileKeys ? block_size : taco::kTileKeys;
+  const int tile = use_tc ? taco::tc_tile_keys() : taco::kTileKeys;
+  const int rpc = block_size < tile ? block_size : tile;
   const int64_t cache_rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tq;
   st = make_cache_map(&tk, k_cache, dtype, head_dim, cache_rows, rpc);
   if (st != TACO_OK) return st;
   st = make_cache_map(&tv, v_cache, dtype, head_dim, cache_rows, rpc);
   if (st != TACO_OK) return st;
+  if (use_tc) {
+    st = make_query_map(&tq, q, dtype, head_dim, num_q_heads, static_cast<int64_t>(batch) * max_candidates, G,
+                        cands_per_group);
+    if (st != TACO_OK) return st;
+  }
 
   taco::VerifyParams p{};
   p.q = q;
@@ -255,7 +294,14 @@ taco_status paged_tree_attention(const void* q, const void* k_cache, const void*
   p.max_blocks = max_blocks_per_seq;
   p.rows_per_unit = rows;
   p.row_groups = row_groups;
+  p.cands_per_group = cands_per_group;
+  p.tile_keys = use_tc ? taco::tc_tile_keys() : taco::kTileKeys;
 
+  if (use_tc) {
+    e = taco::launch_verify_tc(tk, tv, tq, p, dtype, grid, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "verify kernel launch");
+    return TACO_OK;
+  }
   e = taco::launch_verify_mma(tk, tv, p, dtype, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "verify kernel launch");
   return TACO_OK;

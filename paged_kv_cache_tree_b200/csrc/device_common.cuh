@@ -29,7 +29,9 @@ struct VerifyParams {
   float scale_log2;      // scale * log2(e)
   int B, C, Hq, Hkv, G, D, bs, num_blocks, max_blocks;
   int rows_per_unit;     // packed query rows handled by one unit (row group)
-  int row_groups;        // ceil(G * C / rows_per_unit)
+  int row_groups;        // number of row groups per (sequence, KV head)
+  int cands_per_group;   // tensor-core path: candidates per row group (rows = cands_per_group * G)
+  int tile_keys;         // keys per work tile of the kernel (64 or 128)
 };
 
 // ---------------------------------------------------------------------------------------------
@@ -70,6 +72,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
       : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Non-blocking test of phase completion.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Test for phase completion, suspending up to about `hint_ns` if it is not complete yet.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return done != 0;
 }
@@ -174,7 +202,7 @@ struct MmaOp<__half> {
 // split-KV work schedule ("stream-K" over key tiles)
 //
 // Work unit u = (b, kv head g, row group rg), ordered u = (b * Hkv + g) * RG + rg. Unit u holds
-// T_b = max(1, ceil(L_b / kTileKeys)) key tiles (an empty sequence still gets one tile, which
+// T_b = max(1, ceil(L_b / tile_keys)) key tiles (an empty sequence still gets one tile, which
 // writes its zero rows). All units' tiles are concatenated into one range [0, W); CTA c of the nC
 // working CTAs takes tiles [c*W/nC, (c+1)*W/nC). A unit that falls into several CTAs' ranges is
 // split: each piece writes a partial (normalised output + log-sum-exp), and the CTA that arrives
@@ -201,7 +229,7 @@ __device__ __forceinline__ int clamp_candidates(const VerifyParams& p, int b, in
   return n;
 }
 
-__device__ __forceinline__ int tiles_of(int L) { return L <= 0 ? 1 : (L + kTileKeys - 1) / kTileKeys; }
+__device__ __forceinline__ int tiles_of(int L, int tile) { return L <= 0 ? 1 : (L + tile - 1) / tile; }
 
 // first CTA (of nC over W tiles) whose range contains tile t
 __device__ __forceinline__ int cta_of_tile(int64_t t, int64_t W, int64_t nC) {
@@ -221,7 +249,7 @@ __device__ __forceinline__ SchedStart schedule_start(const VerifyParams& p, int 
   const int lane = threadIdx.x & 31;
   const int HR = p.Hkv * p.row_groups;
   int64_t W = 0;
-  for (int b = lane; b < p.B; b += 32) W += static_cast<int64_t>(tiles_of(clamp_context(p, b, false))) * HR;
+  for (int b = lane; b < p.B; b += 32) W += static_cast<int64_t>(tiles_of(clamp_context(p, b, false), p.tile_keys)) * HR;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
   SchedStart s;
@@ -237,7 +265,7 @@ __device__ __forceinline__ SchedStart schedule_start(const VerifyParams& p, int 
   int64_t run = 0;
   for (int b0 = 0; b0 < p.B; b0 += 32) {
     const int b = b0 + lane;
-    int64_t mine = b < p.B ? static_cast<int64_t>(tiles_of(clamp_context(p, b, false))) * HR : 0;
+    int64_t mine = b < p.B ? static_cast<int64_t>(tiles_of(clamp_context(p, b, false), p.tile_keys)) * HR : 0;
     int64_t incl = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -257,5 +285,88 @@ __device__ __forceinline__ SchedStart schedule_start(const VerifyParams& p, int 
   }
   return s;  // not reached for lo < W
 }
+
+// Walks one CTA's work as segments: a segment is the part of one unit (b, j = g * RG + rg) that
+// falls into the CTA's tile range; tiles [tile, seg_end()) of the unit.
+struct SegCursor {
+  int b;
+  int64_t base_b;  // first global tile of sequence b's units
+  int L, Tb, j, tile;
+  int64_t t, hi;
+  int HR;
+  int ui;          // segment ordinal within the CTA
+
+  __device__ __forceinline__ void init(const VerifyParams& p, int b0, int64_t base_b0, int64_t lo, int64_t hi_,
+                                       bool report) {
+    b = b0;
+    base_b = base_b0;
+    HR = p.Hkv * p.row_groups;
+    L = clamp_context(p, b, report);
+    Tb = tiles_of(L, p.tile_keys);
+    t = lo;
+    hi = hi_;
+    j = static_cast<int>((t - base_b) / Tb);
+    tile = static_cast<int>((t - base_b) % Tb);
+    ui = 0;
+  }
+  __device__ __forceinline__ bool valid() const { return t < hi; }
+  __device__ __forceinline__ int seg_end() const {
+    return static_cast<int>(Tb < tile + (hi - t) ? Tb : tile + (hi - t));
+  }
+  __device__ __forceinline__ int64_t unit_base() const { return base_b + static_cast<int64_t>(j) * Tb; }
+  __device__ __forceinline__ void next_segment(const VerifyParams& p, bool report) {
+    t += seg_end() - tile;
+    tile = 0;
+    ++ui;
+    if (++j == HR) {
+      j = 0;
+      base_b += static_cast<int64_t>(Tb) * HR;
+      if (++b < p.B) {
+        L = clamp_context(p, b, report);
+        Tb = tiles_of(L, p.tile_keys);
+      }
+    }
+  }
+};
+
+struct TileInfo {
+  int ui;      // segment ordinal within the CTA
+  int tl;      // tile index within the unit
+  int jl;      // tile index within the segment
+  bool first;  // first tile of its segment
+  bool last;   // last tile of its segment
+};
+
+// Tile-by-tile walk over the same sequence of segments.
+struct TileWalker {
+  SegCursor c;
+  int tl, tend;
+  bool have;
+  __device__ __forceinline__ void init(const VerifyParams& p, int b0, int64_t base_b0, int64_t lo, int64_t hi) {
+    c.init(p, b0, base_b0, lo, hi, false);
+    have = c.valid();
+    if (have) {
+      tl = c.tile;
+      tend = c.seg_end();
+    }
+  }
+  __device__ __forceinline__ bool next(const VerifyParams& p, TileInfo& ti) {
+    if (!have) return false;
+    ti.ui = c.ui;
+    ti.tl = tl;
+    ti.jl = tl - c.tile;
+    ti.first = (tl == c.tile);
+    ti.last = (tl == tend - 1);
+    if (++tl == tend) {
+      c.next_segment(p, false);
+      have = c.valid();
+      if (have) {
+        tl = c.tile;
+        tend = c.seg_end();
+      }
+    }
+    return true;
+  }
+};
 
 }  // namespace taco

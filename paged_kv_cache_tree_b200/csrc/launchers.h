@@ -29,6 +29,12 @@ int mma_smem_bytes(int D, int rows_per_unit);
 cudaError_t launch_verify_mma(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p,
                               int dtype, int grid, cudaStream_t stream);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+// Keys per work tile of the tcgen05 verify kernel.
+int tc_tile_keys();
+// Dynamic shared memory of the tcgen05 verify kernel.
+int tc_smem_bytes(int D);
+cudaError_t launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                             const VerifyParams& p, int dtype, int grid, cudaStream_t stream);
 // Store the message taco_attn_last_error() returns on this thread.
 void set_last_error_message(const char* msg);
 

@@ -191,6 +191,7 @@ extern "C" taco_status paged_tree_attention_noalloc(
   p.max_blocks = max_blocks_per_seq;
   p.rows_per_unit = rows;
   p.row_groups = row_groups;
+  p.tile_keys = taco::kTileKeys;
   e = taco::launch_verify_mma(maps[0], maps[1], p, dtype, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "verify kernel launch: %s", cudaGetErrorString(e));
   return TACO_OK;

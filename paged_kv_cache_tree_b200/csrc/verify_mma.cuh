@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     int b = sched->b;
     int64_t base_b = sched->base_b;
     int L = clamp_context(p, b, true);
-    int Tb = tiles_of(L);
+    int Tb = tiles_of(L, kTileKeys);
     int64_t t = lo;
     int j = static_cast<int>((t - base_b) / Tb);
     int tile = static_cast<int>((t - base_b) % Tb);
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
         base_b += static_cast<int64_t>(Tb) * HR;
         if (++b < p.B) {
           L = clamp_context(p, b, true);
-          Tb = tiles_of(L);
+          Tb = tiles_of(L, kTileKeys);
         }
       }
     }
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
   int b = sched->b;
   int64_t base_b = sched->base_b;
   int L = clamp_context(p, b, false);
-  int Tb = tiles_of(L);
+  int Tb = tiles_of(L, kTileKeys);
   int64_t t = lo;
   int j = static_cast<int>((t - base_b) / Tb);
   int tile = static_cast<int>((t - base_b) % Tb);
@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
       base_b += static_cast<int64_t>(Tb) * HR;
       if (++b < p.B) {
         L = clamp_context(p, b, false);
-        Tb = tiles_of(L);
+        Tb = tiles_of(L, kTileKeys);
       }
     }
   }

@@ -1,0 +1,678 @@
+// Verify kernel for wide packed query tiles (G * C >= 48 rows): the tcgen05 / tensor-memory path.
+//
+// The candidates of one (sequence, KV head) form up to 128 query rows (r = i_local * G + h'), the
+// M = 128 operand of tcgen05.mma; this is how several candidates turn the decode GEMV into a GEMM
+// ("大模型倍速推理引擎 TACO-LLM 的设计与实践", TurboAttention bullets under "整体方案分为两大部分").
+// One CTA per SM, persistent over the same stream-K tile ranges as the mma.sync path:
+//   warps 0, 10 producers: TMA loads of each segment's Q tile (3-D box over [B*C, Hq, D]) and of
+//               every 64-key tile's K chunks (warp 0) and V chunks (warp 10) reached through the block
+//               table, into separate K and V rings (K is released as soon as its Q K^T is done, V
+//               after its P V);
+//   warp 1      MMA issuer (one thread): S = Q K^T into one of four tensor-memory S buffers
+//               (64 fp32 columns each), up to three tiles ahead; O += P V with P read back from
+//               tensor memory (A operand) and V from shared memory (MN-major B operand);
+//   warps 2..9  two softmax warpgroups; tile k belongs to warpgroup k % 2, which owns its own O
+//               accumulator in tensor memory. Thread r of a warpgroup owns query row r (lane r):
+//               base-2 online softmax in fp32 whose reference max only moves when a row's max grows
+//               by more than 2^8 (so O is rescaled rarely), P written back as bf16/fp16 pairs into
+//               the S buffer. At the end of a segment warpgroup 0 merges the two accumulators
+//               (log-sum-exp weights) and normalises, or writes a split-KV partial.
+// MMA completion is signalled with tcgen05.commit on mbarriers; every wait is bounded.
+#pragma once
+
+#include <type_traits>
+
+#include "device_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace taco {
+
+constexpr int kTcTileKeys = 64;   // keys per work tile of this kernel (QK^T is M=128 x N=64)
+
+template <int D>
+struct TcCfg {
+  static constexpr int kThreads = 352;
+  static constexpr int kTK = kTcTileKeys;
+  static constexpr int kPanels = D / 64;
+  static constexpr int kPanelBytes = kTK * 128;            // kTK keys x 128 bytes
+  static constexpr int kTensorBytes = kPanels * kPanelBytes;
+  static constexpr int kKStages = (D == 128) ? 4 : 8;
+  static constexpr int kVStages = (D == 128) ? 7 : 14;
+  static constexpr int kQPanelBytes = 128 * 128;           // 128 rows x 128 bytes
+  static constexpr int kQBytes = kPanels * kQPanelBytes;
+  static constexpr int kSBufs = 4;                         // S/P buffers of kTK columns at 0, 64, 128, 192
+  static constexpr int kTmemCols = 512;
+  static constexpr int kOCol = 256;                        // O of warpgroup w at kOCol + w * 128
+  static constexpr int kSharedBytes = 4096;
+  static constexpr int kSmemBytes =
+      1024 + (kKStages + kVStages) * kTensorBytes + kQBytes + kSharedBytes;
+};
+
+struct TcShared {
+  uint64_t k_full[8], k_empty[8], v_full[14], v_empty[14];
+  uint64_t q_full, q_empty, s_full[4], p_full[4], pv_done[4], o_free;
+  uint32_t tmem_base;
+  int merge_flag, abort_flag;
+  long long W, lo, hi, base_b;
+  int nC, b;
+  float xm[2][128];  // warpgroup 1's reference max per row, double-buffered by segment
+  float xl[2][128];  // warpgroup 1's running sum per row
+};
+
+// 3-D TMA tile load (Q tile: x = column, y = head, z = sequence * C + candidate).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int32_t x,
+                                            int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(352, 1)
+    verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                     const __grid_constant__ CUtensorMap tmap_q, const VerifyParams p) {
+  using Cfg = TcCfg<D>;
+  using Op = MmaOp<T>;
+  constexpr int SK = Cfg::kKStages;
+  constexpr int SV = Cfg::kVStages;
+  constexpr int NS = Cfg::kSBufs;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  constexpr int TK = Cfg::kTK;
+  constexpr uint32_t kIdescQK = tc::idesc_f16(kBf16 ? 1 : 0, 128, TK, 0);
+  constexpr uint32_t kIdescPV = tc::idesc_f16(kBf16 ? 1 : 0, 128, D, 1);
+  static_assert(sizeof(TcShared) <= Cfg::kSharedBytes, "shared bookkeeping too large");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* kring = smem;
+  uint8_t* vring = kring + SK * Cfg::kTensorBytes;
+  uint8_t* qbuf = vring + SV * Cfg::kTensorBytes;
+  TcShared* sh = reinterpret_cast<TcShared*>(qbuf + Cfg::kQBytes);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  if (tid == 0) {
+    for (int s = 0; s < SK; ++s) {
+      mbar_init(smem_addr(&sh->k_full[s]), 1);
+      mbar_init(smem_addr(&sh->k_empty[s]), 1);
+    }
+    for (int s = 0; s < SV; ++s) {
+      mbar_init(smem_addr(&sh->v_full[s]), 1);
+      mbar_init(smem_addr(&sh->v_empty[s]), 1);
+    }
+    mbar_init(smem_addr(&sh->q_full), 1);
+    mbar_init(smem_addr(&sh->q_empty), 1);
+    for (int j = 0; j < NS; ++j) {
+      mbar_init(smem_addr(&sh->s_full[j]), 1);
+      mbar_init(smem_addr(&sh->p_full[j]), 4);
+      mbar_init(smem_addr(&sh->pv_done[j]), 1);
+    }
+    mbar_init(smem_addr(&sh->o_free), 4);
+    sh->merge_flag = 0;
+    sh->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_addr(&sh->tmem_base), Cfg::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (warp == 0) {
+    SchedStart s0 = schedule_start(p, blockIdx.x, gridDim.x);
+    if (lane == 0) {
+      sh->W = s0.W;
+      sh->lo = s0.lo;
+      sh->hi = s0.hi;
+      sh->base_b = s0.base_b;
+      sh->nC = s0.nC;
+      sh->b = s0.b;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = sh->tmem_base;
+  const int64_t W = sh->W;
+  const int nC = sh->nC;
+  if (static_cast<int>(blockIdx.x) >= nC) {
+    if (warp == 1) tc::tmem_dealloc(tmem, Cfg::kTmemCols);
+    return;
+  }
+  const int64_t lo = sh->lo, hi = sh->hi;
+  volatile int* abort_flag = &sh->abort_flag;
+  const int cpg = p.cands_per_group;
+  const int qrows = cpg * p.G;
+
+  if (warp == 0 || warp == 10) {
+    // ------------------------------------------------------------------ producers
+    // warp 0 streams Q and K, warp 10 streams V: both walk the same tiles and block table, so each
+    // pays only its own share of the per-copy issue cost
+    const bool is_k = (warp == 0);
+    prefetch_tensormap(is_k ? &tmap_k : &tmap_v);
+    if (is_k) prefetch_tensormap(&tmap_q);
+    const uint64_t policy = policy_evict_first();
+    const int rpc = p.bs < TK ? p.bs : TK;
+    const int chunks_per_tile = TK / rpc;
+    const uint32_t chunk_bytes = static_cast<uint32_t>(rpc) * 128u;
+    const uint32_t q_bytes = static_cast<uint32_t>(Cfg::kPanels * qrows * 128);
+    SegCursor cur;
+    cur.init(p, sh->b, sh->base_b, lo, hi, true);
+    int64_t k = 0;  // tile ordinal within the CTA
+    while (cur.valid()) {
+      const int g = cur.j / p.row_groups;
+      const int rg = cur.j % p.row_groups;
+      const int tend = cur.seg_end();
+      const int L = cur.L;
+      const int nblk = (L + p.bs - 1) / p.bs;
+      const int32_t* bt_row = p.block_tables + static_cast<int64_t>(cur.b) * p.max_blocks;
+      int win = -1000000;
+      int32_t win_val = -1;
+      // The segment's Q tile goes into the single Q buffer once the previous segment's last Q K^T
+      // is done. K/V tiles of this segment may be issued first, but not more than SK - 1 of them:
+      // from the SK-th on, a K slot's previous user belongs to this segment and needs its Q.
+      bool q_issued = false;
+      const int q_deadline = (tend - cur.tile - 1) < (SK - 2) ? (tend - cur.tile - 1) : (SK - 2);
+      const uint32_t q_parity_prev = static_cast<uint32_t>((cur.ui & 1) ^ 1);
+      for (int tl = cur.tile; tl < tend; ++tl, ++k) {
+        if (!is_k) q_issued = true;
+        if (!q_issued && lane == 0) {
+          bool ready = (*abort_flag != 0) || mbar_test(smem_addr(&sh->q_empty), q_parity_prev);
+          if (!ready && tl - cur.tile >= q_deadline) {
+            ready = true;
+            if (!mbar_wait(smem_addr(&sh->q_empty), q_parity_prev, p.error_word)) *abort_flag = 1;
+          }
+          if (ready) {
+            const bool go = (*abort_flag == 0);
+            mbar_arrive_expect_tx(smem_addr(&sh->q_full), go ? q_bytes : 0u);
+            if (go) {
+#pragma unroll
+              for (int pn = 0; pn < Cfg::kPanels; ++pn)
+                tma_load_3d(smem_addr(qbuf) + pn * Cfg::kQPanelBytes, &tmap_q, smem_addr(&sh->q_full), pn * 64,
+                            g * p.G, cur.b * p.C + rg * cpg);
+            }
+            q_issued = true;
+          }
+        }
+        q_issued = __shfl_sync(0xffffffffu, q_issued, 0);
+        const int key0 = tl * TK;
+        int nvalid = L > key0 ? (L - key0 + rpc - 1) / rpc : 0;
+        if (nvalid > chunks_per_tile) nvalid = chunks_per_tile;
+        const int lb_first = key0 / p.bs;
+        if (nvalid > 0 && (lb_first < win || (key0 + (nvalid - 1) * rpc) / p.bs >= win + 32)) {
+          win = lb_first;
+          const int lb = win + lane;
+          win_val = lb < nblk ? __ldg(bt_row + lb) : -1;
+        }
+        const int my_lb = (key0 + lane * rpc) / p.bs;
+        const int32_t blk = __shfl_sync(0xffffffffu, win_val, (my_lb - win) & 31);
+        bool ok = lane < nvalid;
+        if (ok && (blk < 0 || blk >= p.num_blocks)) {
+          atomicOr(p.error_word, TACO_DEVERR_BLOCK_ID);
+          ok = false;
+        }
+        const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, ok)) * chunk_bytes * Cfg::kPanels;
+        const int row = (blk * p.Hkv + g) * p.bs + (key0 + lane * rpc) % p.bs;
+        if (is_k) {  // K
+          const int st = static_cast<int>(k % SK);
+          bool go = true;
+          if (lane == 0) {
+            go = (*abort_flag == 0) &&
+                 mbar_wait(smem_addr(&sh->k_empty[st]), static_cast<uint32_t>(((k / SK) & 1) ^ 1), p.error_word);
+            if (!go) *abort_flag = 1;
+            mbar_arrive_expect_tx(smem_addr(&sh->k_full[st]), go ? bytes : 0u);
+          }
+          go = __shfl_sync(0xffffffffu, go, 0);
+          if (go && ok) {
+            const uint32_t dst = smem_addr(kring + st * Cfg::kTensorBytes) + lane * chunk_bytes;
+#pragma unroll
+            for (int pn = 0; pn < Cfg::kPanels; ++pn)
+              tma_load_2d(dst + pn * Cfg::kPanelBytes, &tmap_k, smem_addr(&sh->k_full[st]), pn * 64, row, policy);
+          }
+          __syncwarp();
+        }
+        if (!is_k) {  // V
+          const int st = static_cast<int>(k % SV);
+          bool go = true;
+          if (lane == 0) {
+            go = (*abort_flag == 0) &&
+                 mbar_wait(smem_addr(&sh->v_empty[st]), static_cast<uint32_t>(((k / SV) & 1) ^ 1), p.error_word);
+            if (!go) *abort_flag = 1;
+            mbar_arrive_expect_tx(smem_addr(&sh->v_full[st]), go ? bytes : 0u);
+          }
+          go = __shfl_sync(0xffffffffu, go, 0);
+          if (go && ok) {
+            const uint32_t dst = smem_addr(vring + st * Cfg::kTensorBytes) + lane * chunk_bytes;
+#pragma unroll
+            for (int pn = 0; pn < Cfg::kPanels; ++pn)
+              tma_load_2d(dst + pn * Cfg::kPanelBytes, &tmap_v, smem_addr(&sh->v_full[st]), pn * 64, row, policy);
+          }
+          __syncwarp();
+        }
+      }
+      cur.next_segment(p, true);
+    }
+    // wait (bounded) for our own copies: the last use of every ring slot and Q buffer
+    if (lane == 0 && is_k) {
+      for (int s = 0; s < SK; ++s) {
+        const int64_t uses = k / SK + (s < k % SK ? 1 : 0);
+        if (uses > 0) mbar_wait(smem_addr(&sh->k_full[s]), static_cast<uint32_t>((uses - 1) & 1), p.error_word);
+      }
+      if (cur.ui > 0) mbar_wait(smem_addr(&sh->q_full), static_cast<uint32_t>((cur.ui - 1) & 1), p.error_word);
+    }
+    if (lane == 0 && !is_k) {
+      for (int s = 0; s < SV; ++s) {
+        const int64_t uses = k / SV + (s < k % SV ? 1 : 0);
+        if (uses > 0) mbar_wait(smem_addr(&sh->v_full[s]), static_cast<uint32_t>((uses - 1) & 1), p.error_word);
+      }
+    }
+    return;
+  }
+
+  if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    // One thread issues all tensor-core work: S = Q K^T up to kLookahead tiles ahead of the oldest
+    // tile whose P has not been consumed, and O += P V for that tile once its P is in tensor memory
+    // and its V has landed. S buffer (tile % 4) is reused only after the PV of the tile four earlier
+    // has completed. It suspends on barriers (short time hints) instead of spinning, since it shares
+    // its scheduler with two softmax warps.
+    constexpr int kLookahead = NS - 1;
+    if (lane == 0) {
+      TileWalker wq, wp;
+      wq.init(p, sh->b, sh->base_b, lo, hi);
+      wp.init(p, sh->b, sh->base_b, lo, hi);
+      TileInfo tq, tp;
+      bool have_q = wq.next(p, tq);
+      bool have_p = wp.next(p, tp);
+      int64_t kq = 0, kp = 0;
+      // descriptor bases; every K step only adds a constant to the 14-bit start-address field
+      const uint64_t q_desc = tc::smem_desc_sw128(smem_addr(qbuf), 16, 1024);
+      const uint64_t k_desc = tc::smem_desc_sw128(smem_addr(kring), 16, 1024);
+      const uint64_t v_desc = tc::smem_desc_sw128(smem_addr(vring), Cfg::kPanelBytes, 1024);
+      const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
+      bool ok = true;
+      auto qk_ready = [&]() -> bool {
+        return mbar_test(smem_addr(&sh->k_full[kq % SK]), static_cast<uint32_t>((kq / SK) & 1)) &&
+               (kq < NS ||
+                mbar_test(smem_addr(&sh->pv_done[kq % NS]), static_cast<uint32_t>(((kq / NS) - 1) & 1))) &&
+               (!tq.first || mbar_test(smem_addr(&sh->q_full), static_cast<uint32_t>(tq.ui & 1)));
+      };
+      auto issue_qk = [&]() {
+        tc::fence_after_sync();
+        const int kst = static_cast<int>(kq % SK);
+        const int sb = static_cast<int>(kq % NS);
+        const uint64_t kd = k_desc + static_cast<uint64_t>((kst * Cfg::kTensorBytes) >> 4);
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(sb * TK);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          // panel (ks / 4), then 16 elements = 32 bytes along the 128-byte swizzled row
+          const uint64_t qoff = static_cast<uint64_t>(((ks >> 2) * Cfg::kQPanelBytes + (ks & 3) * 32) >> 4);
+          const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kPanelBytes + (ks & 3) * 32) >> 4);
+          tc::mma_ss(d_tmem, q_desc + qoff, kd + koff, kIdescQK, ks > 0 ? 1u : 0u);
+        }
+        tc::commit(smem_addr(&sh->s_full[sb]));
+        tc::commit(smem_addr(&sh->k_empty[kst]));
+        if (tq.last) tc::commit(smem_addr(&sh->q_empty));
+        ++kq;
+        have_q = wq.next(p, tq);
+      };
+      auto pv_ready = [&]() -> bool {
+        return mbar_test(smem_addr(&sh->p_full[kp % NS]), static_cast<uint32_t>((kp / NS) & 1)) &&
+               mbar_test(smem_addr(&sh->v_full[kp % SV]), static_cast<uint32_t>((kp / SV) & 1)) &&
+               (!tp.first || tp.ui == 0 || mbar_test(smem_addr(&sh->o_free), static_cast<uint32_t>((tp.ui - 1) & 1)));
+      };
+      while (have_p && ok) {
+        // S = Q K^T for every tile that is ready, up to the lookahead; the tile whose P comes next
+        // must have its S before we wait for that P, so that one is waited for
+        while (have_q && kq <= kp + kLookahead) {
+          if (!qk_ready()) {
+            if (kq != kp) break;
+            while (ok && !qk_ready()) {
+              mbar_try_wait_hint(smem_addr(&sh->k_full[kq % SK]), static_cast<uint32_t>((kq / SK) & 1), 200);
+              ok = (*abort_flag == 0) && global_timer_ns() < deadline;
+            }
+            if (!ok) break;
+          }
+          issue_qk();
+        }
+        if (!ok) break;
+        // O += P V for tile kp: suspend on its P, issuing any S that becomes ready meanwhile
+        while (ok && !pv_ready()) {
+          mbar_try_wait_hint(smem_addr(&sh->p_full[kp % NS]), static_cast<uint32_t>((kp / NS) & 1), 200);
+          if (have_q && kq <= kp + kLookahead && qk_ready()) issue_qk();
+          ok = (*abort_flag == 0) && global_timer_ns() < deadline;
+        }
+        if (!ok) break;
+        tc::fence_after_sync();
+        const int sb = static_cast<int>(kp % NS);
+        const int vs = static_cast<int>(kp % SV);
+        const uint64_t vd = v_desc + static_cast<uint64_t>((vs * Cfg::kTensorBytes) >> 4);
+        const uint32_t a_tmem = tmem + static_cast<uint32_t>(sb * TK);
+        const uint32_t o_tmem = tmem + Cfg::kOCol + static_cast<uint32_t>((kp & 1) * 128);
+        const bool fresh = tp.jl < 2;  // first tile of this segment for its warpgroup
+#pragma unroll
+        for (int ks = 0; ks < TK / 16; ++ks) {
+          // V as the MN-major B operand: 64-column panels kPanelBytes apart (LBO), 8-key groups 1024
+          // bytes apart (SBO); 16 keys per step = 2048 bytes; P: 16 keys = 8 packed columns
+          tc::mma_ts(o_tmem, a_tmem + ks * 8, vd + static_cast<uint64_t>((ks * 2048) >> 4), kIdescPV,
+                     (fresh && ks == 0) ? 0u : 1u);
+        }
+        tc::commit(smem_addr(&sh->v_empty[vs]));
+        tc::commit(smem_addr(&sh->pv_done[sb]));
+        ++kp;
+        have_p = wp.next(p, tp);
+      }
+      if (!ok) {
+        // gave up (2 s without finishing, or another role aborted): release everyone still waiting
+        if (*abort_flag == 0) atomicOr(p.error_word, TACO_DEVERR_WAIT_TIMEOUT);
+        *abort_flag = 1;
+        while (have_q) {
+          tc::commit(smem_addr(&sh->s_full[kq % NS]));
+          tc::commit(smem_addr(&sh->k_empty[kq % SK]));
+          if (tq.last) tc::commit(smem_addr(&sh->q_empty));
+          ++kq;
+          have_q = wq.next(p, tq);
+        }
+        while (have_p) {
+          tc::commit(smem_addr(&sh->v_empty[kp % SV]));
+          tc::commit(smem_addr(&sh->pv_done[kp % NS]));
+          ++kp;
+          have_p = wp.next(p, tp);
+        }
+      }
+    }
+    __syncwarp();
+    tc::fence_before_sync();
+    named_bar_sync(2, 288);
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, Cfg::kTmemCols);
+    return;
+  }
+
+  // -------------------------------------------------------------------- softmax warpgroups
+  const int wg = (warp - 2) >> 2;             // 0 or 1: owns the tiles with k % 2 == wg (warps 2..9)
+  const int sub = warp & 3;                   // tensor-memory lane quarter of this warp
+  const int r = sub * 32 + lane;              // query row owned by this thread
+  const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
+  const uint32_t my_o = tmem + lane_base + Cfg::kOCol + static_cast<uint32_t>(wg * 128);
+  SegCursor cur;
+  cur.init(p, sh->b, sh->base_b, lo, hi, false);
+  int64_t k = 0;
+  bool first_segment = true;
+  while (cur.valid()) {
+    const int b = cur.b;
+    const int g = cur.j / p.row_groups;
+    const int rg = cur.j % p.row_groups;
+    const int L = cur.L;
+    const int tbegin = cur.tile;
+    const int tend = cur.seg_end();
+    const int Tb = cur.Tb;
+    const int n = clamp_candidates(p, b, L, false);
+    const int P = L - n;
+    const uint32_t nmask = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+    const int i = rg * cpg + r / p.G;            // candidate of this row
+    const int hh = r % p.G;
+    const bool row_real = r < qrows && i < p.C;  // a row of the output
+    const bool active = row_real && i < n;       // a row with a query
+    const uint32_t mw = active ? (__ldg(p.tree_mask_bits + static_cast<int64_t>(b) * p.C + i) & nmask) : 0u;
+
+    float m_ref = -INFINITY;
+    float l_run = 0.f;
+    int64_t k_mine_last = -1;
+    for (int tl = tbegin; tl < tend; ++tl, ++k) {
+      if (static_cast<int>(k & 1) != wg) continue;
+      const int key0 = tl * TK;
+      const int sb = static_cast<int>(k % NS);
+      const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(sb * TK);
+      bool ok = (*abort_flag == 0);
+      if (ok) ok = mbar_wait(smem_addr(&sh->s_full[sb]), static_cast<uint32_t>((k / NS) & 1), p.error_word);
+      if (!ok) *abort_flag = 1;
+      tc::fence_after_sync();
+      uint32_t sraw[2][32];
+      tc::ld_32x32b_x32(s_col, sraw[0]);
+      tc::ld_32x32b_x32(s_col + 32, sraw[1]);
+      if (key0 + TK > L) {
+        // keys >= L in this tile: their V rows may be stale or NaN-poisoned; zero them once V landed
+        const int vs = static_cast<int>(k % SV);
+        bool okv = (*abort_flag == 0);
+        if (okv) okv = mbar_wait(smem_addr(&sh->v_full[vs]), static_cast<uint32_t>((k / SV) & 1), p.error_word);
+        if (!okv) *abort_flag = 1;
+        int z0 = L - key0;
+        if (z0 < 0) z0 = 0;
+        uint8_t* vgen = vring + vs * Cfg::kTensorBytes;
+        const int per_row = Cfg::kPanels * 8;
+        for (int idx = r; idx < (TK - z0) * per_row; idx += 128) {
+          const int row = z0 + idx / per_row;
+          const int rem = idx % per_row;
+          *reinterpret_cast<uint4*>(vgen + (rem / 8) * Cfg::kPanelBytes + row * 128 + (rem % 8) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
+      tc::wait_ld();
+      static_assert(TK == 64, "the softmax below holds one 64-column tile per thread");
+      // Row max of the raw scores (a positive scale_log2 commutes with max; otherwise the scaled
+      // values are used). Masked keys become -inf; only the tiles that reach the candidates mask.
+      const bool need_mask = key0 + TK > P;
+      const bool pos_scale = p.scale_log2 > 0.f;
+      float v[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) v[c] = __uint_as_float(sraw[c >> 5][c & 31]);
+      if (!pos_scale) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) v[c] *= p.scale_log2;
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int key = key0 + c;
+          const bool vis = key < P || (key < L && ((mw >> ((key - P) & 31)) & 1u));
+          v[c] = vis ? v[c] : -INFINITY;
+        }
+      }
+      float m8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float a = tc::max3(v[8 * e], v[8 * e + 1], v[8 * e + 2]);
+        a = tc::max3(a, v[8 * e + 3], v[8 * e + 4]);
+        a = tc::max3(a, v[8 * e + 5], v[8 * e + 6]);
+        m8[e] = fmaxf(a, v[8 * e + 7]);
+      }
+      const float mraw = tc::max3(tc::max3(m8[0], m8[1], m8[2]), tc::max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+      const bool first = (k_mine_last < 0);
+      // rows without a query (padding) keep whatever their scores are; they never reach the output,
+      // so they are simply kept out of the rescale decision
+      float mx = pos_scale ? mraw * p.scale_log2 : mraw;  // row max of the base-2 logits
+      if (!active) mx = first ? 0.f : m_ref;
+      bool rescale = false;
+      float alpha = 1.f;
+      if (first) {
+        m_ref = mx;
+      } else if (mx > m_ref + 8.f) {
+        rescale = true;
+        alpha = fast_exp2(m_ref - mx);
+        l_run *= alpha;
+        m_ref = mx;
+      }
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // p = 2^(s * scale_log2 - m) on fp32 pairs; sums in four independent pair accumulators
+      const float sc = pos_scale ? p.scale_log2 : 1.f;
+      const uint64_t sc2 = tc::f2(sc, sc);
+      const uint64_t nm2 = tc::f2(-m_use, -m_use);
+      uint64_t acc2[4] = {tc::f2(0.f, 0.f), tc::f2(0.f, 0.f), tc::f2(0.f, 0.f), tc::f2(0.f, 0.f)};
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float a0, a1;
+        tc::f2_split(tc::f2_fma(tc::f2(v[2 * c], v[2 * c + 1]), sc2, nm2), a0, a1);
+        const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+        acc2[c & 3] = tc::f2_add(acc2[c & 3], tc::f2(p0, p1));
+        pk[c] = Op::pack(p0, p1);
+      }
+      {
+        float s0, s1, s2, s3, s4, s5, s6, s7;
+        tc::f2_split(acc2[0], s0, s1);
+        tc::f2_split(acc2[1], s2, s3);
+        tc::f2_split(acc2[2], s4, s5);
+        tc::f2_split(acc2[3], s6, s7);
+        l_run += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+      }
+      tc::st_32x32b_x32(s_col, pk);
+      if (__any_sync(0xffffffffu, rescale)) {
+        // this warpgroup's O must be stable: the PV of its previous tile has to be complete
+        const int64_t kprev = k_mine_last;
+        bool okw = (*abort_flag == 0);
+        if (okw)
+          okw = mbar_wait(smem_addr(&sh->pv_done[kprev % NS]), static_cast<uint32_t>((kprev / NS) & 1), p.error_word);
+        if (!okw) *abort_flag = 1;
+        tc::fence_after_sync();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tc::ld_32x32b_x32(my_o + c * 32, o);
+          tc::wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tc::st_32x32b_x32(my_o + c * 32, o);
+        }
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&sh->p_full[sb]));
+      k_mine_last = k;
+    }
+
+    // ---------------------------------------------------------------- segment epilogue
+    // wait for this warpgroup's last PV (each S buffer has its own completion barrier)
+    if (k_mine_last >= 0) {
+      bool ok = (*abort_flag == 0);
+      if (ok)
+        ok = mbar_wait(smem_addr(&sh->pv_done[k_mine_last % NS]), static_cast<uint32_t>((k_mine_last / NS) & 1),
+                       p.error_word);
+      if (!ok) *abort_flag = 1;
+    }
+    if (wg == 1) {
+      sh->xm[cur.ui & 1][r] = k_mine_last >= 0 ? m_ref : -INFINITY;
+      sh->xl[cur.ui & 1][r] = k_mine_last >= 0 ? l_run : 0.f;
+      tc::fence_before_sync();
+      named_bar_sync(3, 256);
+    } else {
+      named_bar_sync(3, 256);
+      tc::fence_after_sync();
+      const float m1 = sh->xm[cur.ui & 1][r];
+      const float l1 = sh->xl[cur.ui & 1][r];
+      const float m0 = k_mine_last >= 0 ? m_ref : -INFINITY;
+      const float l0 = k_mine_last >= 0 ? l_run : 0.f;
+      const float M = fmaxf(m0, m1);
+      const float f0 = l0 > 0.f ? fast_exp2(m0 - M) : 0.f;
+      const float f1 = l1 > 0.f ? fast_exp2(m1 - M) : 0.f;
+      const float ltot = f0 * l0 + f1 * l1;
+      const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+      const float w0 = f0 * inv, w1 = f1 * inv;
+      const bool use0 = f0 > 0.f, use1 = f1 > 0.f;
+      const bool whole_unit = (tbegin == 0 && tend == Tb);
+      const int slot = 2 * static_cast<int>(blockIdx.x) + (first_segment ? 0 : 1);
+      T* dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D;
+      float* pdst = p.part_o + (static_cast<int64_t>(slot) * 128 + r) * D;
+      const uint32_t o0 = tmem + lane_base + Cfg::kOCol;
+      const uint32_t o1 = o0 + 128;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32], bb[32];
+        tc::ld_32x32b_x32(o0 + c * 32, a);
+        tc::ld_32x32b_x32(o1 + c * 32, bb);
+        tc::wait_ld();
+        float x[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          x[e] = (use0 ? w0 * __uint_as_float(a[e]) : 0.f) + (use1 ? w1 * __uint_as_float(bb[e]) : 0.f);
+        if (whole_unit) {
+          if (row_real) {
+            uint32_t wv[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) wv[e] = active ? Op::pack(x[2 * e], x[2 * e + 1]) : 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              *reinterpret_cast<uint4*>(dst + c * 32 + e * 8) =
+                  make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            __stcg(reinterpret_cast<float4*>(pdst + c * 32 + e * 4),
+                   make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]));
+        }
+      }
+      if (!whole_unit)
+        __stcg(p.part_lse + static_cast<int64_t>(slot) * 128 + r, ltot > 0.f ? M + __log2f(ltot) : -INFINITY);
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&sh->o_free));
+
+      if (!whole_unit) {
+        __threadfence();
+        named_bar_sync(1, 128);
+        const int64_t unit_base = cur.unit_base();
+        const int c_first = cta_of_tile(unit_base, W, nC);
+        const int c_last = cta_of_tile(unit_base + Tb - 1, W, nC);
+        const int u = (b * p.Hkv + g) * p.row_groups + rg;
+        if (warp == 2 && lane == 0) {
+          const uint32_t prev = atomicAdd(p.counters + u, 1u);
+          const bool last = prev == static_cast<uint32_t>(c_last - c_first);
+          if (last) {
+            p.counters[u] = 0u;
+            __threadfence();
+          }
+          sh->merge_flag = last ? 1 : 0;
+        }
+        named_bar_sync(1, 128);
+        if (sh->merge_flag) {
+          // combine the unit's partials in CTA order: out = sum_s 2^(lse_s - max) O_s / sum_s 2^(...)
+          const int64_t lo_first = static_cast<int64_t>(c_first) * W / nC;
+          for (int rr = warp - 2; rr < qrows; rr += 4) {
+            const int ii = rg * cpg + rr / p.G;
+            if (ii >= p.C) break;
+            const int h2 = rr % p.G;
+            T* o_dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + ii) * p.Hq + g * p.G + h2) * D;
+            float acc[D / 32];
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+            float wsum = 0.f;
+            if (ii < n) {
+              float lmax = -INFINITY;
+              for (int c = c_first; c <= c_last; ++c) {
+                const int sl = (c == c_first && lo_first < unit_base) ? 2 * c + 1 : 2 * c;
+                lmax = fmaxf(lmax, __ldcg(p.part_lse + static_cast<int64_t>(sl) * 128 + rr));
+              }
+              if (lmax != -INFINITY) {
+                for (int c = c_first; c <= c_last; ++c) {
+                  const int sl = (c == c_first && lo_first < unit_base) ? 2 * c + 1 : 2 * c;
+                  const float ls = __ldcg(p.part_lse + static_cast<int64_t>(sl) * 128 + rr);
+                  const float wgt = ls == -INFINITY ? 0.f : exp2f(ls - lmax);
+                  wsum += wgt;
+                  const float* src = p.part_o + (static_cast<int64_t>(sl) * 128 + rr) * D + lane * (D / 32);
+#pragma unroll
+                  for (int e = 0; e < D / 32; ++e) acc[e] += wgt * __ldcg(src + e);
+                }
+              }
+            }
+            const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+            for (int e = 0; e < D / 32; e += 2)
+              *reinterpret_cast<uint32_t*>(o_dst + lane * (D / 32) + e) = Op::pack(acc[e] * winv, acc[e + 1] * winv);
+          }
+        }
+        named_bar_sync(1, 128);
+      }
+    }
+    first_segment = false;
+    cur.next_segment(p, false);
+  }
+  tc::fence_before_sync();
+  named_bar_sync(2, 288);
+}
+
+}  // namespace taco

@@ -48,10 +48,15 @@ SMALL_CASES = [
 ]
 
 
+KERNELS = [1, 2]   # 1 = mma.sync path, 2 = tcgen05 path (forced, whatever the tile width)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("case", range(len(SMALL_CASES)))
-def test_small_shapes_full_oracle(case):
+def test_small_shapes_full_oracle(case, kernel):
     dtype, B, Hq, Hkv, D, bs, C, tree, ctx, ncand = SMALL_CASES[case]
     spec = dict(dtype=dtype, B=B, Hq=Hq, Hkv=Hkv, D=D, bs=bs, C=C, tree=tree, ctx=ctx)
+    taco.set_option(taco.TACO_OPT_KERNEL, kernel)
     w = wl.make_workload(spec, seed=100 + case, candidates_in_cache=False, num_candidates=ncand)
     out, kc, vc = gpu_step(w)
     ref, rkc, rvc = oracle_step(w)
@@ -60,19 +65,23 @@ def test_small_shapes_full_oracle(case):
     assert_parity(out, ref, w)
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("grid", [1, 3, 7, 64, 500])
-def test_split_kv_partitions_agree(grid):
-    spec = dict(dtype="bf16", B=3, Hq=16, Hkv=4, D=128, bs=16, C=4, tree="forest", ctx=("uniform", 100, 700))
+def test_split_kv_partitions_agree(grid, kernel):
+    spec = dict(dtype="bf16", B=3, Hq=32, Hkv=4, D=128, bs=16, C=6, tree="forest", ctx=("uniform", 100, 900))
     w = wl.make_workload(spec, seed=7)
     ref, _, _ = oracle_step(w, append=False)
     taco.set_option(taco.TACO_OPT_GRID_CTAS, grid)
+    taco.set_option(taco.TACO_OPT_KERNEL, kernel)
     out, _, _ = gpu_step(w, append=False)
     assert_parity(out, ref, w)
     again, _, _ = gpu_step(w, append=False)
     assert torch.equal(out.view(torch.int16), again.view(torch.int16)), "not deterministic run to run"
 
 
-def test_block_permutation_gives_bitwise_identical_output():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_block_permutation_gives_bitwise_identical_output(kernel):
+    taco.set_option(taco.TACO_OPT_KERNEL, kernel)
     spec = dict(dtype="bf16", B=4, Hq=32, Hkv=8, D=128, bs=16, C=4, tree="forest", ctx=("uniform", 50, 600))
     w = wl.make_workload(spec, seed=17)
     out1, _, _ = gpu_step(w, append=False)
@@ -90,7 +99,9 @@ def test_block_permutation_gives_bitwise_identical_output():
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
-def test_only_ancestors_matter_on_gpu():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_only_ancestors_matter_on_gpu(kernel):
+    taco.set_option(taco.TACO_OPT_KERNEL, kernel)
     spec = dict(dtype="bf16", B=1, Hq=8, Hkv=2, D=128, bs=16, C=5, tree="chain", ctx=("fixed", [90]))
     w = wl.make_workload(spec, seed=23, parents=[[-1, 0, 0, 1, -1]])
     out1, _, _ = gpu_step(w, append=False)
@@ -104,7 +115,9 @@ def test_only_ancestors_matter_on_gpu():
         assert same == (i != 2), i
 
 
-def test_one_key_context_returns_v_exactly():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_one_key_context_returns_v_exactly(kernel):
+    taco.set_option(taco.TACO_OPT_KERNEL, kernel)
     spec = dict(dtype="bf16", B=3, Hq=8, Hkv=2, D=128, bs=16, C=1, tree="chain", ctx=("fixed", [1, 1, 1]))
     w = wl.make_workload(spec, seed=5)
     out, _, _ = gpu_step(w, append=False)
@@ -139,7 +152,9 @@ def test_full_size_workloads_sampled_rows(name):
     assert torch.isfinite(out.float()).all()
 
 
-def test_device_range_errors_are_reported_not_faulted():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_device_range_errors_are_reported_not_faulted(kernel):
+    taco.set_option(taco.TACO_OPT_KERNEL, kernel)
     spec = dict(dtype="bf16", B=2, Hq=8, Hkv=2, D=128, bs=16, C=2, tree="chain", ctx=("fixed", [40, 70]))
     w = wl.make_workload(spec, seed=2)
     d = w.to("cuda")
