@@ -286,6 +286,117 @@ __device__ __forceinline__ SchedStart schedule_start(const VerifyParams& p, int 
   return s;  // not reached for lo < W
 }
 
+// Destination of merged row r of a unit: dst == nullptr for a padding row (nothing is written),
+// active == false for a row of a padding candidate (written as zeros).
+template <typename T>
+struct MergeRow {
+  T* dst;
+  bool active;
+};
+
+// Combines the partials of one split unit into its output rows:
+//   out_r = sum_s 2^(lse_s,r - M_r) O_s,r / sum_s 2^(lse_s,r - M_r),   M_r = max_s lse_s,r,
+// over the pieces s = 0 .. c_last - c_first (CTA order; piece 0 sits in slot 2*c_first + 1 when
+// it is not c_first's first segment, every other piece in slot 2c). Partials are stored
+// [slot][row (stride rows)][D] fp32 with normalised O, lse in base 2; lse = -inf means the piece
+// saw no visible key and weighs 0.
+// Run by the 4 warps (wid 0..3) of one 128-thread group. A warp takes 8 rows x 2 pieces per pass,
+// with the lse and O loads of the pass all issued before use, so a pass costs one L2 round trip;
+// pieces beyond 2 are folded in with an online rescale.
+template <typename T, int D, typename RowFn>
+__device__ __forceinline__ void merge_split_unit(const VerifyParams& p, int rows, int stride, int c_first,
+                                                 int c_last, bool first_odd, int wid, int lane, RowFn row_of) {
+  constexpr int RB = 8, SC = 2, V = D / 32;
+  static_assert(V == 2 || V == 4, "head_dim 64 or 128");
+  const int nsl = c_last - c_first + 1;
+  auto slot_of = [&](int s) -> int64_t {
+    const int c = c_first + s;
+    return (s == 0 && first_odd) ? 2 * c + 1 : 2 * c;
+  };
+  for (int r0 = wid * RB; r0 < rows; r0 += 4 * RB) {
+    float acc[RB][V], m[RB], l[RB];
+#pragma unroll
+    for (int k = 0; k < RB; ++k) {
+      m[k] = -INFINITY;
+      l[k] = 0.f;
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[k][e] = 0.f;
+    }
+    for (int s0 = 0; s0 < nsl; s0 += SC) {
+      float ls = -INFINITY;  // lane j*RB + k holds lse of (piece s0 + j, row r0 + k)
+      {
+        const int k = lane % RB, j = lane / RB;
+        if (j < SC && s0 + j < nsl && r0 + k < rows) ls = __ldcg(p.part_lse + slot_of(s0 + j) * stride + r0 + k);
+      }
+      float v[SC][RB][V];
+#pragma unroll
+      for (int j = 0; j < SC; ++j) {
+        const bool have = s0 + j < nsl;
+        const int64_t sl = have ? slot_of(s0 + j) : 0;
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+          if (have && r0 + k < rows) {
+            const float* src = p.part_o + (sl * stride + r0 + k) * D + lane * V;
+            if constexpr (V == 4) {
+              const float4 x = __ldcg(reinterpret_cast<const float4*>(src));
+              v[j][k][0] = x.x;
+              v[j][k][1] = x.y;
+              v[j][k][2] = x.z;
+              v[j][k][3] = x.w;
+            } else {
+              const float2 x = __ldcg(reinterpret_cast<const float2*>(src));
+              v[j][k][0] = x.x;
+              v[j][k][1] = x.y;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < V; ++e) v[j][k][e] = 0.f;
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < RB; ++k) {
+        float lj[SC];
+        float cm = m[k];
+#pragma unroll
+        for (int j = 0; j < SC; ++j) {
+          lj[j] = __shfl_sync(0xffffffffu, ls, j * RB + k);
+          cm = fmaxf(cm, lj[j]);
+        }
+        if (cm == -INFINITY) continue;  // nothing visible in this row so far (warp-uniform)
+        const float f = m[k] == -INFINITY ? 0.f : exp2f(m[k] - cm);
+        l[k] *= f;
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[k][e] *= f;
+#pragma unroll
+        for (int j = 0; j < SC; ++j) {
+          if (lj[j] == -INFINITY) continue;
+          const float w = exp2f(lj[j] - cm);
+          l[k] += w;
+#pragma unroll
+          for (int e = 0; e < V; ++e) acc[k][e] = fmaf(w, v[j][k][e], acc[k][e]);
+        }
+        m[k] = cm;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < RB; ++k) {
+      if (r0 + k >= rows) break;
+      const MergeRow<T> d = row_of(r0 + k);
+      if (d.dst == nullptr) continue;
+      const float inv = (d.active && l[k] > 0.f) ? 1.f / l[k] : 0.f;
+      uint32_t w2[V / 2];
+#pragma unroll
+      for (int e = 0; e < V / 2; ++e)
+        w2[e] = d.active ? MmaOp<T>::pack(acc[k][2 * e] * inv, acc[k][2 * e + 1] * inv) : 0u;
+      if constexpr (V == 4)
+        *reinterpret_cast<uint2*>(d.dst + lane * V) = make_uint2(w2[0], w2[1]);
+      else
+        *reinterpret_cast<uint32_t*>(d.dst + lane * V) = w2[0];
+    }
+  }
+}
+
 // Walks one CTA's work as segments: a segment is the part of one unit (b, j = g * RG + rg) that
 // falls into the CTA's tile range; tiles [tile, seg_end()) of the unit.
 struct SegCursor {

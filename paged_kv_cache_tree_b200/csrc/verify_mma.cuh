@@ -457,40 +457,16 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
       }
       named_bar_sync(1, 128);
       if (sched->merge_flag) {
-        // combine the unit's partials in CTA order: out = sum_s 2^(lse_s - max) O_s / sum_s 2^(...)
         const int64_t lo_first = static_cast<int64_t>(c_first) * W / nC;
-        for (int r = warp; r < ROWS; r += 4) {
-          const int R = rg * ROWS + r;
-          if (R >= p.G * p.C) break;
-          const int i = R / p.G, hh = R % p.G;
-          T* dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D;
-          float acc[D / 32];
-#pragma unroll
-          for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
-          float wsum = 0.f;
-          if (R < p.G * n) {
-            float lmax = -INFINITY;
-            for (int c = c_first; c <= c_last; ++c) {
-              const int sl = (c == c_first && lo_first < unit_base) ? 2 * c + 1 : 2 * c;
-              lmax = fmaxf(lmax, __ldcg(p.part_lse + static_cast<int64_t>(sl) * ROWS + r));
-            }
-            if (lmax != -INFINITY) {
-              for (int c = c_first; c <= c_last; ++c) {
-                const int sl = (c == c_first && lo_first < unit_base) ? 2 * c + 1 : 2 * c;
-                const float ls = __ldcg(p.part_lse + static_cast<int64_t>(sl) * ROWS + r);
-                const float wgt = ls == -INFINITY ? 0.f : exp2f(ls - lmax);
-                wsum += wgt;
-                const float* src = p.part_o + (static_cast<int64_t>(sl) * ROWS + r) * D + lane * (D / 32);
-#pragma unroll
-                for (int e = 0; e < D / 32; ++e) acc[e] += wgt * __ldcg(src + e);
-              }
-            }
-          }
-          const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-#pragma unroll
-          for (int e = 0; e < D / 32; e += 2)
-            *reinterpret_cast<uint32_t*>(dst + lane * (D / 32) + e) = Op::pack(acc[e] * inv, acc[e + 1] * inv);
-        }
+        const int64_t row0 = static_cast<int64_t>(b) * p.C;
+        merge_split_unit<T, D>(p, ROWS, ROWS, c_first, c_last, lo_first < unit_base, warp, lane,
+                               [&](int r) -> MergeRow<T> {
+                                 const int R = rg * ROWS + r;
+                                 if (R >= p.G * p.C) return MergeRow<T>{nullptr, false};
+                                 const int i = R / p.G;
+                                 T* d = static_cast<T*>(p.out) + ((row0 + i) * p.Hq + g * p.G + R % p.G) * D;
+                                 return MergeRow<T>{d, i < n};
+                               });
       }
       named_bar_sync(1, 128);
     }

@@ -630,40 +630,15 @@ __global__ void __launch_bounds__(352, 1)
         }
         named_bar_sync(1, 128);
         if (sh->merge_flag) {
-          // combine the unit's partials in CTA order: out = sum_s 2^(lse_s - max) O_s / sum_s 2^(...)
           const int64_t lo_first = static_cast<int64_t>(c_first) * W / nC;
-          for (int rr = warp - 2; rr < qrows; rr += 4) {
-            const int ii = rg * cpg + rr / p.G;
-            if (ii >= p.C) break;
-            const int h2 = rr % p.G;
-            T* o_dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + ii) * p.Hq + g * p.G + h2) * D;
-            float acc[D / 32];
-#pragma unroll
-            for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
-            float wsum = 0.f;
-            if (ii < n) {
-              float lmax = -INFINITY;
-              for (int c = c_first; c <= c_last; ++c) {
-                const int sl = (c == c_first && lo_first < unit_base) ? 2 * c + 1 : 2 * c;
-                lmax = fmaxf(lmax, __ldcg(p.part_lse + static_cast<int64_t>(sl) * 128 + rr));
-              }
-              if (lmax != -INFINITY) {
-                for (int c = c_first; c <= c_last; ++c) {
-                  const int sl = (c == c_first && lo_first < unit_base) ? 2 * c + 1 : 2 * c;
-                  const float ls = __ldcg(p.part_lse + static_cast<int64_t>(sl) * 128 + rr);
-                  const float wgt = ls == -INFINITY ? 0.f : exp2f(ls - lmax);
-                  wsum += wgt;
-                  const float* src = p.part_o + (static_cast<int64_t>(sl) * 128 + rr) * D + lane * (D / 32);
-#pragma unroll
-                  for (int e = 0; e < D / 32; ++e) acc[e] += wgt * __ldcg(src + e);
-                }
-              }
-            }
-            const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
-#pragma unroll
-            for (int e = 0; e < D / 32; e += 2)
-              *reinterpret_cast<uint32_t*>(o_dst + lane * (D / 32) + e) = Op::pack(acc[e] * winv, acc[e + 1] * winv);
-          }
+          const int64_t row0 = static_cast<int64_t>(b) * p.C;
+          merge_split_unit<T, D>(p, qrows, 128, c_first, c_last, lo_first < unit_base, warp - 2, lane,
+                                 [&](int rr) -> MergeRow<T> {
+                                   const int ii = rg * cpg + rr / p.G;
+                                   if (ii >= p.C) return MergeRow<T>{nullptr, false};
+                                   T* d = static_cast<T*>(p.out) + ((row0 + ii) * p.Hq + g * p.G + rr % p.G) * D;
+                                   return MergeRow<T>{d, ii < n};
+                                 });
         }
         named_bar_sync(1, 128);
       }
