@@ -1,11 +1,13 @@
 // Verify kernel for narrow packed query tiles (G * C up to 64 rows per unit): the warp-level
 // mma.sync path.
 //
-// One CTA = 4 consumer warps + 1 producer warp, two CTAs per SM, persistent over a stream-K range of
-// key tiles (device_common.cuh). The producer warp walks the block table and streams each tile's
-// K and V chunks (one chunk = min(bs, 64) consecutive slots of one physical block and one KV head,
-// contiguous in the [NB, Hkv, bs, D] cache) into a ring of shared-memory stages with TMA, 128-byte
-// swizzled so that ldmatrix reads are conflict-free. Consumer warps own 16 packed query rows each
+// One CTA = 4 consumer warps + 2 producer warps, two CTAs per SM, persistent over a stream-K range of
+// key tiles (device_common.cuh). The producer warps walk the block table and stream each tile's
+// K chunks (first producer) and V chunks (second producer) (one chunk = min(bs, 64) consecutive
+// slots of one physical block and one KV head, contiguous in the [NB, Hkv, bs, D] cache) into a ring
+// of shared-memory stages with TMA, 128-byte swizzled so that ldmatrix reads are conflict-free. A
+// single warp can keep only so many TMA copies moving, so K and V are issued from separate warps;
+// both walk every stage in order and arm the stage's full barrier (arrival count 2). Consumer warps own 16 packed query rows each
 // (rows r = i * G + h' of candidate i and head g*G + h') and, when fewer than 4 row tiles exist,
 // split the tile's keys between them; S = Q K^T and O += P V run on mma.sync m16n8k16 with fp32
 // accumulators, and the softmax is the flash-style online form in base 2 (fp32 running max / sum).
@@ -19,7 +21,8 @@ namespace taco {
 template <int D, int MT>
 struct MmaCfg {
   static constexpr int kConsumerWarps = 4;
-  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+  static constexpr int kProducerWarps = 2;                   // K and V
+  static constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
   static constexpr int KG = kConsumerWarps / MT;              // key groups
   static constexpr int kKeysPerWarp = kTileKeys / KG;         // 16, 32 or 64
   static constexpr int kRows = 16 * MT;                       // packed rows per unit
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
 
   if (tid == 0) {
     for (int s = 0; s < Cfg::kStages; ++s) {
-      mbar_init(smem_addr(full_bar + s), 1);
+      mbar_init(smem_addr(full_bar + s), Cfg::kProducerWarps);
       mbar_init(smem_addr(empty_bar + s), Cfg::kConsumerWarps);
     }
     fence_mbar_init();
@@ -94,10 +97,11 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
   const int64_t lo = sched->lo, hi = sched->hi;
   volatile int* abort_flag = &sched->abort_flag;
 
-  if (warp == Cfg::kConsumerWarps) {
-    // ------------------------------------------------------------------ producer warp
-    prefetch_tensormap(&tmap_k);
-    prefetch_tensormap(&tmap_v);
+  if (warp >= Cfg::kConsumerWarps) {
+    // ------------------------------------------------------------------ producer warps (K, V)
+    const bool is_k = (warp == Cfg::kConsumerWarps);
+    const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
+    prefetch_tensormap(tmap);
     const uint64_t policy = policy_evict_first();
     const int rpc = p.bs < kTileKeys ? p.bs : kTileKeys;   // rows per chunk
     const int chunks_per_tile = kTileKeys / rpc;
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     uint32_t phase = 0;
     int b = sched->b;
     int64_t base_b = sched->base_b;
-    int L = clamp_context(p, b, true);
+    int L = clamp_context(p, b, is_k);
     int Tb = tiles_of(L, kTileKeys);
     int64_t t = lo;
     int j = static_cast<int>((t - base_b) / Tb);
@@ -133,11 +137,11 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
         int32_t blk = __shfl_sync(0xffffffffu, win_val, (my_lb - win) & 31);
         bool ok = lane < nvalid;
         if (ok && (blk < 0 || blk >= p.num_blocks)) {
-          atomicOr(p.error_word, TACO_DEVERR_BLOCK_ID);
+          if (is_k) atomicOr(p.error_word, TACO_DEVERR_BLOCK_ID);
           ok = false;
         }
         const uint32_t okmask = __ballot_sync(0xffffffffu, ok);
-        const uint32_t bytes = __popc(okmask) * chunk_bytes * Cfg::kPanels * 2u;
+        const uint32_t bytes = __popc(okmask) * chunk_bytes * Cfg::kPanels;
         bool go = true;
         if (lane == 0) {
           go = (*abort_flag == 0) && mbar_wait(smem_addr(empty_bar + stage), phase ^ 1u, p.error_word);
@@ -146,15 +150,12 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
         }
         go = __shfl_sync(0xffffffffu, go, 0);
         if (go && ok) {
-          const uint32_t kdst = smem_addr(stages + stage * Cfg::kStageBytes) + lane * chunk_bytes;
-          const uint32_t vdst = kdst + Cfg::kTensorBytes;
+          const uint32_t dst = smem_addr(stages + stage * Cfg::kStageBytes) + (is_k ? 0u : Cfg::kTensorBytes) +
+                               lane * chunk_bytes;
           const int row = (blk * p.Hkv + g) * p.bs + (key0 + lane * rpc) % p.bs;
           const uint32_t fb = smem_addr(full_bar + stage);
 #pragma unroll
-          for (int pn = 0; pn < Cfg::kPanels; ++pn) {
-            tma_load_2d(kdst + pn * Cfg::kPanelBytes, &tmap_k, fb, pn * 64, row, policy);
-            tma_load_2d(vdst + pn * Cfg::kPanelBytes, &tmap_v, fb, pn * 64, row, policy);
-          }
+          for (int pn = 0; pn < Cfg::kPanels; ++pn) tma_load_2d(dst + pn * Cfg::kPanelBytes, tmap, fb, pn * 64, row, policy);
         }
         __syncwarp();
         if (++stage == Cfg::kStages) {
@@ -168,7 +169,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
         j = 0;
         base_b += static_cast<int64_t>(Tb) * HR;
         if (++b < p.B) {
-          L = clamp_context(p, b, true);
+          L = clamp_context(p, b, is_k);
           Tb = tiles_of(L, kTileKeys);
         }
       }
