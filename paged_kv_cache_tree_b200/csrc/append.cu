@@ -10,6 +10,7 @@ namespace taco {
 
 template <int VEC_PER_ROW>
 __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
+  grid_launch_dependents();  // a verify launched next may start its prologue now
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t total = static_cast<int64_t>(a.B) * a.C * a.Hkv * VEC_PER_ROW;
   if (gid >= total) return;

@@ -77,6 +77,8 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     }
     fence_mbar_init();
   }
+  // inputs (and the cache an append just wrote) are read only after the grids this launch depends on
+  grid_dependency_wait();
   if (warp == Cfg::kConsumerWarps) {
     SchedStart s = schedule_start(p, blockIdx.x, gridDim.x);
     if (lane == 0) {

@@ -120,6 +120,8 @@ __global__ void __launch_bounds__(352, 1)
     tc::tmem_alloc(smem_addr(&sh->tmem_base), Cfg::kTmemCols);
     tc::tmem_relinquish();
   }
+  // inputs (and the cache an append just wrote) are read only after the grids this launch depends on
+  grid_dependency_wait();
   if (warp == 0) {
     SchedStart s0 = schedule_start(p, blockIdx.x, gridDim.x);
     if (lane == 0) {
