@@ -1,4 +1,4 @@
-"""CPU oracle (test infrastructure only; see ``oracle.paged_attention``)."""
+"""CPU oracle (test infrastructure only; see ``oracle.paged_attention`` and ``oracle.tree_accept``)."""
 from .paged_attention import (  # noqa: F401
     gather_sequence_kv,
     paged_kv_append,
@@ -8,3 +8,4 @@ from .paged_attention import (  # noqa: F401
     widen_to_f64,
     within_tolerance,
 )
+from . import tree_accept  # noqa: F401,E402

@@ -275,6 +275,64 @@ def make_workload(
     )
 
 
+@dataclasses.dataclass
+class AcceptInputs:
+    """Host tensors of one acceptance step (after a verify): candidate tokens and target logits."""
+
+    vocab: int
+    tokens: torch.Tensor          # int32 [B, C]   candidate token ids (rows i >= n_b: -1)
+    target_logits: torch.Tensor   # bf16/fp16 [B, C + 1, V]   row 0: after the prefix, row i + 1: after candidate i
+    planted: torch.Tensor         # int32 [B, C + 1]  the index each row's margin was planted at
+
+    def logits_bytes(self) -> int:
+        return self.target_logits.numel() * self.target_logits.element_size()
+
+    def to(self, device) -> "AcceptInputs":
+        return AcceptInputs(self.vocab, self.tokens.to(device), self.target_logits.to(device), self.planted.to(device))
+
+
+def make_accept_inputs(w: Workload, *, vocab: int = 128256, seed: Optional[int] = None, hit_prob: float = 0.7,
+                       margin: float = 8.0, ties: bool = False) -> AcceptInputs:
+    """Draw the target model's logits and the candidates' tokens for workload ``w``'s candidate trees.
+
+    Recipe (one generator, seed = 5000 + the workload's seed unless given), in draw order:
+      1. per (b, row) of the B x (C + 1) rows a planted index, uniform in [0, V);
+      2. the logits, ~N(0, 1) rounded to ``w``'s dtype, then ``margin`` added at each planted index
+         (so that row's largest value sits there; with ``ties`` every third row also gets the same
+         value at a second, uniformly drawn index);
+      3. per candidate a coin with P(hit) = ``hit_prob``: a hit copies the planted index of its
+         parent's row (row 0 for a root), a miss draws a uniform index different from it.
+    Vocabulary 128256 is the size of the Llama-3.1 tokenizer the pages' models use.
+    """
+    B, C = w.B, w.C
+    if seed is None:
+        seed = 5000 + int(w.context_lens.sum().item()) % 100000
+    g = torch.Generator().manual_seed(int(seed))
+    rows = C + 1
+    planted = torch.randint(0, vocab, (B, rows), generator=g, dtype=torch.int64)
+    logits = _randn(B * rows * vocab, g, TORCH_DTYPES[w.dtype]).view(B, rows, vocab)
+    second = torch.randint(0, vocab, (B, rows), generator=g, dtype=torch.int64)
+    for b in range(B):
+        for r in range(rows):
+            top = logits[b, r, planted[b, r]].float() + margin
+            logits[b, r, planted[b, r]] = top
+            if ties and (b * rows + r) % 3 == 0 and int(second[b, r]) != int(planted[b, r]):
+                logits[b, r, second[b, r]] = logits[b, r, planted[b, r]]
+    coins = torch.rand((B, C), generator=g)
+    other = torch.randint(0, vocab - 1, (B, C), generator=g, dtype=torch.int64)
+    tokens = torch.full((B, C), -1, dtype=torch.int32)
+    for b in range(B):
+        for i in range(int(w.num_candidates[b])):
+            p = int(w.parents[b, i])
+            want = int(planted[b, 0 if p < 0 else p + 1])
+            if float(coins[b, i]) < hit_prob:
+                tokens[b, i] = want
+            else:
+                o = int(other[b, i])
+                tokens[b, i] = o if o < want else o + 1
+    return AcceptInputs(vocab=vocab, tokens=tokens, target_logits=logits, planted=planted.to(torch.int32))
+
+
 def to_numpy_bits(t: torch.Tensor):
     """Raw 16-bit patterns of a bf16/fp16 tensor as a numpy uint16 array (no value conversion)."""
     return t.contiguous().view(torch.int16).numpy().view("uint16")
