@@ -56,6 +56,7 @@ typedef int32_t taco_status;
 #define TACO_DEVERR_NUM_CAND 0x4u       /* num_candidates[b] outside [0, min(C, context_lens[b])] */
 #define TACO_DEVERR_SLOT 0x8u           /* slot_offsets[b][i] >= maxblk * bs */
 #define TACO_DEVERR_WAIT_TIMEOUT 0x10u  /* a pipeline wait gave up (the kernel returned early) */
+#define TACO_DEVERR_PARENT 0x20u        /* parents[b][i] outside [-1, i) */
 
 /*
  * paged_tree_attention: masked softmax attention of every candidate query over its sequence's
@@ -136,6 +137,63 @@ taco_status paged_tree_attention_noalloc(const void* q, const void* k_cache, con
                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                          int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
                                          void* stream);
+
+/*
+ * The step after the verify. The pages ("大模型倍速推理引擎 TACO-LLM 的设计与实践", sections
+ * "TACO-LLM 如何解决大模型推理瓶颈?", "优化方案设计思路" and "优化策略总结") have the target model
+ * validate candidate tokens obtained ahead of time, organised as a forest (multi-branch prediction),
+ * and count the candidates' hit length; they fix no acceptance rule. These calls implement the plain
+ * greedy one:
+ *  - candidate i is correct iff its token equals the target's argmax after its parent (after the
+ *    committed prefix for a root);
+ *  - a candidate is accepted iff it and all its ancestors are correct; the hit is the deepest accepted
+ *    candidate (the smallest index among equally deep ones) and the accepted path runs from its root
+ *    to it;
+ *  - the target's argmax after the hit (after the prefix when nothing is accepted) is one more token
+ *    the step emits (the bonus token);
+ *  - the accepted candidates' K/V move to the contiguous tail: the path's d-th node (0-based) goes to
+ *    logical slot P_b + d, P_b = L_b - n_b. Passing slot_offsets_out with the step's k_new / v_new to
+ *    paged_kv_append performs that move.
+ *
+ * tree_mask_from_parents: the tree_mask_bits of paged_tree_attention from parent links.
+ *   parents         int32 [B, C]; parents[b][i] = -1 (a root) or a candidate j < i
+ *   num_candidates  int32 [B]; n_b in [0, C]
+ *   mask_out        uint32 [B, C]; bit j of word (b, i) is set iff j is i or an ancestor of i; rows
+ *                   i >= n_b are 0
+ * C in 1..32. A parent outside [-1, i) sets TACO_DEVERR_PARENT and ends that row's walk.
+ */
+taco_status tree_mask_from_parents(const int32_t* parents, const int32_t* num_candidates, int32_t batch,
+                                   int32_t max_candidates, uint32_t* mask_out, void* stream);
+
+/*
+ * logits_argmax: per row of a [rows, vocab] matrix of 16-bit floats, the smallest index of the largest
+ * value. NaN never wins; a row without a number above -inf gives 0.
+ *   logits     [rows, vocab] dtype (TACO_DTYPE_F16 / TACO_DTYPE_BF16), dense
+ *   out_index  int32 [rows]
+ * rows >= 0, vocab >= 1. The pointer need not be 16-byte aligned (a slower kernel reads it then).
+ */
+taco_status logits_argmax(const void* logits, int32_t dtype, int64_t rows, int32_t vocab, int32_t* out_index,
+                          void* stream);
+
+/*
+ * tree_greedy_accept: acceptance of each sequence's candidate forest (rules above).
+ *   target_argmax     int32 [B, C + 1]; row 0: the target's argmax after the prefix, row i + 1: after
+ *                     candidate i (e.g. logits_argmax over [B, C + 1, vocab] logits)
+ *   candidate_tokens  int32 [B, C]
+ *   parents           int32 [B, C]; -1 or an earlier candidate
+ *   num_candidates    int32 [B]; n_b in [0, min(C, L_b)]
+ *   context_lens      int32 [B]; L_b as in paged_tree_attention (candidates included)
+ *   accept_len        int32 [B]; length of the accepted path (0..n_b)
+ *   accepted_path     int32 [B, C]; its nodes root first, -1 after accept_len
+ *   bonus_token       int32 [B]
+ *   slot_offsets_out  int32 [B, C]; P_b + d for the path's d-th node, -1 for every other candidate
+ * C in 1..32. Parents outside [-1, i) set TACO_DEVERR_PARENT (that candidate is treated as an
+ * incorrect root); n_b out of range sets TACO_DEVERR_NUM_CAND and is clamped.
+ */
+taco_status tree_greedy_accept(const int32_t* target_argmax, const int32_t* candidate_tokens,
+                               const int32_t* parents, const int32_t* num_candidates, const int32_t* context_lens,
+                               int32_t batch, int32_t max_candidates, int32_t* accept_len, int32_t* accepted_path,
+                               int32_t* bonus_token, int32_t* slot_offsets_out, void* stream);
 
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char* taco_attn_last_error(void);

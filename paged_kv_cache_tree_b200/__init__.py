@@ -9,10 +9,13 @@ from ._lib import (  # noqa: F401
     TacoError,
     check_device,
     load,
+    logits_argmax,
     paged_kv_append,
     paged_tree_attention,
     paged_tree_attention_noalloc,
     release_workspace,
     set_option,
+    tree_greedy_accept,
+    tree_mask_from_parents,
     version,
 )

@@ -37,6 +37,9 @@ EXPORTED = (
     "taco_attn_release_workspace",
     "taco_attn_set_option",
     "taco_attn_version",
+    "tree_mask_from_parents",
+    "logits_argmax",
+    "tree_greedy_accept",
 )
 
 _lib = None
@@ -73,6 +76,12 @@ def load() -> ctypes.CDLL:
     lib.taco_attn_set_option.restype = i32
     lib.taco_attn_version.argtypes = []
     lib.taco_attn_version.restype = i32
+    lib.tree_mask_from_parents.argtypes = [vp, vp, i32, i32, vp, vp]
+    lib.tree_mask_from_parents.restype = i32
+    lib.logits_argmax.argtypes = [vp, i32, ctypes.c_int64, i32, vp, vp]
+    lib.logits_argmax.restype = i32
+    lib.tree_greedy_accept.argtypes = [vp] * 5 + [i32, i32] + [vp] * 4 + [vp]
+    lib.tree_greedy_accept.restype = i32
     _lib = lib
     return lib
 
@@ -169,6 +178,65 @@ def paged_kv_append(k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, 
         k_new.data_ptr(), v_new.data_ptr(), block_tables.data_ptr(), slot_offsets.data_ptr(),
         k_cache.data_ptr(), v_cache.data_ptr(), _dtype_code(k_new), B, C, Hkv, D, bs, NB,
         block_tables.shape[1], _stream_handle(stream, k_new.device)))
+
+
+def tree_mask_from_parents(parents, num_candidates, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """parents int32 [B, C] (-1 = root); num_candidates int32 [B]. Returns uint32 bit patterns in an
+    int32 [B, C] tensor (the tree_mask_bits of paged_tree_attention)."""
+    _need_cuda("parents", parents, torch.int32, 2)
+    _need_cuda("num_candidates", num_candidates, torch.int32, 1)
+    B, C = parents.shape
+    if num_candidates.shape[0] != B:
+        raise ValueError("batch dimension mismatch")
+    if out is None:
+        out = torch.empty_like(parents)
+    _need_cuda("out", out, (torch.int32, torch.uint32), 2)
+    if tuple(out.shape) != (B, C):
+        raise ValueError("out must be [B, C]")
+    _check(load().tree_mask_from_parents(parents.data_ptr(), num_candidates.data_ptr(), B, C, out.data_ptr(),
+                                         _stream_handle(stream, parents.device)))
+    return out
+
+
+def logits_argmax(logits, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """logits [..., V] bf16/fp16 (dense). Returns int32 [...]: per row the smallest index of the largest
+    value (NaN never wins; a row without a number above -inf gives 0)."""
+    _need_cuda("logits", logits, (torch.bfloat16, torch.float16))
+    V = logits.shape[-1]
+    rows = logits.numel() // V if V > 0 else 0
+    if out is None:
+        out = torch.empty(logits.shape[:-1], dtype=torch.int32, device=logits.device)
+    _need_cuda("out", out, torch.int32)
+    if out.numel() != rows:
+        raise ValueError("out must have one entry per row")
+    _check(load().logits_argmax(logits.data_ptr(), _dtype_code(logits), rows, V, out.data_ptr(),
+                                _stream_handle(stream, logits.device)))
+    return out
+
+
+def tree_greedy_accept(target_argmax, candidate_tokens, parents, num_candidates, context_lens, stream=None):
+    """target_argmax int32 [B, C+1]; candidate_tokens, parents int32 [B, C]; num_candidates, context_lens
+    int32 [B]. Returns (accept_len [B], accepted_path [B, C], bonus_token [B], slot_offsets [B, C])."""
+    _need_cuda("target_argmax", target_argmax, torch.int32, 2)
+    _need_cuda("candidate_tokens", candidate_tokens, torch.int32, 2)
+    _need_cuda("parents", parents, torch.int32, 2)
+    _need_cuda("num_candidates", num_candidates, torch.int32, 1)
+    _need_cuda("context_lens", context_lens, torch.int32, 1)
+    B, C = candidate_tokens.shape
+    if tuple(parents.shape) != (B, C) or tuple(target_argmax.shape) != (B, C + 1):
+        raise ValueError("parents must be [B, C] and target_argmax [B, C + 1]")
+    if num_candidates.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("batch dimension mismatch")
+    dev = candidate_tokens.device
+    accept_len = torch.empty(B, dtype=torch.int32, device=dev)
+    path = torch.empty(B, C, dtype=torch.int32, device=dev)
+    bonus = torch.empty(B, dtype=torch.int32, device=dev)
+    slots = torch.empty(B, C, dtype=torch.int32, device=dev)
+    _check(load().tree_greedy_accept(
+        target_argmax.data_ptr(), candidate_tokens.data_ptr(), parents.data_ptr(), num_candidates.data_ptr(),
+        context_lens.data_ptr(), B, C, accept_len.data_ptr(), path.data_ptr(), bonus.data_ptr(), slots.data_ptr(),
+        _stream_handle(stream, dev)))
+    return accept_len, path, bonus, slots
 
 
 def check_device(stream=None, device=None) -> int:

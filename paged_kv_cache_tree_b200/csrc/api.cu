@@ -17,7 +17,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 
 thread_local std::string g_last_error;
 
@@ -337,6 +337,68 @@ taco_status paged_kv_append(const void* k_new, const void* v_new, const int32_t*
   return TACO_OK;
 }
 
+// Error word of the current device (creates the workspace's header on first use).
+static taco_status device_error_word(uint32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(TACO_ERR_UNSUPPORTED, "device index %d too large", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  taco_status st = ensure_workspace(dev, 0, 0, 0);
+  if (st != TACO_OK) return st;
+  *out = g_ws[dev].error_word;
+  return TACO_OK;
+}
+
+taco_status tree_mask_from_parents(const int32_t* parents, const int32_t* num_candidates, int32_t batch,
+                                   int32_t max_candidates, uint32_t* mask_out, void* stream) {
+  if (batch < 0) return fail(TACO_ERR_INVALID_ARG, "batch must be >= 0");
+  if (max_candidates < 1 || max_candidates > 32)
+    return fail(TACO_ERR_UNSUPPORTED, "max_candidates must be in 1..32 (one mask bit per candidate)");
+  if (!parents || !num_candidates || !mask_out) return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (batch == 0) return TACO_OK;
+  uint32_t* err = nullptr;
+  taco_status st = device_error_word(&err);
+  if (st != TACO_OK) return st;
+  taco::MaskArgs a{parents, num_candidates, mask_out, err, batch, max_candidates};
+  cudaError_t e = taco::launch_tree_masks(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tree mask kernel launch");
+  return TACO_OK;
+}
+
+taco_status logits_argmax(const void* logits, int32_t dtype, int64_t rows, int32_t vocab, int32_t* out_index,
+                          void* stream) {
+  if (dtype != TACO_DTYPE_F16 && dtype != TACO_DTYPE_BF16) return fail(TACO_ERR_INVALID_ARG, "dtype must be f16 or bf16");
+  if (rows < 0 || vocab < 1) return fail(TACO_ERR_INVALID_ARG, "need rows >= 0 and vocab >= 1");
+  if (rows > 0x7fffffff) return fail(TACO_ERR_UNSUPPORTED, "at most 2^31 - 1 rows per call");
+  if (!logits || !out_index) return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (rows == 0) return TACO_OK;
+  cudaError_t e = taco::launch_argmax(logits, dtype, rows, vocab, out_index, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "argmax kernel launch");
+  return TACO_OK;
+}
+
+taco_status tree_greedy_accept(const int32_t* target_argmax, const int32_t* candidate_tokens,
+                               const int32_t* parents, const int32_t* num_candidates, const int32_t* context_lens,
+                               int32_t batch, int32_t max_candidates, int32_t* accept_len, int32_t* accepted_path,
+                               int32_t* bonus_token, int32_t* slot_offsets_out, void* stream) {
+  if (batch < 0) return fail(TACO_ERR_INVALID_ARG, "batch must be >= 0");
+  if (max_candidates < 1 || max_candidates > 32)
+    return fail(TACO_ERR_UNSUPPORTED, "max_candidates must be in 1..32 (one lane per candidate)");
+  if (!target_argmax || !candidate_tokens || !parents || !num_candidates || !context_lens || !accept_len ||
+      !accepted_path || !bonus_token || !slot_offsets_out)
+    return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (batch == 0) return TACO_OK;
+  uint32_t* err = nullptr;
+  taco_status st = device_error_word(&err);
+  if (st != TACO_OK) return st;
+  taco::AcceptArgs a{target_argmax, candidate_tokens, parents, num_candidates, context_lens, accept_len,
+                     accepted_path, bonus_token, slot_offsets_out, err, batch, max_candidates};
+  cudaError_t e = taco::launch_accept(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "accept kernel launch");
+  return TACO_OK;
+}
+
 taco_status taco_attn_check_device(void* stream, uint32_t* bits_out) {
   if (bits_out) *bits_out = 0;
   int dev = 0;
@@ -355,12 +417,13 @@ taco_status taco_attn_check_device(void* stream, uint32_t* bits_out) {
   if (bits == 0) return TACO_OK;
   cudaMemset(w.error_word, 0, 4);
   if (bits & TACO_DEVERR_WAIT_TIMEOUT) cudaMemset(w.counters, 0, w.counters_cap * 4);
-  return fail(TACO_ERR_DEVICE_CHECK, "device range check failed: bits 0x%x%s%s%s%s%s", bits,
+  return fail(TACO_ERR_DEVICE_CHECK, "device range check failed: bits 0x%x%s%s%s%s%s%s", bits,
               (bits & TACO_DEVERR_BLOCK_ID) ? " [block id out of range]" : "",
               (bits & TACO_DEVERR_CONTEXT_LEN) ? " [context length out of range]" : "",
               (bits & TACO_DEVERR_NUM_CAND) ? " [candidate count out of range]" : "",
               (bits & TACO_DEVERR_SLOT) ? " [slot out of range]" : "",
-              (bits & TACO_DEVERR_WAIT_TIMEOUT) ? " [pipeline wait timed out]" : "");
+              (bits & TACO_DEVERR_WAIT_TIMEOUT) ? " [pipeline wait timed out]" : "",
+              (bits & TACO_DEVERR_PARENT) ? " [parent index out of range]" : "");
 }
 
 void taco_attn_release_workspace(void) {

@@ -22,6 +22,32 @@ struct AppendArgs {
   int B, C, Hkv, D, bs, num_blocks, max_blocks;
 };
 
+struct MaskArgs {
+  const int32_t* parents;
+  const int32_t* num_candidates;
+  uint32_t* mask_out;
+  uint32_t* error_word;
+  int B, C;
+};
+
+struct AcceptArgs {
+  const int32_t* target_argmax;
+  const int32_t* tokens;
+  const int32_t* parents;
+  const int32_t* num_candidates;
+  const int32_t* context_lens;
+  int32_t* accept_len;
+  int32_t* accepted_path;
+  int32_t* bonus_token;
+  int32_t* slot_offsets_out;
+  uint32_t* error_word;
+  int B, C;
+};
+
+cudaError_t launch_tree_masks(const MaskArgs& a, cudaStream_t stream);
+cudaError_t launch_argmax(const void* logits, int dtype, int64_t rows, int vocab, int32_t* out, cudaStream_t stream);
+cudaError_t launch_accept(const AcceptArgs& a, cudaStream_t stream);
+
 // Rows of packed queries one unit of the mma.sync verify kernel covers for a given G * C.
 int mma_rows_per_unit(int packed_rows);
 // Dynamic shared memory the mma.sync verify kernel needs.

@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.taco_attn_version() == 1
+    assert lib.taco_attn_version() == 2
 
 
 def _attn_args(**over):
@@ -90,3 +90,27 @@ def test_options(lib):
     assert lib.taco_attn_set_option(_lib.TACO_OPT_GRID_CTAS, 0) == _lib.TACO_OK
     assert lib.taco_attn_set_option(_lib.TACO_OPT_KERNEL, 5) == _lib.TACO_ERR_INVALID_ARG
     assert lib.taco_attn_set_option(99, 1) == _lib.TACO_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("call,status", [
+    (lambda l: l.tree_mask_from_parents(None, 16, 2, 4, 16, None), _lib.TACO_ERR_INVALID_ARG),
+    (lambda l: l.tree_mask_from_parents(16, 16, 2, 33, 16, None), _lib.TACO_ERR_UNSUPPORTED),
+    (lambda l: l.tree_mask_from_parents(16, 16, -1, 4, 16, None), _lib.TACO_ERR_INVALID_ARG),
+    (lambda l: l.logits_argmax(None, 1, 4, 100, 16, None), _lib.TACO_ERR_INVALID_ARG),
+    (lambda l: l.logits_argmax(16, 5, 4, 100, 16, None), _lib.TACO_ERR_INVALID_ARG),
+    (lambda l: l.logits_argmax(16, 1, 4, 0, 16, None), _lib.TACO_ERR_INVALID_ARG),
+    (lambda l: l.logits_argmax(16, 1, -2, 10, 16, None), _lib.TACO_ERR_INVALID_ARG),
+    (lambda l: l.tree_greedy_accept(16, 16, 16, 16, 16, 2, 0, 16, 16, 16, 16, None), _lib.TACO_ERR_UNSUPPORTED),
+    (lambda l: l.tree_greedy_accept(16, 16, 16, 16, 16, 2, 40, 16, 16, 16, 16, None), _lib.TACO_ERR_UNSUPPORTED),
+    (lambda l: l.tree_greedy_accept(16, None, 16, 16, 16, 2, 4, 16, 16, 16, 16, None), _lib.TACO_ERR_INVALID_ARG),
+    (lambda l: l.tree_greedy_accept(16, 16, 16, 16, 16, 2, 4, 16, 16, 16, None, None), _lib.TACO_ERR_INVALID_ARG),
+])
+def test_acceptance_calls_reject_bad_arguments_on_host(lib, call, status):
+    assert call(lib) == status
+    assert lib.taco_attn_last_error().decode()
+
+
+def test_acceptance_calls_with_nothing_to_do_are_no_ops(lib):
+    assert lib.tree_mask_from_parents(16, 16, 0, 4, 16, None) == _lib.TACO_OK
+    assert lib.logits_argmax(16, 1, 0, 100, 16, None) == _lib.TACO_OK
+    assert lib.tree_greedy_accept(16, 16, 16, 16, 16, 0, 4, 16, 16, 16, 16, None) == _lib.TACO_OK
