@@ -248,6 +248,51 @@ def run_reference(args, world, rank):
     return line
 
 
+def measure_accept(taco, w, d, dev, stream, args):
+    """The step after the verify, timed on its own: argmax of the target's logits over the vocabulary,
+    greedy acceptance, and the compaction append of the accepted candidates' K/V. The logits
+    ([B, C + 1, 128256], 33-70 MB) fit in L2, so L2 is flushed before each timed iteration by reading a
+    256 MB buffer (a read leaves clean lines: a write would make the next kernel pay for writing back
+    L2's dirty lines); each launch is timed with CUDA events on its stream."""
+    a = wl.make_accept_inputs(w)
+    logits = a.target_logits.to(dev)
+    tokens = a.tokens.to(dev)
+    amax = torch.empty(w.B, w.C + 1, dtype=torch.int32, device=dev)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    steps = max(10, min(args.steps, 200))
+    t_arg, t_acc, t_app = [], [], []
+    acc_len = None
+    for it in range(args.warmup + steps):
+        flush.sum()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        taco.logits_argmax(logits, out=amax, stream=stream)
+        ev[1].record(stream)
+        acc_len, path, bonus, slots = taco.tree_greedy_accept(amax, tokens, d.parents, d.num_candidates,
+                                                              d.context_lens, stream=stream)
+        ev[2].record(stream)
+        taco.paged_kv_append(d.k_new, d.v_new, d.block_tables, slots, d.k_cache, d.v_cache, stream=stream)
+        ev[3].record(stream)
+        torch.cuda.synchronize(dev)
+        if it >= args.warmup:
+            t_arg.append(ev[0].elapsed_time(ev[1]))
+            t_acc.append(ev[1].elapsed_time(ev[2]))
+            t_app.append(ev[2].elapsed_time(ev[3]))
+    taco.check_device(stream)
+    med = lambda x: statistics.median(x)
+    arg_bytes = a.logits_bytes() + amax.numel() * 4
+    return {
+        "vocab": a.vocab, "logits_bytes": a.logits_bytes(),
+        "argmax_us": 1e3 * med(t_arg), "accept_us": 1e3 * med(t_acc), "compaction_append_us": 1e3 * med(t_app),
+        "argmax_roofline": {"bound": "hbm", "achieved": arg_bytes / (med(t_arg) * 1e-3) / 1e9, "unit": "GB/s",
+                            "traffic": None},
+        "mean_accept_len": float(acc_len.float().mean().item()),
+        "tokens_per_step": float(acc_len.float().sum().item()) + w.B,
+        "l2": "flushed before each iteration (256 MB read)",
+        "inputs": "seeded synthetic logits with a planted maximum per row; candidate hits with p = 0.7",
+    }
+
+
 def run_ours(args, world, rank, local):
     import paged_kv_cache_tree_b200 as taco
 
@@ -327,6 +372,8 @@ def run_ours(args, world, rank, local):
     taco.check_device(stream)
     e2e_value = world * nbytes / (e2e_ms * 1e-3) / 1e9
 
+    accept = measure_accept(taco, w, d, dev, stream, args)
+
     if rank != 0:
         return None
     peak, peak_kind = measured_peaks()
@@ -350,7 +397,10 @@ def run_ours(args, world, rank, local):
                 "ms_per_step": e2e_ms},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
+        "accept": accept,
     }
+    accept["argmax_roofline"]["peak"] = peak
+    accept["argmax_roofline"]["frac"] = accept["argmax_roofline"]["achieved"] / peak
     if world == 1 and not args.no_cpu_baseline:
         nb, ncnd, secs, desc = oracle_sample(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
