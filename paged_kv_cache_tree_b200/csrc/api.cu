@@ -370,7 +370,7 @@ taco_status logits_argmax(const void* logits, int32_t dtype, int64_t rows, int32
                           void* stream) {
   if (dtype != TACO_DTYPE_F16 && dtype != TACO_DTYPE_BF16) return fail(TACO_ERR_INVALID_ARG, "dtype must be f16 or bf16");
   if (rows < 0 || vocab < 1) return fail(TACO_ERR_INVALID_ARG, "need rows >= 0 and vocab >= 1");
-  if (rows > (1ll << 27)) return fail(TACO_ERR_UNSUPPORTED, "at most 2^27 rows per call");
+  if (rows > 0x7fffffff) return fail(TACO_ERR_UNSUPPORTED, "at most 2^31 - 1 rows per call");
   if (!logits || !out_index) return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
   if (rows == 0) return TACO_OK;
   cudaError_t e = taco::launch_argmax(logits, dtype, rows, vocab, out_index, static_cast<cudaStream_t>(stream));
