@@ -12,7 +12,9 @@ value        = algorithmic bytes of the step / device time per step, summed over
                each appended K/V row.
 e2e          = the same metric through the public Python API with the step's per-call inputs
                (q, k_new, v_new, tables, lengths, masks, slots) copied host->device from pinned memory
-               and the output copied back, every step; the KV cache is device-resident state.
+               and the output copied back, every step; the KV cache is device-resident state. The
+               copies run on their own streams with two buffer sets, so step k's transfers overlap the
+               kernels of steps k - 1 and k + 1.
 roofline     = the attention kernel alone: its algorithmic bytes / its mean launch time (CUDA events on
                its stream) against the measured HBM copy bandwidth.
 cpu_baseline = the CPU oracle (fp64 NumPy) timed on a bounded sample of the same workload.
@@ -340,32 +342,54 @@ def run_ours(args, world, rank, local):
     ms_per_step = region_ms / args.steps
     value = world * nbytes / (ms_per_step * 1e-3) / 1e9
 
-    # ---- end to end through the public API with host buffers
-    host = {k: getattr(w, k).pin_memory() for k in ("q", "k_new", "v_new", "block_tables", "context_lens",
-                                                     "num_candidates", "tree_mask", "slot_offsets")}
-    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
-    out_host = torch.empty(w.q.shape, dtype=w.q.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_host.numel() * out_host.element_size()
+    # ---- end to end through the public API with host buffers. Two sets of buffers: step k's inputs
+    # are copied host->device on one stream and its output device->host on another, overlapping the
+    # kernels of the neighbouring steps on the compute stream; events order every buffer's reuse.
+    host_keys = ("q", "k_new", "v_new", "block_tables", "context_lens", "num_candidates", "tree_mask", "slot_offsets")
+    hosts = [{k: getattr(w, k).pin_memory() for k in host_keys} for _ in range(2)]
+    dev_in = [{k: torch.empty_like(v, device=dev) for k, v in hosts[0].items()} for _ in range(2)]
+    out_dev = [torch.empty_like(d.q) for _ in range(2)]
+    out_host = [torch.empty(w.q.shape, dtype=w.q.dtype).pin_memory() for _ in range(2)]
+    h2d = sum(v.numel() * v.element_size() for v in hosts[0].values())
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    s_h2d = torch.cuda.Stream(dev)
+    s_d2h = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of the slot landed
+    ev_used = [torch.cuda.Event() for _ in range(2)]   # the slot's kernels finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # the slot's output is on the host
 
-    def e2e_step():
-        for k, v in host.items():
-            dev_in[k].copy_(v, non_blocking=True)
-        taco.paged_kv_append(dev_in["k_new"], dev_in["v_new"], dev_in["block_tables"], dev_in["slot_offsets"],
-                             d.k_cache, d.v_cache, stream=stream)
-        taco.paged_tree_attention(dev_in["q"], d.k_cache, d.v_cache, dev_in["block_tables"], dev_in["context_lens"],
-                                  dev_in["num_candidates"], dev_in["tree_mask"], w.scale, out=out, stream=stream)
-        out_host.copy_(out, non_blocking=True)
+    def e2e_step(k):
+        j = k % 2
+        with torch.cuda.stream(s_h2d):
+            s_h2d.wait_event(ev_used[j])               # step k - 2 no longer reads these inputs
+            for key, v in hosts[j].items():
+                dev_in[j][key].copy_(v, non_blocking=True)
+            ev_in[j].record(s_h2d)
+        stream.wait_event(ev_in[j])
+        stream.wait_event(ev_out[j])                   # step k - 2's output has left this buffer
+        di = dev_in[j]
+        taco.paged_kv_append(di["k_new"], di["v_new"], di["block_tables"], di["slot_offsets"], d.k_cache, d.v_cache,
+                             stream=stream)
+        taco.paged_tree_attention(di["q"], d.k_cache, d.v_cache, di["block_tables"], di["context_lens"],
+                                  di["num_candidates"], di["tree_mask"], w.scale, out=out_dev[j], stream=stream)
+        ev_used[j].record(stream)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(ev_used[j])
+            out_host[j].copy_(out_dev[j], non_blocking=True)
+            ev_out[j].record(s_d2h)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    for k in range(args.warmup):
+        e2e_step(k)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    s_h2d.wait_event(e0)
+    for k in range(args.steps):
+        e2e_step(k)
+    stream.wait_event(ev_out[(args.steps - 1) % 2])
+    stream.wait_event(ev_out[(args.steps - 2) % 2] if args.steps > 1 else ev_out[(args.steps - 1) % 2])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
