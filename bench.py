@@ -412,6 +412,8 @@ def run_ours(args, world, rank, local):
                    "candidate_tokens_per_step": w.candidate_tokens(),
                    "l2": "inputs larger than L2 (KV cache > 126 MB), no flush", "parallelism": f"dp{world} (independent batches)"},
         "candidate_tokens_per_s": world * w.candidate_tokens() / (ms_per_step * 1e-3),
+        # the same rate at the roofline: every step's bytes moved at the measured copy bandwidth
+        "candidate_tokens_per_s_at_roofline": world * w.candidate_tokens() * measured_peaks()[0] * 1e9 / nbytes,
         "hbm_frac_of_measured": value / world / peak,
         "hbm_frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
