@@ -9,3 +9,4 @@ from .paged_attention import (  # noqa: F401
     within_tolerance,
 )
 from . import tree_accept  # noqa: F401,E402
+from . import fp8  # noqa: F401,E402

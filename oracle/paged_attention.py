@@ -94,16 +94,28 @@ def softmax_attend(q_row: np.ndarray, keys: np.ndarray, values: np.ndarray, visi
     return (w @ values[visible]) / w.sum()
 
 
+def _widen_kv(x: np.ndarray, kv_dtype: str, scale, g: int) -> np.ndarray:
+    """K or V rows of KV head g as float64: 16-bit floats widen exactly; e4m3 codes decode and take
+    the head's scale (see ``oracle.fp8``)."""
+    if kv_dtype == "e4m3":
+        from .fp8 import e4m3_decode
+
+        return e4m3_decode(x) * float(np.asarray(scale, dtype=np.float64)[g])
+    return widen_to_f64(x, kv_dtype)
+
+
 def paged_tree_attention(q, k_cache, v_cache, block_tables, context_lens, num_candidates,
-                         tree_mask_bits, scale, dtype, rows=None):
+                         tree_mask_bits, scale, dtype, rows=None, kv_dtype=None, k_scale=None, v_scale=None):
     """Oracle of the verify attention.
 
-    q: uint16 bits [B, C, Hq, D]; k_cache, v_cache: uint16 bits [NB, Hkv, bs, D];
+    q: uint16 bits [B, C, Hq, D]; k_cache, v_cache: uint16 bits [NB, Hkv, bs, D] (or uint8 e4m3
+    codes with ``kv_dtype="e4m3"`` and per-KV-head float scales ``k_scale`` / ``v_scale``);
     block_tables: int [B, maxblk]; context_lens, num_candidates: int [B];
-    tree_mask_bits: uint32 [B, C]; dtype: "bf16" | "fp16".
+    tree_mask_bits: uint32 [B, C]; dtype: "bf16" | "fp16" (of q, and of K/V unless kv_dtype is given).
     rows: optional iterable of (b, i, h) to evaluate; other rows are left as NaN.
     Returns float64 [B, C, Hq, D] (not rounded to the storage dtype).
     """
+    kvd = dtype if kv_dtype is None else kv_dtype
     B, C, Hq, D = q.shape
     Hkv, bs = k_cache.shape[1], k_cache.shape[2]
     G = Hq // Hkv
@@ -120,8 +132,8 @@ def paged_tree_attention(q, k_cache, v_cache, block_tables, context_lens, num_ca
         for g in range(Hkv):
             if want is not None and (b, g) not in want:
                 continue
-            K = widen_to_f64(gather_sequence_kv(k_cache, block_tables[b], g, L, bs), dtype)
-            V = widen_to_f64(gather_sequence_kv(v_cache, block_tables[b], g, L, bs), dtype)
+            K = _widen_kv(gather_sequence_kv(k_cache, block_tables[b], g, L, bs), kvd, k_scale, g)
+            V = _widen_kv(gather_sequence_kv(v_cache, block_tables[b], g, L, bs), kvd, v_scale, g)
             pairs = want[(b, g)] if want is not None else [(i, h) for i in range(C)
                                                               for h in range(g * G, (g + 1) * G)]
             for (i, h) in pairs:
