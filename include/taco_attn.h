@@ -139,6 +139,46 @@ taco_status paged_tree_attention_noalloc(const void* q, const void* k_cache, con
                                          void* stream);
 
 /*
+ * 8-bit KV cache. The 53ai.com workshop page (section "5. 支持 Quantization（模型量化）") lists 8-bit
+ * (INT8 / FP8) storage among the engine's features for its lower memory and bandwidth needs, and the
+ * 17173xz.com overview counts quantised operators among its kernels; neither fixes a format. These
+ * calls use e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinities; 0x7F / 0xFF
+ * are NaN; largest finite 448) with one float32 scale per KV head for K and one for V:
+ *   stored code  = e4m3(x / scale[h])  (float32 quotient correctly rounded, then the nearest e4m3 value,
+ *                  ties to the even code, magnitudes above 448 saturate to 448, NaN stays NaN)
+ *   value read   = decode(code) * scale[h]
+ * The cache layout is [NB, Hkv, bs, D] with one byte per element.
+ *
+ * paged_kv_append_e4m3: paged_kv_append into e4m3 caches. k_new / v_new are [B, C, Hkv, D] `dtype`
+ * (F16 / BF16); k_scale, v_scale are device float32 [Hkv] (finite and nonzero: not checked). Every
+ * other argument and rule is that of paged_kv_append; D is 64 or 128.
+ */
+taco_status paged_kv_append_e4m3(const void* k_new, const void* v_new, const int32_t* block_tables,
+                                 const int32_t* slot_offsets, const float* k_scale, const float* v_scale,
+                                 void* k_cache, void* v_cache, int32_t dtype, int32_t batch,
+                                 int32_t max_candidates, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                 void* stream);
+
+/*
+ * paged_tree_attention_e4m3: paged_tree_attention over e4m3 caches (layout and scales as above): the
+ * result is that of paged_tree_attention with K = decode(k_cache) * k_scale[h] and V = decode(v_cache) *
+ * v_scale[h]. q and out are `dtype` (F16 / BF16). Supported: head_dim 128 and packed query rows
+ * (num_q_heads / num_kv_heads) * max_candidates <= 64; other sizes return TACO_ERR_UNSUPPORTED. The
+ * workspace rules of paged_tree_attention apply. k_scale, v_scale: device float32 [Hkv], finite and
+ * nonzero (not checked).
+ */
+taco_status paged_tree_attention_e4m3(const void* q, const void* k_cache, const void* v_cache,
+                                      const float* k_scale, const float* v_scale,
+                                      const int32_t* block_tables, const int32_t* context_lens,
+                                      const int32_t* num_candidates, const uint32_t* tree_mask_bits,
+                                      float scale, void* out,
+                                      int32_t dtype, int32_t batch, int32_t max_candidates,
+                                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                      void* stream);
+
+/*
  * The step after the verify. The pages ("大模型倍速推理引擎 TACO-LLM 的设计与实践", sections
  * "TACO-LLM 如何解决大模型推理瓶颈?", "优化方案设计思路" and "优化策略总结") have the target model
  * validate candidate tokens obtained ahead of time, organised as a forest (multi-branch prediction),

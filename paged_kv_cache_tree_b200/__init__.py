@@ -11,7 +11,9 @@ from ._lib import (  # noqa: F401
     load,
     logits_argmax,
     paged_kv_append,
+    paged_kv_append_e4m3,
     paged_tree_attention,
+    paged_tree_attention_e4m3,
     paged_tree_attention_noalloc,
     release_workspace,
     set_option,

@@ -32,6 +32,8 @@ EXPORTED = (
     "paged_tree_attention",
     "paged_kv_append",
     "paged_tree_attention_noalloc",
+    "paged_tree_attention_e4m3",
+    "paged_kv_append_e4m3",
     "taco_attn_last_error",
     "taco_attn_check_device",
     "taco_attn_release_workspace",
@@ -66,6 +68,10 @@ def load() -> ctypes.CDLL:
     lib.paged_tree_attention_noalloc.restype = i32
     lib.paged_kv_append.argtypes = [vp] * 6 + [i32] * 8 + [vp]
     lib.paged_kv_append.restype = i32
+    lib.paged_tree_attention_e4m3.argtypes = [vp] * 9 + [f32, vp] + [i32] * 9 + [vp]
+    lib.paged_tree_attention_e4m3.restype = i32
+    lib.paged_kv_append_e4m3.argtypes = [vp] * 8 + [i32] * 8 + [vp]
+    lib.paged_kv_append_e4m3.restype = i32
     lib.taco_attn_last_error.argtypes = []
     lib.taco_attn_last_error.restype = ctypes.c_char_p
     lib.taco_attn_check_device.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -177,6 +183,70 @@ def paged_kv_append(k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, 
     _check(lib.paged_kv_append(
         k_new.data_ptr(), v_new.data_ptr(), block_tables.data_ptr(), slot_offsets.data_ptr(),
         k_cache.data_ptr(), v_cache.data_ptr(), _dtype_code(k_new), B, C, Hkv, D, bs, NB,
+        block_tables.shape[1], _stream_handle(stream, k_new.device)))
+
+
+def _need_scales(k_scale, v_scale, Hkv: int) -> None:
+    for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+        _need_cuda(name, t, torch.float32, 1)
+        if t.shape[0] != Hkv:
+            raise ValueError(f"{name} must be float32 [num_kv_heads]")
+
+
+def paged_tree_attention_e4m3(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_candidates,
+                              tree_mask_bits, scale: float, out: Optional[torch.Tensor] = None,
+                              stream=None) -> torch.Tensor:
+    """Attention over e4m3 caches: q [B,C,Hq,D] bf16/fp16; k/v_cache uint8 [NB,Hkv,bs,D] e4m3 codes;
+    k_scale / v_scale float32 [Hkv] (value = decode(code) * scale[h]). Returns ``out`` (q's dtype)."""
+    _need_cuda("q", q, (torch.bfloat16, torch.float16), 4)
+    _need_cuda("k_cache", k_cache, torch.uint8, 4)
+    _need_cuda("v_cache", v_cache, torch.uint8, 4)
+    _need_cuda("block_tables", block_tables, torch.int32, 2)
+    _need_cuda("context_lens", context_lens, torch.int32, 1)
+    _need_cuda("num_candidates", num_candidates, torch.int32, 1)
+    _need_cuda("tree_mask_bits", tree_mask_bits, (torch.int32, torch.uint32), 2)
+    B, C, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache / v_cache shape mismatch with q")
+    if block_tables.shape[0] != B or context_lens.shape[0] != B or num_candidates.shape[0] != B:
+        raise ValueError("batch dimension mismatch")
+    if tuple(tree_mask_bits.shape) != (B, C):
+        raise ValueError("tree_mask_bits must be [B, C]")
+    _need_scales(k_scale, v_scale, Hkv)
+    if out is None:
+        out = torch.empty_like(q)
+    _need_cuda("out", out, q.dtype, 4)
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must have q's shape")
+    _check(load().paged_tree_attention_e4m3(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(),
+        block_tables.data_ptr(), context_lens.data_ptr(), num_candidates.data_ptr(), tree_mask_bits.data_ptr(),
+        float(scale), out.data_ptr(), _dtype_code(q), B, C, Hq, Hkv, D, bs, NB, block_tables.shape[1],
+        _stream_handle(stream, q.device)))
+    return out
+
+
+def paged_kv_append_e4m3(k_new, v_new, block_tables, slot_offsets, k_scale, v_scale, k_cache, v_cache,
+                         stream=None) -> None:
+    """Quantising append: k_new, v_new [B,C,Hkv,D] bf16/fp16; k/v_cache uint8 [NB,Hkv,bs,D] e4m3 codes,
+    updated in place with e4m3(x / scale[h]); slot_offsets int32 [B,C] (-1 = skip)."""
+    _need_cuda("k_new", k_new, (torch.bfloat16, torch.float16), 4)
+    _need_cuda("v_new", v_new, k_new.dtype, 4)
+    _need_cuda("block_tables", block_tables, torch.int32, 2)
+    _need_cuda("slot_offsets", slot_offsets, torch.int32, 2)
+    _need_cuda("k_cache", k_cache, torch.uint8, 4)
+    _need_cuda("v_cache", v_cache, torch.uint8, 4)
+    B, C, Hkv, D = k_new.shape
+    NB, Hkv2, bs, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(v_new.shape) != tuple(k_new.shape):
+        raise ValueError("shape mismatch between new rows and caches")
+    if tuple(slot_offsets.shape) != (B, C) or block_tables.shape[0] != B:
+        raise ValueError("slot_offsets must be [B, C] and block_tables [B, maxblk]")
+    _need_scales(k_scale, v_scale, Hkv)
+    _check(load().paged_kv_append_e4m3(
+        k_new.data_ptr(), v_new.data_ptr(), block_tables.data_ptr(), slot_offsets.data_ptr(), k_scale.data_ptr(),
+        v_scale.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), _dtype_code(k_new), B, C, Hkv, D, bs, NB,
         block_tables.shape[1], _stream_handle(stream, k_new.device)))
 
 

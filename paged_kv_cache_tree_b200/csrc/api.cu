@@ -17,7 +17,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 
 thread_local std::string g_last_error;
 
@@ -116,17 +116,21 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [NB * Hkv * bs rows, D columns] view of a cache; box = 64 columns (one 128-byte swizzle row) x
-// rows_per_chunk rows.
-taco_status make_cache_map(CUtensorMap* map, const void* base, int dtype, int D, int64_t rows, int rows_per_chunk) {
+// [NB * Hkv * bs rows, D columns] view of a cache; box = one 128-byte swizzle row (64 16-bit values,
+// or 128 e4m3 codes when kv8) x rows_per_chunk rows.
+taco_status make_cache_map(CUtensorMap* map, const void* base, int dtype, int D, int64_t rows, int rows_per_chunk,
+                           bool kv8 = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int elt = kv8 ? 1 : 2;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(rows_per_chunk)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * elt};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elt), static_cast<cuuint32_t>(rows_per_chunk)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, dtype == TACO_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                   2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  const CUtensorMapDataType ty = kv8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                     : (dtype == TACO_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  CUresult r = enc(map, ty, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return TACO_OK;
@@ -199,12 +203,14 @@ taco_status taco_attn_set_option(int32_t key, int64_t value) {
   return fail(TACO_ERR_INVALID_ARG, "unknown option key %d", key);
 }
 
-taco_status paged_tree_attention(const void* q, const void* k_cache, const void* v_cache,
-                                 const int32_t* block_tables, const int32_t* context_lens,
-                                 const int32_t* num_candidates, const uint32_t* tree_mask_bits, float scale,
-                                 void* out, int32_t dtype, int32_t batch, int32_t max_candidates,
-                                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
-                                 int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
+// Both attention entry points; k_scale / v_scale non-null selects e4m3 caches.
+static taco_status attention_impl(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                                  const float* v_scale, const int32_t* block_tables, const int32_t* context_lens,
+                                  const int32_t* num_candidates, const uint32_t* tree_mask_bits, float scale,
+                                  void* out, int32_t dtype, int32_t batch, int32_t max_candidates,
+                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                  int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
+  const bool kv8 = k_scale != nullptr;
   taco_status st = check_common(dtype, batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks,
                                 max_blocks_per_seq);
   if (st != TACO_OK) return st;
@@ -212,6 +218,13 @@ taco_status paged_tree_attention(const void* q, const void* k_cache, const void*
     return fail(TACO_ERR_INVALID_ARG, "num_q_heads must be a positive multiple of num_kv_heads");
   if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !num_candidates || !tree_mask_bits || !out)
     return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (kv8) {
+    if (!v_scale) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (v_scale)");
+    if (head_dim != 128) return fail(TACO_ERR_UNSUPPORTED, "e4m3 caches: head_dim must be 128");
+    if ((num_q_heads / num_kv_heads) * max_candidates > 64)
+      return fail(TACO_ERR_UNSUPPORTED, "e4m3 caches: (num_q_heads / num_kv_heads) * max_candidates must be <= 64");
+    if (g_opt_kernel == 2) return fail(TACO_ERR_UNSUPPORTED, "e4m3 caches have no tensor-core (tcgen05) kernel");
+  }
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return fail(TACO_ERR_INVALID_ARG, "q, k_cache, v_cache and out must be 16-byte aligned");
   if (!(scale == scale)) return fail(TACO_ERR_INVALID_ARG, "scale is NaN");
@@ -229,7 +242,7 @@ taco_status paged_tree_attention(const void* q, const void* k_cache, const void*
   // kernel choice: the tcgen05 path once the packed (GQA group x candidates) tile is wide enough to
   // keep tensor cores busy; the mma.sync path for narrow tiles
   const bool tc_possible = G <= 128;
-  bool use_tc = tc_possible && packed >= 48;
+  bool use_tc = tc_possible && packed >= 48 && !kv8;
   if (g_opt_kernel == 1) use_tc = false;
   if (g_opt_kernel == 2) {
     if (!tc_possible) return fail(TACO_ERR_UNSUPPORTED, "tensor-core path needs num_q_heads / num_kv_heads <= 128");
@@ -257,13 +270,13 @@ taco_status paged_tree_attention(const void* q, const void* k_cache, const void*
   if (st != TACO_OK) return st;
   Workspace& w = g_ws[dev];
 
-  const int tile = use_tc ? taco::tc_tile_keys() : taco::kTileKeys;
+  const int tile = use_tc ? taco::tc_tile_keys() : taco::mma_tile_keys(rows, kv8);
   const int rpc = block_size < tile ? block_size : tile;
   const int64_t cache_rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
   CUtensorMap tk, tv, tq;
-  st = make_cache_map(&tk, k_cache, dtype, head_dim, cache_rows, rpc);
+  st = make_cache_map(&tk, k_cache, dtype, head_dim, cache_rows, rpc, kv8);
   if (st != TACO_OK) return st;
-  st = make_cache_map(&tv, v_cache, dtype, head_dim, cache_rows, rpc);
+  st = make_cache_map(&tv, v_cache, dtype, head_dim, cache_rows, rpc, kv8);
   if (st != TACO_OK) return st;
   if (use_tc) {
     st = make_query_map(&tq, q, dtype, head_dim, num_q_heads, static_cast<int64_t>(batch) * max_candidates, G,
@@ -295,7 +308,9 @@ taco_status paged_tree_attention(const void* q, const void* k_cache, const void*
   p.rows_per_unit = rows;
   p.row_groups = row_groups;
   p.cands_per_group = cands_per_group;
-  p.tile_keys = use_tc ? taco::tc_tile_keys() : taco::kTileKeys;
+  p.tile_keys = tile;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
 
   if (use_tc) {
     e = taco::launch_verify_tc(tk, tv, tq, p, dtype, grid, static_cast<cudaStream_t>(stream));
@@ -305,6 +320,30 @@ taco_status paged_tree_attention(const void* q, const void* k_cache, const void*
   e = taco::launch_verify_mma(tk, tv, p, dtype, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "verify kernel launch");
   return TACO_OK;
+}
+
+taco_status paged_tree_attention(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* block_tables, const int32_t* context_lens,
+                                 const int32_t* num_candidates, const uint32_t* tree_mask_bits, float scale,
+                                 void* out, int32_t dtype, int32_t batch, int32_t max_candidates,
+                                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
+  return attention_impl(q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens, num_candidates,
+                        tree_mask_bits, scale, out, dtype, batch, max_candidates, num_q_heads, num_kv_heads,
+                        head_dim, block_size, num_blocks, max_blocks_per_seq, stream);
+}
+
+taco_status paged_tree_attention_e4m3(const void* q, const void* k_cache, const void* v_cache,
+                                      const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                      const int32_t* context_lens, const int32_t* num_candidates,
+                                      const uint32_t* tree_mask_bits, float scale, void* out, int32_t dtype,
+                                      int32_t batch, int32_t max_candidates, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                      int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
+  if (!k_scale || !v_scale) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (k_scale / v_scale)");
+  return attention_impl(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_candidates,
+                        tree_mask_bits, scale, out, dtype, batch, max_candidates, num_q_heads, num_kv_heads,
+                        head_dim, block_size, num_blocks, max_blocks_per_seq, stream);
 }
 
 taco_status paged_kv_append(const void* k_new, const void* v_new, const int32_t* block_tables,
@@ -333,6 +372,39 @@ taco_status paged_kv_append(const void* k_new, const void* v_new, const int32_t*
   taco::AppendArgs a{k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, err,
                      batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq};
   e = taco::launch_append(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+  return TACO_OK;
+}
+
+taco_status paged_kv_append_e4m3(const void* k_new, const void* v_new, const int32_t* block_tables,
+                                 const int32_t* slot_offsets, const float* k_scale, const float* v_scale,
+                                 void* k_cache, void* v_cache, int32_t dtype, int32_t batch,
+                                 int32_t max_candidates, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                 void* stream) {
+  taco_status st = check_common(dtype, batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks,
+                                max_blocks_per_seq);
+  if (st != TACO_OK) return st;
+  if (!k_new || !v_new || !block_tables || !slot_offsets || !k_scale || !v_scale || !k_cache || !v_cache)
+    return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(TACO_ERR_INVALID_ARG, "k_new, v_new, k_cache and v_cache must be 16-byte aligned");
+  if (batch == 0) return TACO_OK;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(TACO_ERR_UNSUPPORTED, "device index %d too large", dev);
+  uint32_t* err = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    st = ensure_workspace(dev, 0, 0, 0);
+    if (st != TACO_OK) return st;
+    err = g_ws[dev].error_word;
+  }
+  taco::AppendArgs a{k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, err,
+                     batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                     dtype};
+  e = taco::launch_append_e4m3(a, k_scale, v_scale, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
   return TACO_OK;
 }

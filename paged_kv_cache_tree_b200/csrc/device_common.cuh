@@ -3,9 +3,12 @@
 #pragma once
 
 #include <cuda.h>
+#include <float.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "taco_attn.h"
 
@@ -32,6 +35,8 @@ struct VerifyParams {
   int row_groups;        // number of row groups per (sequence, KV head)
   int cands_per_group;   // tensor-core path: candidates per row group (rows = cands_per_group * G)
   int tile_keys;         // keys per work tile of the kernel (64 or 128)
+  const float* k_scale;  // e4m3 caches: per-KV-head scales (K value = code * k_scale[h]); else null
+  const float* v_scale;
 };
 
 // ---------------------------------------------------------------------------------------------
@@ -170,6 +175,28 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
+}
+
+// Two e4m3 codes (low byte first) as an f16x2 MMA operand pair (exact: every e4m3 value is an f16
+// normal or zero).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t h;
+  const uint16_t v = static_cast<uint16_t>(two_codes & 0xffffu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+  return h;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// byte permute: bytes 0-3 of a, then 4-7 of b, picked by the four selector nibbles
+__device__ __forceinline__ uint32_t byte_perm(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
 }
 
 template <typename T>

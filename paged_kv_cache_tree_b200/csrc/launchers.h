@@ -20,6 +20,7 @@ struct AppendArgs {
   void* v_cache;
   uint32_t* error_word;
   int B, C, Hkv, D, bs, num_blocks, max_blocks;
+  int dtype;  // of k_new / v_new (the quantising append converts them)
 };
 
 struct MaskArgs {
@@ -51,10 +52,14 @@ cudaError_t launch_accept(const AcceptArgs& a, cudaStream_t stream);
 // Rows of packed queries one unit of the mma.sync verify kernel covers for a given G * C.
 int mma_rows_per_unit(int packed_rows);
 // Dynamic shared memory the mma.sync verify kernel needs.
-int mma_smem_bytes(int D, int rows_per_unit);
+int mma_smem_bytes(int D, int rows_per_unit, bool kv8 = false);
+// keys per work tile of the mma.sync kernel for this unit height (e4m3 caches: 128 for <= 32 rows)
+int mma_tile_keys(int rows_per_unit, bool kv8);
 cudaError_t launch_verify_mma(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p,
                               int dtype, int grid, cudaStream_t stream);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+// Quantising append into an e4m3 cache: code = e4m3(x / scale[h]) (round to nearest even, saturating).
+cudaError_t launch_append_e4m3(const AppendArgs& a, const float* k_scale, const float* v_scale, cudaStream_t stream);
 // Keys per work tile of the tcgen05 verify kernel.
 int tc_tile_keys();
 // Dynamic shared memory of the tcgen05 verify kernel.

@@ -10,19 +10,27 @@ int mma_rows_per_unit(int packed_rows) {
   return 64;
 }
 
-int mma_smem_bytes(int D, int rows_per_unit) {
+int mma_tile_keys(int rows_per_unit, bool kv8) {
   const int mt = rows_per_unit / 16;
+  if (!kv8) return MmaCfg<128, 1>::kTile;
+  return mt == 1 ? MmaCfg<128, 1, true>::kTile : mt == 2 ? MmaCfg<128, 2, true>::kTile : MmaCfg<128, 4, true>::kTile;
+}
+
+int mma_smem_bytes(int D, int rows_per_unit, bool kv8) {
+  const int mt = rows_per_unit / 16;
+  if (kv8) return mt == 1 ? MmaCfg<128, 1, true>::kSmemBytes : mt == 2 ? MmaCfg<128, 2, true>::kSmemBytes
+                                                                       : MmaCfg<128, 4, true>::kSmemBytes;
   if (D == 128) {
     return mt == 1 ? MmaCfg<128, 1>::kSmemBytes : mt == 2 ? MmaCfg<128, 2>::kSmemBytes : MmaCfg<128, 4>::kSmemBytes;
   }
   return mt == 1 ? MmaCfg<64, 1>::kSmemBytes : mt == 2 ? MmaCfg<64, 2>::kSmemBytes : MmaCfg<64, 4>::kSmemBytes;
 }
 
-template <typename T, int D, int MT>
+template <typename T, int D, int MT, bool KV8 = false>
 static cudaError_t launch_one(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p, int grid,
                               cudaStream_t stream) {
-  using Cfg = MmaCfg<D, MT>;
-  auto kern = verify_mma_kernel<T, D, MT>;
+  using Cfg = MmaCfg<D, MT, KV8>;
+  auto kern = verify_mma_kernel<T, D, MT, KV8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   // programmatic stream serialization: the prologue may overlap the previous kernel's tail; the
@@ -46,6 +54,11 @@ template <typename T>
 static cudaError_t launch_typed(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p, int grid,
                                 cudaStream_t stream) {
   const int mt = p.rows_per_unit / 16;
+  if (p.k_scale != nullptr) {  // e4m3 K/V (D = 128 only)
+    if (mt == 1) return launch_one<T, 128, 1, true>(tk, tv, p, grid, stream);
+    if (mt == 2) return launch_one<T, 128, 2, true>(tk, tv, p, grid, stream);
+    return launch_one<T, 128, 4, true>(tk, tv, p, grid, stream);
+  }
   if (p.D == 128) {
     if (mt == 1) return launch_one<T, 128, 1>(tk, tv, p, grid, stream);
     if (mt == 2) return launch_one<T, 128, 2>(tk, tv, p, grid, stream);

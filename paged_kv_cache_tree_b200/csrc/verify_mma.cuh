@@ -18,19 +18,24 @@
 
 namespace taco {
 
-template <int D, int MT>
+template <int D, int MT, bool KV8 = false>
 struct MmaCfg {
   static constexpr int kConsumerWarps = 4;
   static constexpr int kProducerWarps = 2;                   // K and V
   static constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
   static constexpr int KG = kConsumerWarps / MT;              // key groups
-  static constexpr int kKeysPerWarp = kTileKeys / KG;         // 16, 32 or 64
+  // keys per tile: e4m3 tiles carry half the bytes per key, so narrow units take 128 keys per tile
+  // to keep the per-tile work (and its fixed costs) in proportion to the bytes it brings
+  static constexpr int kTile = (KV8 && MT <= 2) ? 128 : kTileKeys;
+  static constexpr int kKeysPerWarp = kTile / KG;             // 16 .. 64
   static constexpr int kRows = 16 * MT;                       // packed rows per unit
-  static constexpr int kPanels = D / 64;                      // 128-byte-wide column panels
-  static constexpr int kPanelBytes = kTileKeys * 128;
+  // 128-byte-wide column panels of a K or V row: 64 16-bit values, or 128 e4m3 codes (KV8)
+  static constexpr int kColsPerPanel = KV8 ? 128 : 64;
+  static constexpr int kPanels = D / kColsPerPanel;
+  static constexpr int kPanelBytes = kTile * 128;
   static constexpr int kTensorBytes = kPanels * kPanelBytes;  // one of K or V per stage
   static constexpr int kStageBytes = 2 * kTensorBytes;
-  static constexpr int kStages = (D == 128) ? 3 : 6;
+  static constexpr int kStages = (kPanels * kPanelBytes >= 16384) ? 3 : 6;  // 96 KB of stages
   static constexpr int kScratchFloats = 16 * D + 64;          // cross-warp O and l
   static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes +
                                     kScratchFloats * 4 + 64 * 4 /*m publish*/ +
@@ -42,12 +47,14 @@ struct SchedShared {
   int nC, b, merge_flag, abort_flag;
 };
 
-template <typename T, int D, int MT>
+template <typename T, int D, int MT, bool KV8>
 __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     verify_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const VerifyParams p) {
-  using Cfg = MmaCfg<D, MT>;
+  using Cfg = MmaCfg<D, MT, KV8>;
   using Op = MmaOp<T>;
+  // e4m3 caches: every product runs as f16 x f16 (K and V codes widen exactly to f16)
+  using MOp = typename std::conditional<KV8, MmaOp<__half>, MmaOp<T>>::type;
   constexpr int KG = Cfg::KG;
   constexpr int KW = Cfg::kKeysPerWarp;
   constexpr int NT = KW / 8;          // 8-key n-tiles per warp and tile
@@ -105,15 +112,15 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
     prefetch_tensormap(tmap);
     const uint64_t policy = policy_evict_first();
-    const int rpc = p.bs < kTileKeys ? p.bs : kTileKeys;   // rows per chunk
-    const int chunks_per_tile = kTileKeys / rpc;
+    const int rpc = p.bs < Cfg::kTile ? p.bs : Cfg::kTile;   // rows per chunk
+    const int chunks_per_tile = Cfg::kTile / rpc;
     const uint32_t chunk_bytes = static_cast<uint32_t>(rpc) * 128u;
     int stage = 0;
     uint32_t phase = 0;
     int b = sched->b;
     int64_t base_b = sched->base_b;
     int L = clamp_context(p, b, is_k);
-    int Tb = tiles_of(L, kTileKeys);
+    int Tb = tiles_of(L, Cfg::kTile);
     int64_t t = lo;
     int j = static_cast<int>((t - base_b) / Tb);
     int tile = static_cast<int>((t - base_b) % Tb);
@@ -125,7 +132,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
       int win = -1000000;
       int32_t win_val = -1;
       for (int tl = tile; tl < tend; ++tl) {
-        const int key0 = tl * kTileKeys;
+        const int key0 = tl * Cfg::kTile;
         int nvalid = L > key0 ? (L - key0 + rpc - 1) / rpc : 0;
         if (nvalid > chunks_per_tile) nvalid = chunks_per_tile;
         // block ids of this tile's chunks (window of 32 logical blocks held one per lane)
@@ -157,7 +164,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
           const int row = (blk * p.Hkv + g) * p.bs + (key0 + lane * rpc) % p.bs;
           const uint32_t fb = smem_addr(full_bar + stage);
 #pragma unroll
-          for (int pn = 0; pn < Cfg::kPanels; ++pn) tma_load_2d(dst + pn * Cfg::kPanelBytes, tmap, fb, pn * 64, row, policy);
+          for (int pn = 0; pn < Cfg::kPanels; ++pn) tma_load_2d(dst + pn * Cfg::kPanelBytes, tmap, fb, pn * Cfg::kColsPerPanel, row, policy);
         }
         __syncwarp();
         if (++stage == Cfg::kStages) {
@@ -172,7 +179,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
         base_b += static_cast<int64_t>(Tb) * HR;
         if (++b < p.B) {
           L = clamp_context(p, b, is_k);
-          Tb = tiles_of(L, kTileKeys);
+          Tb = tiles_of(L, Cfg::kTile);
         }
       }
     }
@@ -198,7 +205,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
   int b = sched->b;
   int64_t base_b = sched->base_b;
   int L = clamp_context(p, b, false);
-  int Tb = tiles_of(L, kTileKeys);
+  int Tb = tiles_of(L, Cfg::kTile);
   int64_t t = lo;
   int j = static_cast<int>((t - base_b) / Tb);
   int tile = static_cast<int>((t - base_b) % Tb);
@@ -206,6 +213,9 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
 
   while (t < hi) {
     const int g = j / p.row_groups;
+    // e4m3 caches: the K scale joins the logit scale, the V scale multiplies O when it is written
+    const float sl2 = KV8 ? p.scale_log2 * __ldg(p.k_scale + g) : p.scale_log2;
+    const float vsc = KV8 ? __ldg(p.v_scale + g) : 1.f;
     const int rg = j % p.row_groups;
     const int tbegin = tile;
     const int tend = static_cast<int>(Tb < tile + (hi - t) ? Tb : tile + (hi - t));
@@ -225,6 +235,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     }
     // Q fragments (A operand of m16n8k16): rows gq / gq+8, columns 2*tq.. of each 16-wide k step
     uint32_t qf[KSTEPS][4];
+    float sl2r[2] = {sl2, sl2};   // logit scale of this thread's two rows (base 2)
     {
       const uint32_t* qrow[2];
 #pragma unroll
@@ -233,12 +244,59 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
         qrow[h] = reinterpret_cast<const uint32_t*>(static_cast<const T*>(p.q) +
                                                     ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D);
       }
+      if constexpr (!KV8) {
 #pragma unroll
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-        qf[kk][0] = rvalid[0] ? __ldg(qrow[0] + kk * 8 + tq) : 0u;
-        qf[kk][1] = rvalid[1] ? __ldg(qrow[1] + kk * 8 + tq) : 0u;
-        qf[kk][2] = rvalid[0] ? __ldg(qrow[0] + kk * 8 + 4 + tq) : 0u;
-        qf[kk][3] = rvalid[1] ? __ldg(qrow[1] + kk * 8 + 4 + tq) : 0u;
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          qf[kk][0] = rvalid[0] ? __ldg(qrow[0] + kk * 8 + tq) : 0u;
+          qf[kk][1] = rvalid[1] ? __ldg(qrow[1] + kk * 8 + tq) : 0u;
+          qf[kk][2] = rvalid[0] ? __ldg(qrow[0] + kk * 8 + 4 + tq) : 0u;
+          qf[kk][3] = rvalid[1] ? __ldg(qrow[1] + kk * 8 + 4 + tq) : 0u;
+        }
+      } else {
+        // The k order of Q K^T is permuted (the sum does not depend on it) so that a thread's K codes
+        // are 32 consecutive bytes of the key row: k step kk, A/B pair j (0: k = 2tq, 2tq+1; 1: k =
+        // 2tq+8, 2tq+9) takes head dims tq*32 + kk*4 + 2j (+1). bf16 queries go to f16 times a
+        // power of two per row that puts the row's largest magnitude in [2^14, 2^15) (exact for
+        // every element down to 2^-29 of it); the logit scale takes the inverse power.
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w[16];
+          const uint4* q4 = reinterpret_cast<const uint4*>(qrow[h] + tq * 16);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 x = rvalid[h] ? __ldg(q4 + v) : make_uint4(0u, 0u, 0u, 0u);
+            w[4 * v] = x.x;
+            w[4 * v + 1] = x.y;
+            w[4 * v + 2] = x.z;
+            w[4 * v + 3] = x.w;
+          }
+          if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+            float mx = 0.f;
+#pragma unroll
+            for (int v = 0; v < 16; ++v)
+              mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[v] << 16)), fabsf(__uint_as_float(w[v] & 0xffff0000u))));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            int k = 0;
+            if (mx > 0.f && mx <= FLT_MAX) {
+              const int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
+              k = 14 - e < 64 ? 14 - e : 64;
+            }
+            const float up = __uint_as_float(static_cast<uint32_t>(127 + k) << 23);
+            sl2r[h] = sl2 * __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
+#pragma unroll
+            for (int v = 0; v < 16; ++v) {
+              const __half2 hv = __floats2half2_rn(__uint_as_float(w[v] << 16) * up,
+                                                   __uint_as_float(w[v] & 0xffff0000u) * up);
+              w[v] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+          }
+#pragma unroll
+          for (int kk = 0; kk < KSTEPS; ++kk) {
+            qf[kk][h] = w[2 * kk];
+            qf[kk][2 + h] = w[2 * kk + 1];
+          }
+        }
       }
     }
     float m_run[2] = {-INFINITY, -INFINITY};
@@ -248,7 +306,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     for (int dt = 0; dt < DT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
 
     for (int tl = tbegin; tl < tend; ++tl) {
-      const int key0 = tl * kTileKeys;
+      const int key0 = tl * Cfg::kTile;
       bool ready = false;
       if (*abort_flag == 0) {
         ready = mbar_wait(smem_addr(full_bar + stage), phase, p.error_word);
@@ -257,7 +315,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
       const uint32_t kbase = smem_addr(stages + stage * Cfg::kStageBytes);
       const uint32_t vbase = kbase + Cfg::kTensorBytes;
       const int wkey0 = kg * KW;   // first tile-relative key of this warp
-      if (ready && key0 + kTileKeys > L) {
+      if (ready && key0 + Cfg::kTile > L) {
         // keys >= L in this tile: their V rows may be stale or NaN-poisoned; zero this warp's
         int zr0 = L - key0 - wkey0;
         if (zr0 < 0) zr0 = 0;
@@ -275,27 +333,44 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
         float s[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        if constexpr (!KV8) {
 #pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
+          for (int kk = 0; kk < KSTEPS; ++kk) {
 #pragma unroll
-          for (int np = 0; np < NT / 2; ++np) {
-            const int key = wkey0 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
-            const int d = kk * 16 + ((lane >> 3) & 1) * 8;
-            const int c = (d & 63) >> 3;
-            const uint32_t addr = kbase + (d >> 6) * Cfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(addr, b0, b1, b2, b3);
-            Op::run(s[2 * np], qf[kk], b0, b1);
-            Op::run(s[2 * np + 1], qf[kk], b2, b3);
+            for (int np = 0; np < NT / 2; ++np) {
+              const int key = wkey0 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
+              const int d = kk * 16 + ((lane >> 3) & 1) * 8;
+              const int c = (d & 63) >> 3;
+              const uint32_t addr = kbase + (d >> 6) * Cfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4);
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4(addr, b0, b1, b2, b3);
+              Op::run(s[2 * np], qf[kk], b0, b1);
+              Op::run(s[2 * np + 1], qf[kk], b2, b3);
+            }
+          }
+        } else {
+          // e4m3 K rows are 128 bytes, 16-byte chunk c of key row r at (c ^ (r & 7)) * 16; in the permuted
+          // k order a thread needs chunks 2tq and 2tq+1 of its key (r & 7 == gq): word kk holds the B
+          // pairs of k step kk
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const int key = wkey0 + nt * 8 + gq;
+            const uint32_t rowa = kbase + key * 128;
+            const uint4 c0 = lds_v4(rowa + (((2 * tq) ^ gq) << 4));
+            const uint4 c1 = lds_v4(rowa + (((2 * tq + 1) ^ gq) << 4));
+            const uint32_t kw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk)
+              MOp::run(s[nt], qf[kk], e4m3x2_to_f16x2(kw[kk]), e4m3x2_to_f16x2(kw[kk] >> 16));
           }
         }
         // scale, mask, online softmax
-        const bool need_mask = key0 + kTileKeys > P;
+        const bool need_mask = key0 + Cfg::kTile > P;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float v = s[nt][e] * p.scale_log2;
+            float v = s[nt][e] * sl2r[e >> 1];
             if (need_mask) {
               const int key = key0 + wkey0 + nt * 8 + 2 * tq + (e & 1);
               const int h = e >> 1;
@@ -305,6 +380,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
             s[nt][e] = v;
           }
         }
+        float alpha[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float mx = -INFINITY;
@@ -314,7 +390,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
           const float m_new = fmaxf(m_run[h], mx);
           const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          const float alpha = fast_exp2(m_run[h] - m_use);
+          alpha[h] = fast_exp2(m_run[h] - m_use);
           m_run[h] = m_new;
           float rs = 0.f;
 #pragma unroll
@@ -325,31 +401,61 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
             s[nt][2 * h + 1] = p1;
             rs += p0 + p1;
           }
-          l_run[h] = l_run[h] * alpha + rs;
+          l_run[h] = l_run[h] * alpha[h] + rs;
+        }
+        // O only needs rescaling when some row's running max moved (alpha is exactly 1 otherwise)
+        if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
           for (int dt = 0; dt < DT; ++dt) {
-            o[dt][2 * h] *= alpha;
-            o[dt][2 * h + 1] *= alpha;
+            o[dt][0] *= alpha[0];
+            o[dt][1] *= alpha[0];
+            o[dt][2] *= alpha[1];
+            o[dt][3] *= alpha[1];
           }
         }
         // O += P V
 #pragma unroll
         for (int ks = 0; ks < KW / 16; ++ks) {
           uint32_t a[4];
-          a[0] = Op::pack(s[2 * ks][0], s[2 * ks][1]);
-          a[1] = Op::pack(s[2 * ks][2], s[2 * ks][3]);
-          a[2] = Op::pack(s[2 * ks + 1][0], s[2 * ks + 1][1]);
-          a[3] = Op::pack(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+          a[0] = MOp::pack(s[2 * ks][0], s[2 * ks][1]);
+          a[1] = MOp::pack(s[2 * ks][2], s[2 * ks][3]);
+          a[2] = MOp::pack(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+          a[3] = MOp::pack(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+          if constexpr (!KV8) {
 #pragma unroll
-          for (int dp = 0; dp < D / 16; ++dp) {
-            const int key = wkey0 + ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            const int d = dp * 16 + (lane >> 4) * 8;
-            const int c = (d & 63) >> 3;
-            const uint32_t addr = vbase + (d >> 6) * Cfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_trans(addr, b0, b1, b2, b3);
-            Op::run(o[2 * dp], a, b0, b1);
-            Op::run(o[2 * dp + 1], a, b2, b3);
+            for (int dp = 0; dp < D / 16; ++dp) {
+              const int key = wkey0 + ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+              const int d = dp * 16 + (lane >> 4) * 8;
+              const int c = (d & 63) >> 3;
+              const uint32_t addr = vbase + (d >> 6) * Cfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4);
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4_trans(addr, b0, b1, b2, b3);
+              Op::run(o[2 * dp], a, b0, b1);
+              Op::run(o[2 * dp + 1], a, b2, b3);
+            }
+          } else {
+            // Output columns are permuted: column n of n tile dt is head dim n*16 + dt, so the B
+            // fragments of a thread (column gq) are byte dt of chunk gq of key rows 2tq, 2tq+1, 2tq+8,
+            // 2tq+9 (row & 7 == 2tq or 2tq+1), four 16-byte loads per 16 keys
+            const int kr = wkey0 + ks * 16 + 2 * tq;
+            const uint4 x0 = lds_v4(vbase + kr * 128 + ((gq ^ (2 * tq)) << 4));
+            const uint4 x1 = lds_v4(vbase + (kr + 1) * 128 + ((gq ^ (2 * tq + 1)) << 4));
+            const uint4 x2 = lds_v4(vbase + (kr + 8) * 128 + ((gq ^ (2 * tq)) << 4));
+            const uint4 x3 = lds_v4(vbase + (kr + 9) * 128 + ((gq ^ (2 * tq + 1)) << 4));
+            const uint32_t r0[4] = {x0.x, x0.y, x0.z, x0.w}, r1[4] = {x1.x, x1.y, x1.z, x1.w};
+            const uint32_t r2[4] = {x2.x, x2.y, x2.z, x2.w}, r3[4] = {x3.x, x3.y, x3.z, x3.w};
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+#pragma unroll
+              for (int i = 0; i < 4; i += 2) {
+                // bytes (i of row 2tq, i of row 2tq+1, i+1 of row 2tq, i+1 of row 2tq+1)
+                const uint32_t sel = i | ((4 + i) << 4) | ((i + 1) << 8) | ((5 + i) << 12);
+                const uint32_t lo = byte_perm(r0[wd], r1[wd], sel);
+                const uint32_t hi = byte_perm(r2[wd], r3[wd], sel);
+                MOp::run(o[4 * wd + i], a, e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi));
+                MOp::run(o[4 * wd + i + 1], a, e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi >> 16));
+              }
+            }
           }
         }
       }
@@ -420,23 +526,51 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int R = Rrow[h];
-        const float inv = l_run[h] > 0.f ? 1.f / l_run[h] : 0.f;
+        const float inv = (l_run[h] > 0.f ? 1.f / l_run[h] : 0.f) * vsc;
         if (whole_unit) {
           if (R < p.G * p.C) {
             const int i = R / p.G, hh = R % p.G;
             T* dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D;
+            if constexpr (!KV8) {
 #pragma unroll
-            for (int dt = 0; dt < DT; ++dt)
-              *reinterpret_cast<uint32_t*>(dst + dt * 8 + 2 * tq) =
-                  rvalid[h] ? Op::pack(o[dt][2 * h] * inv, o[dt][2 * h + 1] * inv) : 0u;
+              for (int dt = 0; dt < DT; ++dt)
+                *reinterpret_cast<uint32_t*>(dst + dt * 8 + 2 * tq) =
+                    rvalid[h] ? Op::pack(o[dt][2 * h] * inv, o[dt][2 * h + 1] * inv) : 0u;
+            } else {
+              // permuted columns: this thread holds head dims tq*32 + j, j < 16 in o[j][2h], j >= 16 in
+              // o[j - 16][2h + 1]
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const int e = 2 * h + (v >> 1);
+                const int d0 = (v & 1) * 8;
+                uint4 x = make_uint4(0u, 0u, 0u, 0u);
+                if (rvalid[h]) {
+                  x.x = Op::pack(o[d0][e] * inv, o[d0 + 1][e] * inv);
+                  x.y = Op::pack(o[d0 + 2][e] * inv, o[d0 + 3][e] * inv);
+                  x.z = Op::pack(o[d0 + 4][e] * inv, o[d0 + 5][e] * inv);
+                  x.w = Op::pack(o[d0 + 6][e] * inv, o[d0 + 7][e] * inv);
+                }
+                *reinterpret_cast<uint4*>(dst + tq * 32 + v * 8) = x;
+              }
+            }
           }
         } else {
           const int r = mt * 16 + gq + 8 * h;
           float* dst = p.part_o + (static_cast<int64_t>(slot) * ROWS + r) * D;
+          if constexpr (!KV8) {
 #pragma unroll
-          for (int dt = 0; dt < DT; ++dt)
-            __stcg(reinterpret_cast<float2*>(dst + dt * 8 + 2 * tq),
-                   make_float2(o[dt][2 * h] * inv, o[dt][2 * h + 1] * inv));
+            for (int dt = 0; dt < DT; ++dt)
+              __stcg(reinterpret_cast<float2*>(dst + dt * 8 + 2 * tq),
+                     make_float2(o[dt][2 * h] * inv, o[dt][2 * h + 1] * inv));
+          } else {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const int e = 2 * h + (v >> 2);
+              const int d0 = (v & 3) * 4;
+              __stcg(reinterpret_cast<float4*>(dst + tq * 32 + v * 4),
+                     make_float4(o[d0][e] * inv, o[d0 + 1][e] * inv, o[d0 + 2][e] * inv, o[d0 + 3][e] * inv));
+            }
+          }
           if (tq == 0)
             __stcg(p.part_lse + static_cast<int64_t>(slot) * ROWS + r,
                    l_run[h] > 0.f ? m_run[h] + __log2f(l_run[h]) : -INFINITY);
@@ -483,7 +617,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
       base_b += static_cast<int64_t>(Tb) * HR;
       if (++b < p.B) {
         L = clamp_context(p, b, false);
-        Tb = tiles_of(L, kTileKeys);
+        Tb = tiles_of(L, Cfg::kTile);
       }
     }
   }

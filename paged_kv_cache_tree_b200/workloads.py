@@ -24,6 +24,10 @@ candidates) is filled with NaN for parity runs (``fill="nan"``) or zeros for tim
 Candidate i of sequence b sits at logical position P_b + i with P_b = L_b - n_b. With
 ``candidates_in_cache=True`` the cache already holds k_new/v_new there (the state after a
 paged KV-append); otherwise those slots are poisoned too and an append must fill them.
+
+8-bit (e4m3) caches for a workload come from ``make_e4m3_cache``: byte patterns drawn directly (random
+sign and mantissa, exponent field mostly in 9..14, sometimes anywhere in 0..14), the NaN code where the
+16-bit caches hold NaN, and per-KV-head scales uniform on [0.004, 0.012]; no quantisation happens here.
 """
 from __future__ import annotations
 
@@ -273,6 +277,69 @@ def make_workload(
         block_tables=bt, slot_offsets=slots, q=q, k_cache=k_cache, v_cache=v_cache,
         k_new=k_new, v_new=v_new,
     )
+
+
+@dataclasses.dataclass
+class KV8Cache:
+    """e4m3 caches of a workload: uint8 codes [NB, Hkv, bs, D] and float32 per-KV-head scales."""
+
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    k_scale: torch.Tensor
+    v_scale: torch.Tensor
+
+    def to(self, device) -> "KV8Cache":
+        return KV8Cache(*(getattr(self, f.name).to(device) for f in dataclasses.fields(self)))
+
+
+E4M3_NAN = 0x7F
+
+
+def _random_e4m3_codes(n: int, g: torch.Generator) -> torch.Tensor:
+    """n random finite e4m3 byte patterns on the generator's device: sign and 3-bit mantissa uniform;
+    the 4-bit exponent field uniform on 9..14 for 7 of 8 codes and on 0..14 (zeros and subnormals
+    included) for the rest."""
+    dev = g.device
+    out = torch.empty(n, dtype=torch.uint8, device=dev)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        m = e - s
+        draw = lambda lo, hi: torch.randint(lo, hi, (m,), generator=g, dtype=torch.int32, device=dev)
+        sign, man, exp_hi, exp_all = draw(0, 2), draw(0, 8), draw(9, 15), draw(0, 15)
+        wide = draw(0, 8) == 0
+        ex = torch.where(wide, exp_all, exp_hi)
+        out[s:e] = ((sign << 7) | (ex << 3) | man).to(torch.uint8)
+    return out
+
+
+def make_e4m3_cache(w: Workload, *, seed: Optional[int] = None) -> KV8Cache:
+    """Seeded e4m3 caches with the block layout of ``w`` (drawn on the device ``w``'s caches live on):
+    random finite codes wherever ``w``'s 16-bit caches hold numbers, the NaN code 0x7F wherever they hold
+    NaN (unused blocks, slots past L_b and, unless the workload put them there, the candidates' slots);
+    scales uniform on [0.004, 0.012]."""
+    dev = w.k_cache.device
+    g = torch.Generator(device=dev).manual_seed(int(seed if seed is not None else 77 + w.B * 131 + w.Hkv))
+    shape = tuple(w.k_cache.shape)
+    n = w.k_cache.numel()
+    caches = []
+    for src in (w.k_cache, w.v_cache):
+        codes = _random_e4m3_codes(n, g).view(shape)
+        codes[torch.isnan(src)] = E4M3_NAN
+        caches.append(codes)
+    k_scale = (0.004 + 0.008 * torch.rand(w.Hkv, generator=g, device=dev)).to(torch.float32)
+    v_scale = (0.004 + 0.008 * torch.rand(w.Hkv, generator=g, device=dev)).to(torch.float32)
+    return KV8Cache(caches[0], caches[1], k_scale, v_scale)
+
+
+def kv8_attention_bytes(w: Workload) -> int:
+    """Bytes the verify must move with e4m3 caches: K+V codes of every key, Q and O (16-bit)."""
+    return int(w.context_lens.long().sum()) * w.Hkv * w.D * 2 + w.qo_bytes()
+
+
+def kv8_append_bytes(w: Workload) -> int:
+    """Quantising append: 16-bit rows read, e4m3 codes written, for K and V."""
+    rows = int(w.num_candidates.long().sum())
+    return 2 * rows * w.Hkv * w.D * (2 + 1)
 
 
 @dataclasses.dataclass

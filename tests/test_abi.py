@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.taco_attn_version() == 2
+    assert lib.taco_attn_version() == 3
 
 
 def _attn_args(**over):
@@ -114,3 +114,55 @@ def test_acceptance_calls_with_nothing_to_do_are_no_ops(lib):
     assert lib.tree_mask_from_parents(16, 16, 0, 4, 16, None) == _lib.TACO_OK
     assert lib.logits_argmax(16, 1, 0, 100, 16, None) == _lib.TACO_OK
     assert lib.tree_greedy_accept(16, 16, 16, 16, 16, 0, 4, 16, 16, 16, 16, None) == _lib.TACO_OK
+
+
+def _attn8_args(**over):
+    a = dict(ks=16, vs=16)
+    a.update({k: over.pop(k) for k in list(over) if k in a})
+    base = _attn_args(**over)
+    return base[:3] + [a["ks"], a["vs"]] + base[3:]
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(ks=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(vs=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(q=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(D=64), _lib.TACO_ERR_UNSUPPORTED),          # e4m3 caches: head_dim 128 only
+    (dict(Hq=64, Hkv=2, C=4), _lib.TACO_ERR_UNSUPPORTED),  # 32 * 4 packed rows > 64
+    (dict(dtype=3), _lib.TACO_ERR_INVALID_ARG),
+    (dict(k=24), _lib.TACO_ERR_INVALID_ARG),
+])
+def test_e4m3_attention_rejects_bad_arguments_on_host(lib, over, status):
+    assert lib.paged_tree_attention_e4m3(*_attn8_args(**over)) == status
+    assert lib.taco_attn_last_error().decode()
+
+
+def test_e4m3_attention_has_no_tensor_core_kernel(lib):
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_KERNEL, 2) == _lib.TACO_OK
+    try:
+        assert lib.paged_tree_attention_e4m3(*_attn8_args()) == _lib.TACO_ERR_UNSUPPORTED
+    finally:
+        assert lib.taco_attn_set_option(_lib.TACO_OPT_KERNEL, 0) == _lib.TACO_OK
+
+
+def test_e4m3_calls_with_empty_batch_are_no_ops(lib):
+    assert lib.paged_tree_attention_e4m3(*_attn8_args(B=0)) == _lib.TACO_OK
+    args = [16, 16, 16, 16, 16, 16, 16, 16, 1, 0, 4, 2, 128, 16, 40, 8, None]
+    assert lib.paged_kv_append_e4m3(*args) == _lib.TACO_OK
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(ks=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(vs=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(kc=8), _lib.TACO_ERR_INVALID_ARG),
+    (dict(D=96), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(dtype=2), _lib.TACO_ERR_INVALID_ARG),
+])
+def test_e4m3_append_rejects_bad_arguments_on_host(lib, over, status):
+    a = dict(kn=16, vn=16, bt=16, so=16, ks=16, vs=16, kc=16, vc=16, dtype=1, B=2, C=4, Hkv=2, D=128, bs=16,
+             NB=40, maxblk=8, stream=None)
+    a.update(over)
+    args = [a["kn"], a["vn"], a["bt"], a["so"], a["ks"], a["vs"], a["kc"], a["vc"], a["dtype"], a["B"], a["C"],
+            a["Hkv"], a["D"], a["bs"], a["NB"], a["maxblk"], a["stream"]]
+    assert lib.paged_kv_append_e4m3(*args) == status
+    assert lib.taco_attn_last_error().decode()

@@ -1,0 +1,171 @@
+"""GPU parity of the e4m3 (8-bit) KV cache path against the CPU oracle (needs a B200).
+
+The quantising append is byte work: its codes must equal the oracle's bit for bit (division in
+float32, nearest e4m3 with ties to the even code, saturation at 448). The attention over e4m3 caches
+must lie within |gpu - ref| <= 1e-2 + 2e-2 |ref| of the fp64 oracle that decodes the same codes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import fp8
+import paged_kv_cache_tree_b200 as taco
+from paged_kv_cache_tree_b200 import workloads as wl
+from tests.parity_util import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _reset_options():
+    taco.set_option(taco.TACO_OPT_GRID_CTAS, 0)
+    taco.set_option(taco.TACO_OPT_KERNEL, 0)
+    yield
+    taco.set_option(taco.TACO_OPT_GRID_CTAS, 0)
+    taco.set_option(taco.TACO_OPT_KERNEL, 0)
+
+
+def oracle_attention_e4m3(w, c8, rows=None, k_cache=None, v_cache=None):
+    return oracle.paged_tree_attention(
+        wl.to_numpy_bits(w.q), (c8.k_cache if k_cache is None else k_cache).numpy(),
+        (c8.v_cache if v_cache is None else v_cache).numpy(), w.block_tables.numpy(), w.context_lens.numpy(),
+        w.num_candidates.numpy(), wl.as_uint32(w.tree_mask), w.scale, w.dtype, rows=rows, kv_dtype="e4m3",
+        k_scale=c8.k_scale.numpy(), v_scale=c8.v_scale.numpy())
+
+
+def gpu_attention_e4m3(w, c8):
+    d, g8 = w.to("cuda"), c8.to("cuda")
+    out = torch.full_like(d.q, float("nan"))
+    taco.paged_tree_attention_e4m3(d.q, g8.k_cache, g8.v_cache, g8.k_scale, g8.v_scale, d.block_tables,
+                                   d.context_lens, d.num_candidates, d.tree_mask, w.scale, out=out)
+    assert taco.check_device() == 0
+    return out.cpu()
+
+
+def special_rows(w):
+    """Overwrite some new K/V rows with values that probe the rounding: exact midpoints between e4m3
+    neighbours (ties go to the even code), values past 448 (saturation), +-inf, tiny values
+    (subnormal codes and underflow to zero) and signed zeros."""
+    k, v = w.k_new.clone(), w.v_new.clone()
+    D = w.D
+    probe = torch.tensor([1.0625, 1.1875, -1.0625, 0.3125 * 1.0625, 500.0, -1e4, float("inf"), float("-inf"),
+                          2.0 ** -10, -(2.0 ** -10) * 1.5, 2.0 ** -12, 0.0, -0.0, 448.0, 464.0, 480.0])
+    reps = (D + len(probe) - 1) // len(probe)
+    row = probe.repeat(reps)[:D].to(k.dtype)
+    k[0, 0, 0] = row
+    v[0, 0, -1] = -row
+    return k, v
+
+
+@pytest.mark.parametrize("dtype,D,bs", [("bf16", 128, 16), ("fp16", 128, 32), ("bf16", 64, 8), ("fp16", 64, 64)])
+def test_quantising_append_bit_exact(dtype, D, bs):
+    spec = dict(dtype=dtype, B=4, Hq=8, Hkv=2, D=D, bs=bs, C=5, tree="forest", ctx=("uniform", 6, 200))
+    w = wl.make_workload(spec, seed=3 + D + bs, candidates_in_cache=False, num_candidates=[5, 0, 3, 5])
+    c8 = wl.make_e4m3_cache(w, seed=9)
+    k_new, v_new = special_rows(w)
+    scales = (torch.tensor([1.0, 0.0173] if dtype == "bf16" else [0.5, 3.7]),
+              torch.tensor([0.25, 1.0] if dtype == "bf16" else [1.0, 0.011]))
+    so = w.slot_offsets.clone()
+    so[2, 1] = -1                                  # a skipped row
+    g = {k: v.cuda() for k, v in dict(k_new=k_new, v_new=v_new, bt=w.block_tables, so=so,
+                                      kc=c8.k_cache, vc=c8.v_cache).items()}
+    ks, vs = scales[0].float().cuda(), scales[1].float().cuda()
+    taco.paged_kv_append_e4m3(g["k_new"], g["v_new"], g["bt"], g["so"], ks, vs, g["kc"], g["vc"])
+    assert taco.check_device() == 0
+    rk, rv = fp8.paged_kv_append_e4m3(wl.to_numpy_bits(k_new), wl.to_numpy_bits(v_new), dtype,
+                                      w.block_tables.numpy(), so.numpy(), scales[0].numpy(), scales[1].numpy(),
+                                      c8.k_cache.numpy(), c8.v_cache.numpy())
+    assert np.array_equal(g["kc"].cpu().numpy(), rk)
+    assert np.array_equal(g["vc"].cpu().numpy(), rv)
+    # the probes landed where expected (row (0, 0) sits at slot P_0)
+    P0 = int(w.context_lens[0]) - int(w.num_candidates[0])
+    blk = int(w.block_tables[0, P0 // bs])
+    codes = g["kc"][blk, 0, P0 % bs].cpu().numpy()
+    if dtype == "bf16":                            # scale 1: 1.0625 is a tie between 1.0 and 1.125
+        assert codes[0] == 0x38 and codes[2] == 0xB8 and codes[4] == 0x7E and codes[6] == 0x7E
+        assert codes[7] == 0xFE and codes[11] == 0x00 and codes[12] == 0x80
+
+
+@pytest.mark.parametrize("grid", [0, 1, 3, 50])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("shape", [
+    # Hq, Hkv, C, tree, bs, ctx
+    (32, 8, 1, "chain", 16, ("uniform", 1, 700)),        # decode: 4 packed rows
+    (64, 8, 4, "chain", 64, ("uniform", 100, 900)),      # 32 packed rows
+    (64, 8, 8, "forest", 32, ("uniform", 8, 500)),       # 64 packed rows
+    (8, 1, 5, "forest", 16, ("fixed", [5, 64, 65, 129])),
+])
+def test_attention_over_e4m3_cache(shape, dtype, grid):
+    Hq, Hkv, C, tree, bs, ctx = shape
+    B = 4
+    spec = dict(dtype=dtype, B=B, Hq=Hq, Hkv=Hkv, D=128, bs=bs, C=C, tree=tree, ctx=ctx)
+    w = wl.make_workload(spec, seed=40 + C + Hq + bs)
+    c8 = wl.make_e4m3_cache(w)
+    taco.set_option(taco.TACO_OPT_GRID_CTAS, grid)
+    got = gpu_attention_e4m3(w, c8)
+    ref = oracle_attention_e4m3(w, c8)
+    assert_parity(got, ref, w)
+
+
+def test_empty_contexts_and_padding_rows_are_zero():
+    spec = dict(dtype="bf16", B=3, Hq=16, Hkv=4, D=128, bs=16, C=4, tree="chain", ctx=("fixed", [0, 3, 40]))
+    w = wl.make_workload(spec, seed=5, num_candidates=[0, 2, 4])
+    c8 = wl.make_e4m3_cache(w)
+    got = gpu_attention_e4m3(w, c8)
+    assert torch.all(got[0] == 0) and torch.all(got[1, 2:] == 0)
+    assert_parity(got, oracle_attention_e4m3(w, c8), w)
+
+
+def test_query_magnitudes_far_from_one():
+    """bf16 queries with rows scaled by 2^40 .. 2^-40 and single huge or tiny elements: the kernel
+    rescales each query row into f16 range by a power of two and must still match."""
+    spec = dict(dtype="bf16", B=2, Hq=16, Hkv=2, D=128, bs=16, C=2, tree="chain", ctx=("fixed", [90, 300]))
+    w = wl.make_workload(spec, seed=8)
+    q = w.q.float()
+    q[0, 0, 0] *= 2.0 ** 40
+    q[0, 0, 1] *= 2.0 ** -40
+    q[0, 1, 2] *= 2.0 ** -12
+    q[1, 0, 3] = 0.0
+    q[1, 0, 4, 7] = 3e4
+    q[1, 1, 5, :100] *= 2.0 ** -30
+    w.q = q.to(torch.bfloat16)
+    c8 = wl.make_e4m3_cache(w)
+    assert_parity(gpu_attention_e4m3(w, c8), oracle_attention_e4m3(w, c8), w)
+
+
+def test_append_then_attend_end_to_end():
+    spec = dict(dtype="bf16", B=5, Hq=32, Hkv=8, D=128, bs=16, C=4, tree="forest", ctx=("uniform", 4, 400))
+    w = wl.make_workload(spec, seed=21, candidates_in_cache=False)
+    c8 = wl.make_e4m3_cache(w)
+    d, g8 = w.to("cuda"), c8.to("cuda")
+    taco.paged_kv_append_e4m3(d.k_new, d.v_new, d.block_tables, d.slot_offsets, g8.k_scale, g8.v_scale,
+                              g8.k_cache, g8.v_cache)
+    out = torch.full_like(d.q, float("nan"))
+    taco.paged_tree_attention_e4m3(d.q, g8.k_cache, g8.v_cache, g8.k_scale, g8.v_scale, d.block_tables,
+                                   d.context_lens, d.num_candidates, d.tree_mask, w.scale, out=out)
+    assert taco.check_device() == 0
+    rk, rv = fp8.paged_kv_append_e4m3(wl.to_numpy_bits(w.k_new), wl.to_numpy_bits(w.v_new), w.dtype,
+                                      w.block_tables.numpy(), w.slot_offsets.numpy(), c8.k_scale.numpy(),
+                                      c8.v_scale.numpy(), c8.k_cache.numpy(), c8.v_cache.numpy())
+    assert np.array_equal(g8.k_cache.cpu().numpy(), rk)
+    assert np.array_equal(g8.v_cache.cpu().numpy(), rv)
+    ref = oracle_attention_e4m3(w, c8, k_cache=torch.from_numpy(rk), v_cache=torch.from_numpy(rv))
+    assert_parity(out.cpu(), ref, w)
+
+
+@pytest.mark.parametrize("name", ["decode", "chain", "long"])
+def test_full_size_workloads_sampled_rows(name):
+    """The bench's workloads at full size with e4m3 caches, in the default launch configuration:
+    24 sampled rows against the oracle."""
+    w = wl.make_workload(name)
+    c8 = wl.make_e4m3_cache(w)
+    got = gpu_attention_e4m3(w, c8)
+    rng = np.random.default_rng(1)
+    rows = {(0, 0, 0), (w.B - 1, int(w.num_candidates[-1]) - 1, w.Hq - 1)}
+    while len(rows) < 24:
+        b = int(rng.integers(w.B))
+        rows.add((b, int(rng.integers(max(1, int(w.num_candidates[b])))), int(rng.integers(w.Hq))))
+    rows = sorted(rows)
+    assert_parity(got, oracle_attention_e4m3(w, c8, rows=rows), w, rows=rows)
+    assert torch.isfinite(got.float()).all()
