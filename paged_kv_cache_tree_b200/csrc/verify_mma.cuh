@@ -18,17 +18,21 @@
 
 namespace taco {
 
+// MT = number of 16-row query tiles per unit (1, 2, 4), or 0 for the swapped form used for units of at
+// most 8 packed rows: S^T = K Q^T and O^T = V^T P^T, keys and head dims on the MMA's 16-row side and
+// the 8 query rows on its 8-column side, so that no MMA row is spent on padding queries.
 template <int D, int MT, bool KV8 = false>
 struct MmaCfg {
+  static constexpr bool kSwap = (MT == 0);
   static constexpr int kConsumerWarps = 4;
   static constexpr int kProducerWarps = 2;                   // K and V
   static constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
-  static constexpr int KG = kConsumerWarps / MT;              // key groups
+  static constexpr int KG = kSwap ? kConsumerWarps : kConsumerWarps / MT;   // key groups
   // keys per tile: e4m3 tiles carry half the bytes per key, so narrow units take 128 keys per tile
   // to keep the per-tile work (and its fixed costs) in proportion to the bytes it brings
   static constexpr int kTile = (KV8 && MT <= 2) ? 128 : kTileKeys;
   static constexpr int kKeysPerWarp = kTile / KG;             // 16 .. 64
-  static constexpr int kRows = 16 * MT;                       // packed rows per unit
+  static constexpr int kRows = kSwap ? 8 : 16 * MT;           // packed rows per unit
   // 128-byte-wide column panels of a K or V row: 64 16-bit values, or 128 e4m3 codes (KV8)
   static constexpr int kColsPerPanel = KV8 ? 128 : 64;
   static constexpr int kPanels = D / kColsPerPanel;
@@ -47,6 +51,42 @@ struct SchedShared {
   int nC, b, merge_flag, abort_flag;
 };
 
+// e4m3 caches: a query row (16 words of two values per thread, 4 threads per row, neighbouring lanes)
+// as f16 pairs. bf16 rows are multiplied by the power of two 2^k that puts the row's largest magnitude
+// in [2^14, 2^15) (exact for every element down to 2^-29 of it); returns 2^-k, which the logit scale
+// takes. f16 rows are used as they are.
+template <typename T>
+__device__ __forceinline__ float q_row_to_f16(uint32_t (&w)[16]) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    float mx = 0.f;
+#pragma unroll
+    for (int v = 0; v < 16; ++v)
+      mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[v] << 16)), fabsf(__uint_as_float(w[v] & 0xffff0000u))));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    int k = 0;
+    if (mx > 0.f && mx <= FLT_MAX) {
+      const int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
+      k = 14 - e < 64 ? 14 - e : 64;
+    }
+    const float up = __uint_as_float(static_cast<uint32_t>(127 + k) << 23);
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+      const __half2 hv = __floats2half2_rn(__uint_as_float(w[v] << 16) * up, __uint_as_float(w[v] & 0xffff0000u) * up);
+      w[v] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    return __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
+  } else {
+    return 1.f;
+  }
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 template <typename T, int D, int MT, bool KV8>
 __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     verify_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -61,6 +101,10 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
   constexpr int DT = D / 8;           // 8-wide d tiles of the output
   constexpr int KSTEPS = D / 16;      // k steps of Q K^T
   constexpr int ROWS = Cfg::kRows;
+  constexpr bool SW = Cfg::kSwap;
+  constexpr int MTS = SW ? 1 : MT;     // query row tiles (the swapped form has one of 8 rows)
+  constexpr int NM = KW / 16;         // swapped form: 16-key m tiles per warp and tile
+  constexpr int OT = SW ? D / 16 : DT;   // output accumulator tiles (16 head dims x 8 rows when swapped)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -196,8 +240,8 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
   }
 
   // -------------------------------------------------------------------- consumer warps
-  const int mt = warp % MT;
-  const int kg = warp / MT;
+  const int mt = warp % MTS;
+  const int kg = warp / MTS;
   const int gq = lane >> 2;
   const int tq = lane & 3;
   int stage = 0;
@@ -229,14 +273,50 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     uint32_t mw[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      Rrow[h] = rg * ROWS + mt * 16 + gq + 8 * h;
+      // swapped form: the thread's S^T columns (queries 2tq, 2tq+1); otherwise rows gq, gq+8
+      Rrow[h] = SW ? rg * ROWS + 2 * tq + h : rg * ROWS + mt * 16 + gq + 8 * h;
       rvalid[h] = Rrow[h] < p.G * n;
       mw[h] = rvalid[h] ? (__ldg(p.tree_mask_bits + static_cast<int64_t>(b) * p.C + Rrow[h] / p.G) & nmask) : 0u;
     }
-    // Q fragments (A operand of m16n8k16): rows gq / gq+8, columns 2*tq.. of each 16-wide k step
-    uint32_t qf[KSTEPS][4];
-    float sl2r[2] = {sl2, sl2};   // logit scale of this thread's two rows (base 2)
-    {
+    // Q fragments: the A operand of m16n8k16 (rows gq / gq+8, columns 2*tq.. of each 16-wide k step), or
+    // in the swapped form the B operand (query row gq, the same columns)
+    uint32_t qf[KSTEPS][SW ? 2 : 4];
+    float sl2r[2] = {sl2, sl2};   // logit scale of this thread's two rows / columns (base 2)
+    if constexpr (SW) {
+      const int Rq = rg * ROWS + gq;
+      const bool qv = Rq < p.G * n;
+      const uint32_t* qr = reinterpret_cast<const uint32_t*>(
+          static_cast<const T*>(p.q) +
+          ((static_cast<int64_t>(b) * p.C + (qv ? Rq / p.G : 0)) * p.Hq + g * p.G + (qv ? Rq % p.G : 0)) * D);
+      if constexpr (!KV8) {
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          qf[kk][0] = qv ? __ldg(qr + kk * 8 + tq) : 0u;
+          qf[kk][1] = qv ? __ldg(qr + kk * 8 + 4 + tq) : 0u;
+        }
+      } else {
+        // permuted k order (as below): k step kk, pair j takes head dims tq*32 + kk*4 + 2j (+1)
+        uint32_t w[16];
+        const uint4* q4 = reinterpret_cast<const uint4*>(qr + tq * 16);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 x = qv ? __ldg(q4 + v) : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * v] = x.x;
+          w[4 * v + 1] = x.y;
+          w[4 * v + 2] = x.z;
+          w[4 * v + 3] = x.w;
+        }
+        const float down = q_row_to_f16<T>(w);
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          qf[kk][0] = w[2 * kk];
+          qf[kk][1] = w[2 * kk + 1];
+        }
+        // the scale of query column c sits with the lanes that loaded row c (lane c * 4)
+        sl2r[0] = sl2 * __shfl_sync(0xffffffffu, down, (2 * tq) * 4);
+        sl2r[1] = sl2 * __shfl_sync(0xffffffffu, down, (2 * tq + 1) * 4);
+      }
+    } else {
       const uint32_t* qrow[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -255,9 +335,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
       } else {
         // The k order of Q K^T is permuted (the sum does not depend on it) so that a thread's K codes
         // are 32 consecutive bytes of the key row: k step kk, A/B pair j (0: k = 2tq, 2tq+1; 1: k =
-        // 2tq+8, 2tq+9) takes head dims tq*32 + kk*4 + 2j (+1). bf16 queries go to f16 times a
-        // power of two per row that puts the row's largest magnitude in [2^14, 2^15) (exact for
-        // every element down to 2^-29 of it); the logit scale takes the inverse power.
+        // 2tq+8, 2tq+9) takes head dims tq*32 + kk*4 + 2j (+1).
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t w[16];
@@ -270,27 +348,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
             w[4 * v + 2] = x.z;
             w[4 * v + 3] = x.w;
           }
-          if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-            float mx = 0.f;
-#pragma unroll
-            for (int v = 0; v < 16; ++v)
-              mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[v] << 16)), fabsf(__uint_as_float(w[v] & 0xffff0000u))));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            int k = 0;
-            if (mx > 0.f && mx <= FLT_MAX) {
-              const int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
-              k = 14 - e < 64 ? 14 - e : 64;
-            }
-            const float up = __uint_as_float(static_cast<uint32_t>(127 + k) << 23);
-            sl2r[h] = sl2 * __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
-#pragma unroll
-            for (int v = 0; v < 16; ++v) {
-              const __half2 hv = __floats2half2_rn(__uint_as_float(w[v] << 16) * up,
-                                                   __uint_as_float(w[v] & 0xffff0000u) * up);
-              w[v] = *reinterpret_cast<const uint32_t*>(&hv);
-            }
-          }
+          sl2r[h] = sl2 * q_row_to_f16<T>(w);
 #pragma unroll
           for (int kk = 0; kk < KSTEPS; ++kk) {
             qf[kk][h] = w[2 * kk];
@@ -301,9 +359,9 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     }
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.f, 0.f};
-    float o[DT][4];
+    float o[OT][4];
 #pragma unroll
-    for (int dt = 0; dt < DT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+    for (int dt = 0; dt < OT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
 
     for (int tl = tbegin; tl < tend; ++tl) {
       const int key0 = tl * Cfg::kTile;
@@ -330,6 +388,159 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
         __syncwarp();
       }
       if (ready) {
+        if constexpr (SW) {
+          // ---- swapped form. S^T = K Q^T: m tile m holds keys wkey0 + m*16 .. +15 (rows gq, gq+8 of the
+          // C fragment) and the 8 query columns (2tq, 2tq+1); even and odd k steps go to separate
+          // accumulators to halve the dependent MMA chain.
+          float s[NM][4];
+          {
+            float s2[NM][4];
+#pragma unroll
+            for (int m = 0; m < NM; ++m)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) s[m][e] = s2[m][e] = 0.f;
+            if constexpr (!KV8) {
+#pragma unroll
+              for (int kk = 0; kk < KSTEPS; ++kk) {
+#pragma unroll
+                for (int m = 0; m < NM; ++m) {
+                  // A = K rows (keys x head dims), row-major: the four 8x8 pieces of ldmatrix
+                  const int key = wkey0 + m * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                  const int d = kk * 16 + (lane >> 4) * 8;
+                  const int c = (d & 63) >> 3;
+                  const uint32_t addr = kbase + (d >> 6) * Cfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4);
+                  uint32_t a[4];
+                  ldsm_x4(addr, a[0], a[1], a[2], a[3]);
+                  MOp::run((kk & 1) ? s2[m] : s[m], a, qf[kk][0], qf[kk][1]);
+                }
+              }
+            } else {
+              // permuted k order: the A pairs of k step kk are word kk of the 32 bytes at head dim tq*32
+              // of key rows gq and gq+8 (both with row & 7 == gq)
+#pragma unroll
+              for (int m = 0; m < NM; ++m) {
+                const uint32_t r0 = kbase + (wkey0 + m * 16 + gq) * 128;
+                const uint32_t r1 = r0 + 8 * 128;
+                const uint32_t c0 = ((2 * tq) ^ gq) << 4, c1 = ((2 * tq + 1) ^ gq) << 4;
+                const uint4 x00 = lds_v4(r0 + c0), x01 = lds_v4(r0 + c1);
+                const uint4 x10 = lds_v4(r1 + c0), x11 = lds_v4(r1 + c1);
+                const uint32_t k0[8] = {x00.x, x00.y, x00.z, x00.w, x01.x, x01.y, x01.z, x01.w};
+                const uint32_t k1[8] = {x10.x, x10.y, x10.z, x10.w, x11.x, x11.y, x11.z, x11.w};
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk) {
+                  uint32_t a[4];
+                  a[0] = e4m3x2_to_f16x2(k0[kk]);
+                  a[1] = e4m3x2_to_f16x2(k1[kk]);
+                  a[2] = e4m3x2_to_f16x2(k0[kk] >> 16);
+                  a[3] = e4m3x2_to_f16x2(k1[kk] >> 16);
+                  MOp::run((kk & 1) ? s2[m] : s[m], a, qf[kk][0], qf[kk][1]);
+                }
+              }
+            }
+#pragma unroll
+            for (int m = 0; m < NM; ++m)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) s[m][e] += s2[m][e];
+          }
+          // scale, mask (element e: key gq + 8*(e>>1) of the m tile, query column 2tq + (e&1))
+          const bool need_mask = key0 + Cfg::kTile > P;
+#pragma unroll
+          for (int m = 0; m < NM; ++m) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float v = s[m][e] * sl2r[e & 1];
+              if (need_mask) {
+                const int key = key0 + wkey0 + m * 16 + gq + 8 * (e >> 1);
+                const bool vis = key < P || (key < L && ((mw[e & 1] >> ((key - P) & 31)) & 1u));
+                v = vis ? v : -INFINITY;
+              }
+              s[m][e] = v;
+            }
+          }
+          // online softmax per query column: its keys are spread over the 8 lanes of equal tq
+          float alpha[2];
+#pragma unroll
+          for (int jq = 0; jq < 2; ++jq) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int m = 0; m < NM; ++m) mx = fmaxf(mx, fmaxf(s[m][jq], s[m][2 + jq]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float m_new = fmaxf(m_run[jq], mx);
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            alpha[jq] = fast_exp2(m_run[jq] - m_use);
+            m_run[jq] = m_new;
+            float rs = 0.f;
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+              const float p0 = fast_exp2(s[m][jq] - m_use);
+              const float p1 = fast_exp2(s[m][2 + jq] - m_use);
+              s[m][jq] = p0;
+              s[m][2 + jq] = p1;
+              rs += p0 + p1;
+            }
+            l_run[jq] = l_run[jq] * alpha[jq] + rs;
+          }
+          if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+#pragma unroll
+            for (int md = 0; md < OT; ++md) {
+              o[md][0] *= alpha[0];
+              o[md][1] *= alpha[1];
+              o[md][2] *= alpha[0];
+              o[md][3] *= alpha[1];
+            }
+          }
+          // O^T += V^T P^T, one k step per m tile of S^T. P^T's B fragment is the transpose of the
+          // thread's C fragment: pack (keys gq / gq+8 x columns 2tq, 2tq+1) as 8x8 b16 pieces and
+          // transpose them across the warp.
+#pragma unroll
+          for (int ks = 0; ks < NM; ++ks) {
+            const uint32_t pb0 = movmatrix_trans(MOp::pack(s[ks][0], s[ks][1]));
+            const uint32_t pb1 = movmatrix_trans(MOp::pack(s[ks][2], s[ks][3]));
+            if constexpr (!KV8) {
+#pragma unroll
+              for (int md = 0; md < OT; ++md) {
+                // A = V^T (head dims x keys): V rows read transposed; m rows gq / gq+8 are head dims
+                // md*16 + gq / + 8
+                const int key = wkey0 + ks * 16 + (lane & 7) + ((lane >> 4) << 3);
+                const int d = md * 16 + ((lane >> 3) & 1) * 8;
+                const int c = (d & 63) >> 3;
+                const uint32_t addr = vbase + (d >> 6) * Cfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4);
+                uint32_t a[4];
+                ldsm_x4_trans(addr, a[0], a[1], a[2], a[3]);
+                MOp::run(o[md], a, pb0, pb1);
+              }
+            } else {
+              // permuted head dims: m rows gq / gq+8 of m tile md are head dims gq*16 + md / + 8, so
+              // the A pairs are bytes md and 8 + md of chunk gq of key rows 2tq, 2tq+1, 2tq+8, 2tq+9
+              const int kr = wkey0 + ks * 16 + 2 * tq;
+              const uint4 x0 = lds_v4(vbase + kr * 128 + ((gq ^ (2 * tq)) << 4));
+              const uint4 x1 = lds_v4(vbase + (kr + 1) * 128 + ((gq ^ (2 * tq + 1)) << 4));
+              const uint4 x2 = lds_v4(vbase + (kr + 8) * 128 + ((gq ^ (2 * tq)) << 4));
+              const uint4 x3 = lds_v4(vbase + (kr + 9) * 128 + ((gq ^ (2 * tq + 1)) << 4));
+              const uint32_t r0[4] = {x0.x, x0.y, x0.z, x0.w}, r1[4] = {x1.x, x1.y, x1.z, x1.w};
+              const uint32_t r2[4] = {x2.x, x2.y, x2.z, x2.w}, r3[4] = {x3.x, x3.y, x3.z, x3.w};
+#pragma unroll
+              for (int wd = 0; wd < 2; ++wd) {
+#pragma unroll
+                for (int i = 0; i < 4; i += 2) {
+                  const uint32_t sel = i | ((4 + i) << 4) | ((i + 1) << 8) | ((5 + i) << 12);
+                  const uint32_t a0 = byte_perm(r0[wd], r1[wd], sel);
+                  const uint32_t a1 = byte_perm(r0[wd + 2], r1[wd + 2], sel);
+                  const uint32_t a2 = byte_perm(r2[wd], r3[wd], sel);
+                  const uint32_t a3 = byte_perm(r2[wd + 2], r3[wd + 2], sel);
+                  const uint32_t lo[4] = {e4m3x2_to_f16x2(a0), e4m3x2_to_f16x2(a1), e4m3x2_to_f16x2(a2),
+                                          e4m3x2_to_f16x2(a3)};
+                  MOp::run(o[4 * wd + i], lo, pb0, pb1);
+                  const uint32_t hi[4] = {e4m3x2_to_f16x2(a0 >> 16), e4m3x2_to_f16x2(a1 >> 16),
+                                          e4m3x2_to_f16x2(a2 >> 16), e4m3x2_to_f16x2(a3 >> 16)};
+                  MOp::run(o[4 * wd + i + 1], hi, pb0, pb1);
+                }
+              }
+            }
+          }
+        } else {
         float s[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
@@ -458,6 +669,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
             }
           }
         }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(empty_bar + stage));
@@ -468,13 +680,25 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     }
 
     // ---------------------------------------------------------------- segment epilogue
+    // row sums: over the 4 lanes of a row, or (swapped form) over the 8 lanes of a query column
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
-      l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
+      if constexpr (SW) {
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 4);
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 8);
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 16);
+      } else {
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
+      }
     }
     if constexpr (KG > 1) {
-      if (tq == 0) {
+      if constexpr (SW) {
+        if (gq == 0) {
+          m_pub[warp * 8 + 2 * tq] = m_run[0];
+          m_pub[warp * 8 + 2 * tq + 1] = m_run[1];
+        }
+      } else if (tq == 0) {
         m_pub[warp * 16 + gq] = m_run[0];
         m_pub[warp * 16 + gq + 8] = m_run[1];
       }
@@ -483,23 +707,29 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
       for (int h = 0; h < 2; ++h) {
         float mstar = -INFINITY;
 #pragma unroll
-        for (int k2 = 0; k2 < KG; ++k2) mstar = fmaxf(mstar, m_pub[(mt + k2 * MT) * 16 + gq + 8 * h]);
+        for (int k2 = 0; k2 < KG; ++k2)
+          mstar = fmaxf(mstar, SW ? m_pub[k2 * 8 + 2 * tq + h] : m_pub[(mt + k2 * MTS) * 16 + gq + 8 * h]);
         const float f = (m_run[h] == -INFINITY) ? 0.f : fast_exp2(m_run[h] - mstar);
         l_run[h] *= f;
 #pragma unroll
-        for (int dt = 0; dt < DT; ++dt) {
-          o[dt][2 * h] *= f;
-          o[dt][2 * h + 1] *= f;
+        for (int dt = 0; dt < OT; ++dt) {
+          if constexpr (SW) {   // elements h and 2 + h belong to query column 2tq + h
+            o[dt][h] *= f;
+            o[dt][2 + h] *= f;
+          } else {
+            o[dt][2 * h] *= f;
+            o[dt][2 * h + 1] *= f;
+          }
         }
         m_run[h] = mstar;
       }
       // deterministic sequential sum of the key groups' partial O through one scratch tile
-      for (int mr = 0; mr < MT; ++mr) {
+      for (int mr = 0; mr < MTS; ++mr) {
         for (int kr = 0; kr < KG; ++kr) {
           if (mt == mr && kg == kr) {
             if (kr > 0) {
 #pragma unroll
-              for (int dt = 0; dt < DT; ++dt)
+              for (int dt = 0; dt < OT; ++dt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) o[dt][e] += scratch[(dt * 4 + e) * 32 + lane];
               l_run[0] += scratch_l[lane];
@@ -507,7 +737,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
             }
             if (kr < KG - 1) {
 #pragma unroll
-              for (int dt = 0; dt < DT; ++dt)
+              for (int dt = 0; dt < OT; ++dt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) scratch[(dt * 4 + e) * 32 + lane] = o[dt][e];
               scratch_l[lane] = l_run[0];
@@ -522,7 +752,58 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
     const bool whole_unit = (tbegin == 0 && tend == Tb);
     const int64_t unit_base = base_b + static_cast<int64_t>(j) * Tb;
     const int slot = 2 * static_cast<int>(blockIdx.x) + (first_segment ? 0 : 1);
-    if (owner) {
+    if (owner && SW) {
+      // stage the normalised rows in shared memory ([8][D] floats, free once the key groups are summed),
+      // then write them row by row with whole-row coalesced stores
+      float* so = scratch;
+      float inv[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        inv[h] = (l_run[h] > 0.f ? 1.f / l_run[h] : 0.f) * vsc;
+        if (gq == 0) scratch_l[2 * tq + h] = l_run[h] > 0.f ? m_run[h] + __log2f(l_run[h]) : -INFINITY;
+      }
+#pragma unroll
+      for (int md = 0; md < OT; ++md) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          // head dim of m row gq (e < 2) or gq + 8: md*16 + gq (+8), or gq*16 + md (+8) for e4m3 caches
+          const int hd = KV8 ? gq * 16 + (e >> 1) * 8 + md : md * 16 + (e >> 1) * 8 + gq;
+          so[(2 * tq + (e & 1)) * D + hd] = o[md][e] * inv[e & 1];
+        }
+      }
+      __syncwarp();
+      constexpr int PER = D / 32;   // values per lane and row
+#pragma unroll 1
+      for (int r = 0; r < ROWS; ++r) {
+        const int R = rg * ROWS + r;
+        const float* src = so + r * D + lane * PER;
+        if (whole_unit) {
+          if (R < p.G * p.C) {
+            const bool valid = R < p.G * n;
+            T* dst = static_cast<T*>(p.out) +
+                     ((static_cast<int64_t>(b) * p.C + R / p.G) * p.Hq + g * p.G + R % p.G) * D + lane * PER;
+            if constexpr (PER == 4) {
+              uint2 x = make_uint2(0u, 0u);
+              if (valid) {
+                x.x = Op::pack(src[0], src[1]);
+                x.y = Op::pack(src[2], src[3]);
+              }
+              *reinterpret_cast<uint2*>(dst) = x;
+            } else {
+              *reinterpret_cast<uint32_t*>(dst) = valid ? Op::pack(src[0], src[1]) : 0u;
+            }
+          }
+        } else {
+          float* dst = p.part_o + (static_cast<int64_t>(slot) * ROWS + r) * D + lane * PER;
+          if constexpr (PER == 4)
+            __stcg(reinterpret_cast<float4*>(dst), make_float4(src[0], src[1], src[2], src[3]));
+          else
+            __stcg(reinterpret_cast<float2*>(dst), make_float2(src[0], src[1]));
+          if (lane == 0) __stcg(p.part_lse + static_cast<int64_t>(slot) * ROWS + r, scratch_l[r]);
+        }
+      }
+      __syncwarp();
+    } else if (owner) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int R = Rrow[h];
