@@ -474,6 +474,7 @@ def run_ours(args, world, rank, local):
     }
     if kv8 is not None:
         kv8["attention_frac"] = kv8["attention_GBps"] / peak
+        kv8["traffic"] = recorded_traffic(f"{args.workload}_e4m3")
         kv8["attention_speedup_vs_16bit"] = attn_ms / (kv8["attention_us"] * 1e-3)
     accept["argmax_roofline"]["peak"] = peak
     accept["argmax_roofline"]["frac"] = accept["argmax_roofline"]["achieved"] / peak

@@ -57,6 +57,7 @@ typedef int32_t taco_status;
 #define TACO_DEVERR_SLOT 0x8u           /* slot_offsets[b][i] >= maxblk * bs */
 #define TACO_DEVERR_WAIT_TIMEOUT 0x10u  /* a pipeline wait gave up (the kernel returned early) */
 #define TACO_DEVERR_PARENT 0x20u        /* parents[b][i] outside [-1, i) */
+#define TACO_DEVERR_TABLE_FULL 0x40u    /* prefix_cache_insert probed every slot without a place */
 
 /*
  * paged_tree_attention: masked softmax attention of every candidate query over its sequence's
@@ -140,10 +141,12 @@ taco_status paged_tree_attention_noalloc(const void* q, const void* k_cache, con
 
 /*
  * 8-bit KV cache. The 53ai.com workshop page (section "5. 支持 Quantization（模型量化）") lists 8-bit
- * (INT8 / FP8) storage among the engine's features for its lower memory and bandwidth needs, and the
- * 17173xz.com overview counts quantised operators among its kernels; neither fixes a format. These
- * calls use e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinities; 0x7F / 0xFF
- * are NaN; largest finite 448) with one float32 scale per KV head for K and one for V:
+ * (INT8 / FP8) storage among the engine's features for its lower memory and bandwidth needs, the
+ * 618zxw.cn page (section "LLM量子化技術による推論コストの削減") has quantised attention operators with
+ * fast dequantisation, and the 17173xz.com overview counts quantised operators among its kernels; none
+ * fixes a format. These calls use e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities; 0x7F / 0xFF are NaN; largest finite 448) with one float32 scale per KV head for K and
+ * one for V:
  *   stored code  = e4m3(x / scale[h])  (float32 quotient correctly rounded, then the nearest e4m3 value,
  *                  ties to the even code, magnitudes above 448 saturate to 448, NaN stays NaN)
  *   value read   = decode(code) * scale[h]
@@ -234,6 +237,59 @@ taco_status tree_greedy_accept(const int32_t* target_argmax, const int32_t* cand
                                const int32_t* parents, const int32_t* num_candidates, const int32_t* context_lens,
                                int32_t batch, int32_t max_candidates, int32_t* accept_len, int32_t* accepted_path,
                                int32_t* bonus_token, int32_t* slot_offsets_out, void* stream);
+
+/*
+ * Prefix-tree KV lookup for prefill. The 618zxw.cn page (section "プレフィックスキャッシュ技術を使用して
+ * TTFTを削減する"), the 17173xz.com overview's prefill paragraph and the tencentcloud.com document's list
+ * of techniques keep earlier requests' prefill KV in a prefix tree, so that prefill becomes a lookup of
+ * cached KV and only the tokens not found are computed. Here a node is one full KV block of block_size
+ * tokens, identified by the whole token prefix it ends; it owns the physical block holding that
+ * prefix's K/V. A partial trailing block is never cached or matched.
+ *
+ * The tree lives in caller-owned device memory:
+ *   slot_keys    uint64 [capacity]  open-addressing table of node keys, 8-byte aligned; 0 = empty.
+ *                                   Set every entry to 0 once before the first insert.
+ *   slot_nodes   int32  [capacity]  node (physical block) of each claimed slot; set every entry to -1
+ *                                   once, together with slot_keys.
+ *   node_parent  int32  [NB]        node of the prefix one block shorter, -1 for a first block
+ *   node_depth   int32  [NB]        the node's block index within its sequence (0 = first block)
+ *   node_tokens  int32  [NB, block_size]  the node's tokens
+ * capacity is a power of two; keep it at least twice the number of nodes (probe chains stay short).
+ * A key is a 64-bit hash of the whole prefix; every match is confirmed on depth, parent and tokens, so a
+ * hash collision never changes a result. Inserts and lookups that overlap on the GPU race: order them.
+ *
+ * Sequences (both calls): tokens int32 [total]; sequence b is tokens[seq_starts[b] .. seq_starts[b+1])
+ * (seq_starts int32 [batch + 1], non-decreasing: a decreasing pair sets TACO_DEVERR_CONTEXT_LEN and
+ * counts as empty). Only the first min(len_b / block_size, max_blocks_per_seq) full blocks are used.
+ *
+ * prefix_cache_lookup: per sequence, the longest run of its leading full blocks whose path is in the
+ *   tree. out_blocks int32 [batch, max_blocks_per_seq]: the path's physical blocks (a block-table
+ *   prefix), then -1; out_matched int32 [batch]: the run's length in blocks (matched tokens = that
+ *   times block_size).
+ *
+ * prefix_cache_insert: add the full blocks of each sequence, whose K/V sit in block_tables int32
+ *   [batch, max_blocks_per_seq] (entries in [0, NB)). A block whose prefix is already a node keeps that
+ *   node; otherwise the sequence's own block becomes the node (its node_* entries are written). When
+ *   several sequences of one call add the same new prefix, one of their blocks becomes the node (which
+ *   one is not fixed) and all of them get it. out_blocks [batch, max_blocks_per_seq]: per full block,
+ *   the physical block that holds its prefix afterwards (blocks that did not become nodes can be
+ *   freed), then -1. out_inserted int32 [batch] (may be NULL): blocks processed per sequence. A block
+ *   id outside [0, NB) sets TACO_DEVERR_BLOCK_ID, and a table with no free slot on the chain sets
+ *   TACO_DEVERR_TABLE_FULL; either ends that sequence's walk. A bounded wait for another sequence's
+ *   node that times out sets TACO_DEVERR_WAIT_TIMEOUT. A block id that is already a node must not be
+ *   passed for a block whose prefix is new.
+ */
+taco_status prefix_cache_lookup(const int32_t* tokens, const int32_t* seq_starts, const uint64_t* slot_keys,
+                                const int32_t* slot_nodes, int64_t capacity, const int32_t* node_parent,
+                                const int32_t* node_depth, const int32_t* node_tokens, int32_t* out_blocks,
+                                int32_t* out_matched, int32_t batch, int32_t block_size, int32_t num_blocks,
+                                int32_t max_blocks_per_seq, void* stream);
+
+taco_status prefix_cache_insert(const int32_t* tokens, const int32_t* seq_starts, const int32_t* block_tables,
+                                uint64_t* slot_keys, int32_t* slot_nodes, int64_t capacity, int32_t* node_parent,
+                                int32_t* node_depth, int32_t* node_tokens, int32_t* out_blocks,
+                                int32_t* out_inserted, int32_t batch, int32_t block_size, int32_t num_blocks,
+                                int32_t max_blocks_per_seq, void* stream);
 
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char* taco_attn_last_error(void);

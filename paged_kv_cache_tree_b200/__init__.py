@@ -4,6 +4,7 @@ The compute path is the C-ABI library ``libtaco_attn.so`` built from ``csrc/`` f
 functions below only marshal torch tensors into its pointers and sizes.
 """
 from ._lib import (  # noqa: F401
+    PrefixCache,
     TACO_OPT_GRID_CTAS,
     TACO_OPT_KERNEL,
     TacoError,

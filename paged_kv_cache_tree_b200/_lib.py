@@ -42,6 +42,8 @@ EXPORTED = (
     "tree_mask_from_parents",
     "logits_argmax",
     "tree_greedy_accept",
+    "prefix_cache_lookup",
+    "prefix_cache_insert",
 )
 
 _lib = None
@@ -88,6 +90,11 @@ def load() -> ctypes.CDLL:
     lib.logits_argmax.restype = i32
     lib.tree_greedy_accept.argtypes = [vp] * 5 + [i32, i32] + [vp] * 4 + [vp]
     lib.tree_greedy_accept.restype = i32
+    i64 = ctypes.c_int64
+    lib.prefix_cache_lookup.argtypes = [vp] * 4 + [i64] + [vp] * 5 + [i32] * 4 + [vp]
+    lib.prefix_cache_lookup.restype = i32
+    lib.prefix_cache_insert.argtypes = [vp] * 5 + [i64] + [vp] * 5 + [i32] * 4 + [vp]
+    lib.prefix_cache_insert.restype = i32
     _lib = lib
     return lib
 
@@ -329,3 +336,69 @@ def release_workspace() -> None:
 
 def version() -> int:
     return int(load().taco_attn_version())
+
+
+class PrefixCache:
+    """Device memory of a prefix tree of full KV blocks (see prefix_cache_* in include/taco_attn.h):
+    an open-addressing slot table and per-physical-block node arrays, allocated and initialised here
+    with torch (plumbing only); lookups and inserts run in the library's kernels."""
+
+    def __init__(self, num_blocks: int, block_size: int, capacity: int, device="cuda"):
+        if capacity < 2 or capacity & (capacity - 1):
+            raise ValueError("capacity must be a power of two >= 2")
+        self.num_blocks, self.block_size, self.capacity = int(num_blocks), int(block_size), int(capacity)
+        self.slot_keys = torch.zeros(capacity, dtype=torch.int64, device=device)     # uint64 bit patterns
+        self.slot_nodes = torch.full((capacity,), -1, dtype=torch.int32, device=device)
+        self.node_parent = torch.full((num_blocks,), -1, dtype=torch.int32, device=device)
+        self.node_depth = torch.full((num_blocks,), -1, dtype=torch.int32, device=device)
+        self.node_tokens = torch.zeros((num_blocks, block_size), dtype=torch.int32, device=device)
+
+    @staticmethod
+    def _check_seqs(tokens, seq_starts):
+        _need_cuda("tokens", tokens, torch.int32, 1)
+        _need_cuda("seq_starts", seq_starts, torch.int32, 1)
+        if seq_starts.shape[0] < 1:
+            raise ValueError("seq_starts must hold batch + 1 offsets")
+        if tokens.numel() == 0:   # the C ABI wants a real pointer even when no token is read
+            tokens = torch.zeros(1, dtype=torch.int32, device=tokens.device)
+        return seq_starts.shape[0] - 1, tokens
+
+    def lookup(self, tokens, seq_starts, max_blocks: int, out_blocks=None, out_matched=None, stream=None):
+        """Longest cached run of each sequence's leading full blocks: (out_blocks [B, max_blocks]
+        physical blocks then -1, out_matched [B] blocks matched)."""
+        B, tokens = self._check_seqs(tokens, seq_starts)
+        if out_blocks is None:
+            out_blocks = torch.empty((B, max_blocks), dtype=torch.int32, device=tokens.device)
+        if out_matched is None:
+            out_matched = torch.empty((B,), dtype=torch.int32, device=tokens.device)
+        _need_cuda("out_blocks", out_blocks, torch.int32, 2)
+        _need_cuda("out_matched", out_matched, torch.int32, 1)
+        if tuple(out_blocks.shape) != (B, max_blocks) or out_matched.shape[0] != B:
+            raise ValueError("out_blocks must be [B, max_blocks] and out_matched [B]")
+        _check(load().prefix_cache_lookup(
+            tokens.data_ptr(), seq_starts.data_ptr(), self.slot_keys.data_ptr(), self.slot_nodes.data_ptr(),
+            self.capacity, self.node_parent.data_ptr(), self.node_depth.data_ptr(), self.node_tokens.data_ptr(),
+            out_blocks.data_ptr(), out_matched.data_ptr(), B, self.block_size, self.num_blocks, max_blocks,
+            _stream_handle(stream, tokens.device)))
+        return out_blocks, out_matched
+
+    def insert(self, tokens, seq_starts, block_tables, out_blocks=None, out_inserted=None, stream=None):
+        """Insert each sequence's full blocks (K/V in block_tables [B, max_blocks]); returns
+        (out_blocks [B, max_blocks]: the block holding each prefix afterwards, then -1; out_inserted [B])."""
+        B, tokens = self._check_seqs(tokens, seq_starts)
+        _need_cuda("block_tables", block_tables, torch.int32, 2)
+        if block_tables.shape[0] != B:
+            raise ValueError("block_tables must be [B, max_blocks]")
+        max_blocks = block_tables.shape[1]
+        if out_blocks is None:
+            out_blocks = torch.empty((B, max_blocks), dtype=torch.int32, device=tokens.device)
+        if out_inserted is None:
+            out_inserted = torch.empty((B,), dtype=torch.int32, device=tokens.device)
+        _need_cuda("out_blocks", out_blocks, torch.int32, 2)
+        _need_cuda("out_inserted", out_inserted, torch.int32, 1)
+        _check(load().prefix_cache_insert(
+            tokens.data_ptr(), seq_starts.data_ptr(), block_tables.data_ptr(), self.slot_keys.data_ptr(),
+            self.slot_nodes.data_ptr(), self.capacity, self.node_parent.data_ptr(), self.node_depth.data_ptr(),
+            self.node_tokens.data_ptr(), out_blocks.data_ptr(), out_inserted.data_ptr(), B, self.block_size,
+            self.num_blocks, max_blocks, _stream_handle(stream, tokens.device)))
+        return out_blocks, out_inserted

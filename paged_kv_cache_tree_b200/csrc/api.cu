@@ -17,7 +17,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAbiVersion = 3;
+constexpr int kAbiVersion = 4;
 
 thread_local std::string g_last_error;
 
@@ -264,7 +264,7 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   }
   int grid = static_cast<int>(g_opt_grid);
-  if (grid == 0) grid = (use_tc ? 1 : 2) * g_ws[dev].sm_count;
+  if (grid == 0) grid = (use_tc ? 1 : taco::mma_ctas_per_sm(rows)) * g_ws[dev].sm_count;
   const size_t slots = 2 * static_cast<size_t>(grid);
   st = ensure_workspace(dev, static_cast<size_t>(units), slots * rows, slots * rows * head_dim);
   if (st != TACO_OK) return st;
@@ -471,6 +471,60 @@ taco_status tree_greedy_accept(const int32_t* target_argmax, const int32_t* cand
   return TACO_OK;
 }
 
+static taco_status prefix_common(const int32_t* tokens, const int32_t* seq_starts, const void* slot_keys,
+                                 const void* slot_nodes, int64_t capacity, const void* node_parent,
+                                 const void* node_depth, const void* node_tokens, const void* out_blocks,
+                                 int32_t batch, int32_t block_size, int32_t num_blocks, int32_t max_blocks,
+                                 uint32_t** err) {
+  if (!tokens || !seq_starts || !slot_keys || !slot_nodes || !node_parent || !node_depth || !node_tokens ||
+      !out_blocks)
+    return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if ((reinterpret_cast<uintptr_t>(slot_keys) & 7u) != 0) return fail(TACO_ERR_INVALID_ARG, "slot_keys must be 8-byte aligned");
+  if (capacity < 2 || (capacity & (capacity - 1)) != 0) return fail(TACO_ERR_INVALID_ARG, "capacity must be a power of two >= 2");
+  if (batch < 0) return fail(TACO_ERR_INVALID_ARG, "batch must be >= 0");
+  if (block_size < 1 || block_size > 1024) return fail(TACO_ERR_UNSUPPORTED, "block_size must be in [1, 1024]");
+  if (num_blocks < 1) return fail(TACO_ERR_INVALID_ARG, "num_blocks must be >= 1");
+  if (max_blocks < 1) return fail(TACO_ERR_INVALID_ARG, "max_blocks_per_seq must be >= 1");
+  if (batch == 0) return TACO_OK;
+  return device_error_word(err);
+}
+
+taco_status prefix_cache_lookup(const int32_t* tokens, const int32_t* seq_starts, const uint64_t* slot_keys,
+                                const int32_t* slot_nodes, int64_t capacity, const int32_t* node_parent,
+                                const int32_t* node_depth, const int32_t* node_tokens, int32_t* out_blocks,
+                                int32_t* out_matched, int32_t batch, int32_t block_size, int32_t num_blocks,
+                                int32_t max_blocks_per_seq, void* stream) {
+  if (!out_matched) return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  uint32_t* err = nullptr;
+  taco_status st = prefix_common(tokens, seq_starts, slot_keys, slot_nodes, capacity, node_parent, node_depth,
+                                 node_tokens, out_blocks, batch, block_size, num_blocks, max_blocks_per_seq, &err);
+  if (st != TACO_OK || batch == 0) return st;
+  cudaError_t e = taco::launch_prefix_cache(false, tokens, seq_starts, nullptr, const_cast<uint64_t*>(slot_keys),
+                                            const_cast<int32_t*>(slot_nodes), capacity, const_cast<int32_t*>(node_parent),
+                                            const_cast<int32_t*>(node_depth), const_cast<int32_t*>(node_tokens),
+                                            out_blocks, out_matched, err, batch, block_size, num_blocks,
+                                            max_blocks_per_seq, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prefix lookup launch");
+  return TACO_OK;
+}
+
+taco_status prefix_cache_insert(const int32_t* tokens, const int32_t* seq_starts, const int32_t* block_tables,
+                                uint64_t* slot_keys, int32_t* slot_nodes, int64_t capacity, int32_t* node_parent,
+                                int32_t* node_depth, int32_t* node_tokens, int32_t* out_blocks,
+                                int32_t* out_inserted, int32_t batch, int32_t block_size, int32_t num_blocks,
+                                int32_t max_blocks_per_seq, void* stream) {
+  if (!block_tables) return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  uint32_t* err = nullptr;
+  taco_status st = prefix_common(tokens, seq_starts, slot_keys, slot_nodes, capacity, node_parent, node_depth,
+                                 node_tokens, out_blocks, batch, block_size, num_blocks, max_blocks_per_seq, &err);
+  if (st != TACO_OK || batch == 0) return st;
+  cudaError_t e = taco::launch_prefix_cache(true, tokens, seq_starts, block_tables, slot_keys, slot_nodes, capacity,
+                                            node_parent, node_depth, node_tokens, out_blocks, out_inserted, err, batch,
+                                            block_size, num_blocks, max_blocks_per_seq, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prefix insert launch");
+  return TACO_OK;
+}
+
 taco_status taco_attn_check_device(void* stream, uint32_t* bits_out) {
   if (bits_out) *bits_out = 0;
   int dev = 0;
@@ -489,13 +543,14 @@ taco_status taco_attn_check_device(void* stream, uint32_t* bits_out) {
   if (bits == 0) return TACO_OK;
   cudaMemset(w.error_word, 0, 4);
   if (bits & TACO_DEVERR_WAIT_TIMEOUT) cudaMemset(w.counters, 0, w.counters_cap * 4);
-  return fail(TACO_ERR_DEVICE_CHECK, "device range check failed: bits 0x%x%s%s%s%s%s%s", bits,
+  return fail(TACO_ERR_DEVICE_CHECK, "device range check failed: bits 0x%x%s%s%s%s%s%s%s", bits,
               (bits & TACO_DEVERR_BLOCK_ID) ? " [block id out of range]" : "",
               (bits & TACO_DEVERR_CONTEXT_LEN) ? " [context length out of range]" : "",
               (bits & TACO_DEVERR_NUM_CAND) ? " [candidate count out of range]" : "",
               (bits & TACO_DEVERR_SLOT) ? " [slot out of range]" : "",
               (bits & TACO_DEVERR_WAIT_TIMEOUT) ? " [pipeline wait timed out]" : "",
-              (bits & TACO_DEVERR_PARENT) ? " [parent index out of range]" : "");
+              (bits & TACO_DEVERR_PARENT) ? " [parent index out of range]" : "",
+              (bits & TACO_DEVERR_TABLE_FULL) ? " [prefix table full]" : "");
 }
 
 void taco_attn_release_workspace(void) {

@@ -51,6 +51,8 @@ cudaError_t launch_accept(const AcceptArgs& a, cudaStream_t stream);
 
 // Rows of packed queries one unit of the mma.sync verify kernel covers for a given G * C.
 int mma_rows_per_unit(int packed_rows);
+// Resident CTAs per SM the mma.sync verify kernel is built for (the default grid is this times the SMs).
+int mma_ctas_per_sm(int rows_per_unit);
 // Dynamic shared memory the mma.sync verify kernel needs.
 int mma_smem_bytes(int D, int rows_per_unit, bool kv8 = false);
 // keys per work tile of the mma.sync kernel for this unit height (e4m3 caches: 128 for <= 32 rows)
@@ -60,6 +62,12 @@ cudaError_t launch_verify_mma(const CUtensorMap& tk, const CUtensorMap& tv, cons
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 // Quantising append into an e4m3 cache: code = e4m3(x / scale[h]) (round to nearest even, saturating).
 cudaError_t launch_append_e4m3(const AppendArgs& a, const float* k_scale, const float* v_scale, cudaStream_t stream);
+// Prefix-tree lookup (insert = false) or insert of B sequences' full blocks.
+cudaError_t launch_prefix_cache(bool insert, const int32_t* tokens, const int32_t* seq_starts, const int32_t* block_tables,
+                                uint64_t* slot_keys, int32_t* slot_nodes, int64_t capacity, int32_t* node_parent,
+                                int32_t* node_depth, int32_t* node_tokens, int32_t* out_blocks, int32_t* out_count,
+                                uint32_t* error_word, int B, int bs, int num_blocks, int max_blocks,
+                                cudaStream_t stream);
 // Keys per work tile of the tcgen05 verify kernel.
 int tc_tile_keys();
 // Dynamic shared memory of the tcgen05 verify kernel.

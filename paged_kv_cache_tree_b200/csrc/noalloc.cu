@@ -125,10 +125,10 @@ extern "C" taco_status paged_tree_attention_noalloc(
     sms = g_sm_count[dev];
   }
 
-  // grid: two CTAs per SM, fewer if the partials (2 slots per CTA) would not fit in the scratch
+  // grid: the kernel's resident CTAs per SM, fewer if the partials (2 slots per CTA) would not fit
   const size_t slot_bytes = static_cast<size_t>(rows) * (head_dim + 1) * 4 + 512;
   const int max_grid = static_cast<int>(kPartialBytes / slot_bytes / 2);
-  int grid = 2 * sms;
+  int grid = taco::mma_ctas_per_sm(rows) * sms;
   if (grid > max_grid) grid = max_grid;
   if (grid < 1) return fail(TACO_ERR_UNSUPPORTED, "scratch too small for one CTA");
   const size_t slots = 2 * static_cast<size_t>(grid);

@@ -4,6 +4,8 @@
 
 namespace taco {
 
+int mma_ctas_per_sm(int rows_per_unit) { return rows_per_unit == 8 ? MmaCfg<128, 0>::kCtasPerSm : MmaCfg<128, 1>::kCtasPerSm; }
+
 int mma_rows_per_unit(int packed_rows) {
   if (packed_rows <= 8) return 8;     // swapped form
   if (packed_rows <= 16) return 16;

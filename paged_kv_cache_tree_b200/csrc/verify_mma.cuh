@@ -39,7 +39,10 @@ struct MmaCfg {
   static constexpr int kPanelBytes = kTile * 128;
   static constexpr int kTensorBytes = kPanels * kPanelBytes;  // one of K or V per stage
   static constexpr int kStageBytes = 2 * kTensorBytes;
-  static constexpr int kStages = (kPanels * kPanelBytes >= 16384) ? 3 : 6;  // 96 KB of stages
+  // two CTAs per SM with 96 KB of stages each (three CTAs with 64 KB each and threads capped at 112
+  // registers measured slower for the swapped form: the cap spills inside the tile loop)
+  static constexpr int kCtasPerSm = 2;
+  static constexpr int kStages = 98304 / kStageBytes;
   static constexpr int kScratchFloats = 16 * D + 64;          // cross-warp O and l
   static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes +
                                     kScratchFloats * 4 + 64 * 4 /*m publish*/ +
@@ -88,7 +91,7 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 }
 
 template <typename T, int D, int MT, bool KV8>
-__global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, 2)
+__global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasPerSm)
     verify_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const VerifyParams p) {
   using Cfg = MmaCfg<D, MT, KV8>;

@@ -28,10 +28,14 @@ paged KV-append); otherwise those slots are poisoned too and an append must fill
 8-bit (e4m3) caches for a workload come from ``make_e4m3_cache``: byte patterns drawn directly (random
 sign and mantissa, exponent field mostly in 9..14, sometimes anywhere in 0..14), the NaN code where the
 16-bit caches hold NaN, and per-KV-head scales uniform on [0.004, 0.012]; no quantisation happens here.
+
+Token streams for the prefix-tree lookup come from ``make_prefix_inputs`` (its docstring gives the
+recipe); they hold token ids only, no hashing or matching.
 """
 from __future__ import annotations
 
 import dataclasses
+import itertools
 import math
 from typing import Optional, Sequence, Union
 
@@ -340,6 +344,80 @@ def kv8_append_bytes(w: Workload) -> int:
     """Quantising append: 16-bit rows read, e4m3 codes written, for K and V."""
     rows = int(w.num_candidates.long().sum())
     return 2 * rows * w.Hkv * w.D * (2 + 1)
+
+
+@dataclasses.dataclass
+class PrefixInputs:
+    """Host tensors for the prefix-tree lookup: sequences whose KV blocks are cached (to insert) and the
+    prompts of new requests (to look up)."""
+
+    bs: int
+    num_blocks: int
+    max_blocks: int
+    cached_tokens: torch.Tensor   # int32 [total]
+    cached_starts: torch.Tensor   # int32 [S + 1]
+    cached_tables: torch.Tensor   # int32 [S, max_blocks]: distinct physical blocks, -1 padded
+    prompts: torch.Tensor         # int32 [total]
+    prompt_starts: torch.Tensor   # int32 [B + 1]
+
+    def seqs(self, which: str) -> list:
+        toks = (self.cached_tokens if which == "cached" else self.prompts).tolist()
+        st = (self.cached_starts if which == "cached" else self.prompt_starts).tolist()
+        return [toks[st[i]:st[i + 1]] for i in range(len(st) - 1)]
+
+    def prompt_tokens(self) -> int:
+        return int(self.prompts.numel())
+
+    def to(self, device) -> "PrefixInputs":
+        out = dataclasses.replace(self)
+        for f in dataclasses.fields(self):
+            v = getattr(self, f.name)
+            if isinstance(v, torch.Tensor):
+                setattr(out, f.name, v.to(device))
+        return out
+
+
+def make_prefix_inputs(*, n_cached: int = 256, n_prompts: int = 64, bs: int = 16, n_stems: int = 8,
+                       stem_len=(256, 2048), tail_len=(0, 4096), prompt_tail=(0, 2048), vocab: int = 128256,
+                       seed: int = 2024) -> PrefixInputs:
+    """Seeded token streams shaped like a serving cache: a few shared stems (system prompts); each
+    cached sequence extends a stem or, half the time, a random-length prefix of an earlier cached
+    sequence (so the cache forms a branching tree) with a random tail; each prompt is a random-length
+    prefix of a cached sequence plus a divergent random tail (one in ten is wholly new). Tokens are
+    uniform over the vocabulary; cached sequence i takes the next ceil(len/bs) entries of a random
+    permutation of the block pool as its block table."""
+    g = torch.Generator().manual_seed(int(seed))
+    rint = lambda lo, hi: int(torch.randint(int(lo), int(hi) + 1, (1,), generator=g))
+    rand_toks = lambda n: torch.randint(0, vocab, (n,), generator=g, dtype=torch.int32)
+    stems = [rand_toks(rint(*stem_len)) for _ in range(n_stems)]
+    cached = []
+    for i in range(n_cached):
+        if i > 0 and rint(0, 1) == 1:
+            src = cached[rint(0, i - 1)]
+            base = src[: rint(0, src.numel())]
+        else:
+            base = stems[rint(0, n_stems - 1)]
+        cached.append(torch.cat([base, rand_toks(rint(*tail_len))]))
+    prompts = []
+    for _ in range(n_prompts):
+        if rint(0, 9) == 0:
+            prompts.append(rand_toks(rint(1, prompt_tail[1] + stem_len[1])))
+        else:
+            src = cached[rint(0, n_cached - 1)]
+            prompts.append(torch.cat([src[: rint(0, src.numel())], rand_toks(rint(*prompt_tail))]))
+    nblk = [(c.numel() + bs - 1) // bs for c in cached]
+    max_blocks = max([1] + nblk + [(p.numel() + bs - 1) // bs for p in prompts])
+    NB = max(1, math.ceil(1.1 * sum(nblk)))
+    perm = torch.randperm(NB, generator=g).to(torch.int32)
+    tables = torch.full((n_cached, max_blocks), -1, dtype=torch.int32)
+    off = 0
+    for i, k in enumerate(nblk):
+        tables[i, :k] = perm[off:off + k]
+        off += k
+    starts = lambda seqs: torch.tensor([0] + list(itertools.accumulate(int(x.numel()) for x in seqs)), dtype=torch.int32)
+    return PrefixInputs(bs=bs, num_blocks=NB, max_blocks=max_blocks, cached_tokens=torch.cat(cached),
+                        cached_starts=starts(cached), cached_tables=tables, prompts=torch.cat(prompts),
+                        prompt_starts=starts(prompts))
 
 
 @dataclasses.dataclass

@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.taco_attn_version() == 3
+    assert lib.taco_attn_version() == 4
 
 
 def _attn_args(**over):
@@ -166,3 +166,43 @@ def test_e4m3_append_rejects_bad_arguments_on_host(lib, over, status):
             a["Hkv"], a["D"], a["bs"], a["NB"], a["maxblk"], a["stream"]]
     assert lib.paged_kv_append_e4m3(*args) == status
     assert lib.taco_attn_last_error().decode()
+
+
+def _prefix_args(insert, **over):
+    a = dict(tok=16, st=16, bt=16, keys=16, nodes=16, cap=1024, par=16, dep=16, ntok=16, out=16, cnt=16, B=2,
+             bs=16, NB=40, maxblk=8, stream=None)
+    a.update(over)
+    head = [a["tok"], a["st"]] + ([a["bt"]] if insert else [])
+    return head + [a["keys"], a["nodes"], ctypes.c_int64(a["cap"]), a["par"], a["dep"], a["ntok"], a["out"], a["cnt"],
+                   a["B"], a["bs"], a["NB"], a["maxblk"], a["stream"]]
+
+
+@pytest.mark.parametrize("insert", [False, True])
+@pytest.mark.parametrize("over,status", [
+    (dict(tok=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(keys=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(ntok=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(keys=12), _lib.TACO_ERR_INVALID_ARG),     # not 8-byte aligned
+    (dict(cap=1000), _lib.TACO_ERR_INVALID_ARG),    # not a power of two
+    (dict(cap=1), _lib.TACO_ERR_INVALID_ARG),
+    (dict(bs=0), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(bs=2048), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(B=-1), _lib.TACO_ERR_INVALID_ARG),
+    (dict(NB=0), _lib.TACO_ERR_INVALID_ARG),
+    (dict(maxblk=0), _lib.TACO_ERR_INVALID_ARG),
+])
+def test_prefix_calls_reject_bad_arguments_on_host(lib, insert, over, status):
+    fn = lib.prefix_cache_insert if insert else lib.prefix_cache_lookup
+    assert fn(*_prefix_args(insert, **over)) == status
+    assert lib.taco_attn_last_error().decode()
+
+
+def test_prefix_lookup_needs_out_matched_and_insert_needs_tables(lib):
+    assert lib.prefix_cache_lookup(*_prefix_args(False, cnt=None)) == _lib.TACO_ERR_INVALID_ARG
+    assert lib.prefix_cache_insert(*_prefix_args(True, bt=None)) == _lib.TACO_ERR_INVALID_ARG
+    assert lib.prefix_cache_insert(*_prefix_args(True, cnt=None, B=0)) == _lib.TACO_OK   # out_inserted optional
+
+
+def test_prefix_calls_with_empty_batch_are_no_ops(lib):
+    assert lib.prefix_cache_lookup(*_prefix_args(False, B=0)) == _lib.TACO_OK
+    assert lib.prefix_cache_insert(*_prefix_args(True, B=0)) == _lib.TACO_OK
