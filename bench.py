@@ -340,6 +340,51 @@ def measure_kv8(taco, w, d, dev, stream, args):
     }
 
 
+def measure_prefix(taco, dev, stream, args):
+    """Prefix-tree KV lookup for prefill, timed on its own: 256 cached sequences (about 0.9 M tokens,
+    34 k distinct full blocks of 16 tokens) inserted in one call into a fresh table, then 64 prompts
+    (about 176 k tokens, each a prefix of a cached sequence plus a divergent tail) looked up in one
+    call. The table and node arrays (about 6 MB) stay in L2, so the lookup is latency-bound (one warp
+    walks each prompt's blocks); no L2 flush. Launches timed with CUDA events on their stream."""
+    pi = wl.make_prefix_inputs()
+    d = pi.to(dev)
+    cap = 1 << max(2, (2 * pi.num_blocks - 1).bit_length())
+    steps = max(10, min(args.steps, 200))
+    t_ins = []
+    for it in range(3):
+        cache = taco.PrefixCache(pi.num_blocks, pi.bs, cap, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.insert(d.cached_tokens, d.cached_starts, d.cached_tables, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        t_ins.append(e0.elapsed_time(e1))
+    out_b = torch.empty((d.prompt_starts.numel() - 1, pi.max_blocks), dtype=torch.int32, device=dev)
+    out_m = torch.empty((d.prompt_starts.numel() - 1,), dtype=torch.int32, device=dev)
+    t_lk = []
+    for it in range(args.warmup + steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.lookup(d.prompts, d.prompt_starts, pi.max_blocks, out_blocks=out_b, out_matched=out_m, stream=stream)
+        e1.record(stream)
+        if it >= args.warmup:
+            t_lk.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    taco.check_device(stream)
+    lk_ms = statistics.median(a.elapsed_time(b) for a, b in t_lk)
+    matched = int(out_m.sum().item())
+    n_prompts = d.prompt_starts.numel() - 1
+    return {
+        "cached_sequences": int(d.cached_starts.numel() - 1), "cached_tokens": int(pi.cached_tokens.numel()),
+        "prompts": n_prompts, "prompt_tokens": pi.prompt_tokens(), "block_size": pi.bs,
+        "matched_blocks": matched, "matched_token_frac": matched * pi.bs / max(1, pi.prompt_tokens()),
+        "lookup_us": 1e3 * lk_ms, "prompts_per_s": n_prompts / (lk_ms * 1e-3),
+        "prompt_tokens_per_s": pi.prompt_tokens() / (lk_ms * 1e-3),
+        "insert_one_call_us": 1e3 * statistics.median(t_ins), "table_slots": cap,
+        "bound": "latency (table and nodes L2-resident; a warp's probes depend on its scan)",
+    }
+
+
 def run_ours(args, world, rank, local):
     import paged_kv_cache_tree_b200 as taco
 
@@ -443,6 +488,7 @@ def run_ours(args, world, rank, local):
 
     accept = measure_accept(taco, w, d, dev, stream, args)
     kv8 = measure_kv8(taco, w, d, dev, stream, args)
+    prefix = measure_prefix(taco, dev, stream, args)
 
     if rank != 0:
         return None
@@ -471,6 +517,7 @@ def run_ours(args, world, rank, local):
         "clocks": clocks,
         "accept": accept,
         "kv8": kv8,
+        "prefix_cache": prefix,
     }
     if kv8 is not None:
         kv8["attention_frac"] = kv8["attention_GBps"] / peak

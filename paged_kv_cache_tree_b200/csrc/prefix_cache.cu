@@ -101,7 +101,7 @@ struct PrefixArgs {
 __device__ __forceinline__ int full_blocks(const PrefixArgs& a, int b, int lane, int64_t& s0) {
   s0 = __ldg(a.seq_starts + b);
   const int64_t n = static_cast<int64_t>(__ldg(a.seq_starts + b + 1)) - s0;
-  if (n < 0) {
+  if (n < 0 || s0 < 0) {
     if (lane == 0) atomicOr(a.error_word, TACO_DEVERR_CONTEXT_LEN);
     return 0;
   }
