@@ -46,17 +46,16 @@ __device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
-// Keys of full blocks c0 + lane (lane < count) of one sequence, given the prefix hash `carry` of the
-// blocks before c0. Prefix hash of blocks 0..j: H_j = H_(j-1) * base^bs + h_j, h_j the block's own
-// polynomial hash; the recurrence is a scan with (a, q) o (b, r) = (a * r + b, q * r). Returns the key
-// (0 for lanes past count) and updates carry to H of the chunk's last block.
-__device__ __forceinline__ uint64_t chunk_keys(const int32_t* seq, int c0, int count, int bs, uint64_t base_bs,
-                                               uint64_t& carry, int lane) {
-  const int j = c0 + lane;
-  const bool active = lane < count;
-  uint64_t a = 0, q = 1;
-  if (active) {
-    const int32_t* t = seq + static_cast<int64_t>(j) * bs;
+// Per-block hashes of full blocks c0 + lane (lane < count) of one sequence and their inclusive scan
+// with a zero carry. Prefix hash of blocks 0..j: H_j = H_(j-1) * base^bs + h_j, h_j the block's own
+// polynomial hash; the recurrence is a scan with (a, q) o (b, r) = (a * r + b, q * r). On return a
+// lane holds a = H of blocks c0..j alone and q = base^(bs * (j - c0 + 1)); H_j = carry * q + a.
+__device__ __forceinline__ void chunk_scan(const int32_t* seq, int c0, int count, int bs, uint64_t base_bs, int lane,
+                                           uint64_t& a, uint64_t& q) {
+  a = 0;
+  q = 1;
+  if (lane < count) {
+    const int32_t* t = seq + static_cast<int64_t>(c0 + lane) * bs;
     for (int i = 0; i < bs; ++i) a = a * kHashBase + (static_cast<uint64_t>(static_cast<uint32_t>(__ldg(t + i))) + 1ull);
     q = base_bs;
   }
@@ -69,17 +68,42 @@ __device__ __forceinline__ uint64_t chunk_keys(const int32_t* seq, int c0, int c
       q = q2 * q;
     }
   }
-  const uint64_t H = carry * q + a;   // q = base_bs^(lane + 1) on active lanes
-  carry = shfl_u64(H, count - 1);
-  return active ? (fmix64(H + static_cast<uint64_t>(j + 1) * kDepthSalt) | 1ull) : 0ull;
 }
 
-__device__ __forceinline__ bool block_tokens_equal(const int32_t* a, const int32_t* node_tok, int bs, bool coherent) {
-  for (int i = 0; i < bs; ++i) {
-    const int32_t x = coherent ? __ldcg(node_tok + i) : __ldg(node_tok + i);
-    if (__ldg(a + i) != x) return false;
+__device__ __forceinline__ uint64_t block_key(uint64_t H, int j) {
+  return fmix64(H + static_cast<uint64_t>(j + 1) * kDepthSalt) | 1ull;
+}
+
+// Keys of full blocks c0 + lane (lane < count) given the prefix hash `carry` of the blocks before c0;
+// updates carry to H of the chunk's last block. Lanes past count get 0.
+__device__ __forceinline__ uint64_t chunk_keys(const int32_t* seq, int c0, int count, int bs, uint64_t base_bs,
+                                               uint64_t& carry, int lane) {
+  uint64_t a, q;
+  chunk_scan(seq, c0, count, bs, base_bs, lane, a, q);
+  const uint64_t H = carry * q + a;
+  carry = shfl_u64(H, count - 1);
+  return lane < count ? block_key(H, c0 + lane) : 0ull;
+}
+
+// Token-by-token equality of a block, loads issued eight at a time (one dependent round trip per
+// eight tokens rather than per token).
+__device__ __forceinline__ bool block_tokens_equal(const int32_t* a, const int32_t* node_tok, int bs) {
+  int i = 0;
+  for (; i + 8 <= bs; i += 8) {
+    int32_t x[8], y[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      x[k] = __ldg(a + i + k);
+      y[k] = __ldg(node_tok + i + k);
+    }
+    bool eq = true;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) eq &= x[k] == y[k];
+    if (!eq) return false;
   }
-  return true;
+  bool eq = true;
+  for (; i < bs; ++i) eq &= __ldg(a + i) == __ldg(node_tok + i);
+  return eq;
 }
 
 struct PrefixArgs {
@@ -116,91 +140,131 @@ __device__ __forceinline__ uint64_t base_pow_bs(int bs) {
 }
 
 // --------------------------------------------------------------------------------------------- lookup
-// One warp per prompt. Chunk by chunk of 32 blocks: keys by scan, every lane probes its block's slot
-// chain to the first empty slot and keeps the first node whose depth and tokens match (and notes
-// whether a second one exists); then the parent links decide the matched run. A block with two
-// candidates (a full 64-bit collision of two prefixes ending in the same tokens) is resolved in order
-// with its known parent.
-__global__ void __launch_bounds__(256) prefix_lookup_kernel(PrefixArgs a) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= a.B) return;
-  const int b = warp;
+constexpr int kLookupWarps = 8;
+
+// Slot of the node for block j with key `key`, depth j, the given tokens and (if want_parent > -2) the
+// given parent: the first such node on the key's probe chain, or -1. `second` reports whether another
+// node with equal key, depth and tokens follows it on the chain (only when want_parent == -2).
+__device__ __forceinline__ int probe_node(const PrefixArgs& a, uint64_t key, int j, const int32_t* tok, int want_parent,
+                                          bool& second) {
+  const uint64_t mask = static_cast<uint64_t>(a.cap) - 1;
+  uint64_t slot = key & mask;
+  int node = -1;
+  second = false;
+  for (int64_t it = 0; it < a.cap; ++it) {
+    const uint64_t k = __ldg(a.slot_keys + slot);
+    if (k == 0ull) break;
+    if (k == key) {
+      const int nd = __ldg(a.slot_nodes + slot);
+      if (nd >= 0 && nd < a.num_blocks && __ldg(a.node_depth + nd) == j &&
+          (want_parent == -2 || __ldg(a.node_parent + nd) == want_parent) &&
+          block_tokens_equal(tok, a.node_tokens + static_cast<int64_t>(nd) * a.bs, a.bs)) {
+        if (node < 0) {
+          node = nd;
+          if (want_parent != -2) break;
+        } else {
+          second = true;
+          break;
+        }
+      }
+    }
+    slot = (slot + 1) & mask;
+  }
+  return node;
+}
+
+// One CTA of 8 warps per prompt, 256 blocks per round: each warp hashes and scans a chunk of 32 blocks,
+// the chunks' carries combine through shared memory, every block probes its chain in parallel, and
+// the parent links then decide the matched run (the first block whose node is missing or hangs from
+// another parent ends it). A block with two candidates (a full 64-bit collision of two prefixes ending
+// in the same tokens) is resolved in order by warp 0 with its known parent.
+__global__ void __launch_bounds__(kLookupWarps * 32) prefix_lookup_kernel(PrefixArgs a) {
+  constexpr int RB = kLookupWarps * 32;
+  __shared__ uint64_t sh_A[kLookupWarps], sh_Q[kLookupWarps];
+  __shared__ uint64_t sh_key[RB];
+  __shared__ int sh_node[RB];
+  __shared__ unsigned char sh_multi[RB];
+  __shared__ int sh_any_multi, sh_first_bad;
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int64_t s0;
-  const int nfull = full_blocks(a, b, lane, s0);
+  const int nfull = full_blocks(a, b, threadIdx.x, s0);
   const int32_t* seq = a.tokens + s0;
   const uint64_t base_bs = base_pow_bs(a.bs);
-  const uint64_t mask = static_cast<uint64_t>(a.cap) - 1;
   int32_t* out = a.out_blocks + static_cast<int64_t>(b) * a.max_blocks;
   uint64_t carry = 0;
   int prev_node = -1;
   int matched = nfull;
-  for (int c0 = 0; c0 < nfull; c0 += 32) {
-    const int count = nfull - c0 < 32 ? nfull - c0 : 32;
-    const uint64_t key = chunk_keys(seq, c0, count, a.bs, base_bs, carry, lane);
+  for (int r0 = 0; r0 < nfull; r0 += RB) {
+    const int rcount = nfull - r0 < RB ? nfull - r0 : RB;
+    int count = rcount - warp * 32;
+    count = count < 0 ? 0 : (count > 32 ? 32 : count);
+    const int c0 = r0 + warp * 32;
+    uint64_t av, qv;
+    chunk_scan(seq, c0, count, a.bs, base_bs, lane, av, qv);
+    // the chunk's own hash and multiplier (a zero-length chunk gives 0 and 1)
+    const uint64_t chunk_a = shfl_u64(av, count > 0 ? count - 1 : 0);
+    const uint64_t chunk_q = shfl_u64(qv, count > 0 ? count - 1 : 0);
+    if (lane == 0) {
+      sh_A[warp] = chunk_a;
+      sh_Q[warp] = chunk_q;
+    }
+    if (threadIdx.x == 0) {
+      sh_any_multi = 0;
+      sh_first_bad = rcount;
+    }
+    __syncthreads();
+    uint64_t cw = carry, next_carry = carry;
+#pragma unroll
+    for (int i = 0; i < kLookupWarps; ++i) {
+      if (i < warp) cw = cw * sh_Q[i] + sh_A[i];
+      next_carry = next_carry * sh_Q[i] + sh_A[i];
+    }
+    const int idx = warp * 32 + lane;
     const int j = c0 + lane;
+    const bool active = lane < count;
+    const uint64_t key = active ? block_key(cw * qv + av, j) : 0ull;
     int node = -1;
     bool multi = false;
-    if (lane < count) {
-      uint64_t slot = key & mask;
-      for (int64_t it = 0; it < a.cap; ++it) {
-        const uint64_t k = __ldg(a.slot_keys + slot);
-        if (k == 0ull) break;
-        if (k == key) {
-          const int nd = __ldg(a.slot_nodes + slot);
-          if (nd >= 0 && nd < a.num_blocks && __ldg(a.node_depth + nd) == j &&
-              block_tokens_equal(seq + static_cast<int64_t>(j) * a.bs, a.node_tokens + static_cast<int64_t>(nd) * a.bs,
-                                 a.bs, false)) {
-            if (node < 0) {
-              node = nd;
-            } else {
-              multi = true;
-              break;
+    if (active) node = probe_node(a, key, j, seq + static_cast<int64_t>(j) * a.bs, -2, multi);
+    sh_key[idx] = key;
+    sh_node[idx] = node;
+    sh_multi[idx] = multi ? 1 : 0;
+    if (multi) atomicOr(&sh_any_multi, 1);
+    __syncthreads();
+    if (sh_any_multi) {
+      if (warp == 0) {
+        for (int x = 0; x < rcount; ++x) {
+          if (sh_multi[x]) {
+            if (lane == 0) {
+              bool unused;
+              const int want = x == 0 ? prev_node : sh_node[x - 1];
+              sh_node[x] = probe_node(a, sh_key[x], r0 + x, seq + static_cast<int64_t>(r0 + x) * a.bs, want, unused);
             }
+            __syncwarp();
           }
         }
-        slot = (slot + 1) & mask;
       }
+      __syncthreads();
     }
-    // rare: resolve lanes with two candidates in order, each with its predecessor's node as parent
-    uint32_t pending = __ballot_sync(0xffffffffu, multi);
-    while (pending) {
-      const int l = __ffs(pending) - 1;
-      pending &= pending - 1;
-      const int want_parent = l == 0 ? prev_node : __shfl_sync(0xffffffffu, node, l - 1);
-      if (lane == l) {
-        node = -1;
-        uint64_t slot = key & mask;
-        for (int64_t it = 0; it < a.cap; ++it) {
-          const uint64_t k = __ldg(a.slot_keys + slot);
-          if (k == 0ull) break;
-          if (k == key) {
-            const int nd = __ldg(a.slot_nodes + slot);
-            if (nd >= 0 && nd < a.num_blocks && __ldg(a.node_depth + nd) == j && __ldg(a.node_parent + nd) == want_parent &&
-                block_tokens_equal(seq + static_cast<int64_t>(j) * a.bs,
-                                   a.node_tokens + static_cast<int64_t>(nd) * a.bs, a.bs, false)) {
-              node = nd;
-              break;
-            }
-          }
-          slot = (slot + 1) & mask;
-        }
-      }
+    if (active) {
+      const int nd = sh_node[idx];
+      const int expect = idx == 0 ? prev_node : sh_node[idx - 1];
+      if (!(nd >= 0 && __ldg(a.node_parent + nd) == expect)) atomicMin(&sh_first_bad, idx);
     }
-    int expect = __shfl_up_sync(0xffffffffu, node, 1);
-    if (lane == 0) expect = prev_node;
-    const bool ok = lane < count && node >= 0 && __ldg(a.node_parent + node) == expect;
-    const uint32_t bad = __ballot_sync(0xffffffffu, lane < count && !ok);
-    const int first_bad = bad ? __ffs(bad) - 1 : count;
-    if (lane < first_bad) out[j] = node;
-    if (bad) {
-      matched = c0 + first_bad;
+    __syncthreads();
+    const int fb = sh_first_bad;
+    if (active && idx < fb) out[j] = sh_node[idx];
+    if (fb < rcount) {
+      matched = r0 + fb;
       break;
     }
-    prev_node = __shfl_sync(0xffffffffu, node, count - 1);
+    prev_node = sh_node[rcount - 1];
+    carry = next_carry;
+    __syncthreads();
   }
-  for (int jj = matched + lane; jj < a.max_blocks; jj += 32) out[jj] = -1;
-  if (lane == 0) a.out_matched[b] = matched;
+  for (int jj = matched + static_cast<int>(threadIdx.x); jj < a.max_blocks; jj += blockDim.x) out[jj] = -1;
+  if (threadIdx.x == 0) a.out_matched[b] = matched;
 }
 
 // --------------------------------------------------------------------------------------------- insert
@@ -310,11 +374,10 @@ cudaError_t launch_prefix_cache(bool insert, const int32_t* tokens, const int32_
                                 cudaStream_t stream) {
   PrefixArgs a{tokens, seq_starts, block_tables, slot_keys, slot_nodes, node_parent, node_depth, node_tokens,
                out_blocks, out_count, error_word, capacity, B, bs, num_blocks, max_blocks};
-  const int blocks = (B * 32 + 255) / 256;
   if (insert)
-    prefix_insert_kernel<<<blocks, 256, 0, stream>>>(a);
+    prefix_insert_kernel<<<(B * 32 + 255) / 256, 256, 0, stream>>>(a);
   else
-    prefix_lookup_kernel<<<blocks, 256, 0, stream>>>(a);
+    prefix_lookup_kernel<<<B, kLookupWarps * 32, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
