@@ -1,5 +1,5 @@
-"""CPU oracle (test infrastructure only; see ``oracle.paged_attention``, ``oracle.tree_accept``, ``oracle.fp8``
-and ``oracle.prefix_cache``)."""
+"""CPU oracle (test infrastructure only; see ``oracle.paged_attention``, ``oracle.tree_accept``, ``oracle.fp8``,
+``oracle.prefix_cache`` and ``oracle.lookahead_cache``)."""
 from .paged_attention import (  # noqa: F401
     gather_sequence_kv,
     paged_kv_append,
@@ -12,3 +12,4 @@ from .paged_attention import (  # noqa: F401
 from . import tree_accept  # noqa: F401,E402
 from . import fp8  # noqa: F401,E402
 from . import prefix_cache  # noqa: F401,E402
+from . import lookahead_cache  # noqa: F401,E402
