@@ -385,6 +385,46 @@ def measure_prefix(taco, dev, stream, args):
     }
 
 
+def measure_lookahead(taco, dev, stream, args):
+    """Batched Lookahead Cache, timed on its own: candidate forests (C = 16, copy_len U[1, 8], contexts of
+    up to 4 tokens) for 64 sequences with 0.5-4 k-token phrase-structured histories against a 37 k-token
+    global cache; then the copy_len update. The histories and the cache (about 0.8 MB) stay in L2, and
+    each CTA's passes over them end in a sequential trie insertion, so the step is latency-bound. Launches
+    timed with CUDA events on their stream; no L2 flush."""
+    li = wl.make_lookahead_inputs()
+    d = li.to(dev)
+    steps = max(10, min(args.steps, 200))
+    t = []
+    for it in range(args.warmup + steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        tok, par, num = taco.lookahead_propose(d.history, d.hist_starts, d.global_tokens, d.copy_len, li.max_match,
+                                               li.C, stream=stream)
+        e1.record(stream)
+        if it >= args.warmup:
+            t.append((e0, e1))
+    hit = torch.full((d.copy_len.numel(),), 0.5, dtype=torch.float32, device=dev)
+    cl = d.copy_len.clone()
+    acc = torch.div(num, 2, rounding_mode="floor").to(torch.int32)
+    for _ in range(3):   # warm-up: the first launch of a kernel includes loading it
+        taco.lookahead_update_copy_len(acc, num, hit, cl, copy_max=8, stream=stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    taco.lookahead_update_copy_len(acc, num, hit, cl, copy_max=8, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    taco.check_device(stream)
+    ms = statistics.median(a.elapsed_time(b) for a, b in t)
+    B = li.copy_len.numel()
+    return {
+        "sequences": B, "history_tokens": int(li.history.numel()), "global_tokens": int(li.global_tokens.numel()),
+        "max_candidates": li.C, "max_match": li.max_match, "propose_us": 1e3 * ms,
+        "sequences_per_s": B / (ms * 1e-3), "candidates_proposed": int(num.sum().item()),
+        "copy_len_update_us": 1e3 * e0.elapsed_time(e1),
+        "bound": "latency (inputs L2-resident; per-sequence trie insertion is sequential)",
+    }
+
+
 def run_ours(args, world, rank, local):
     import paged_kv_cache_tree_b200 as taco
 
@@ -489,6 +529,7 @@ def run_ours(args, world, rank, local):
     accept = measure_accept(taco, w, d, dev, stream, args)
     kv8 = measure_kv8(taco, w, d, dev, stream, args)
     prefix = measure_prefix(taco, dev, stream, args)
+    lookahead = measure_lookahead(taco, dev, stream, args)
 
     if rank != 0:
         return None
@@ -518,6 +559,7 @@ def run_ours(args, world, rank, local):
         "accept": accept,
         "kv8": kv8,
         "prefix_cache": prefix,
+        "lookahead_cache": lookahead,
     }
     if kv8 is not None:
         kv8["attention_frac"] = kv8["attention_GBps"] / peak

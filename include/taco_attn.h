@@ -279,6 +279,44 @@ taco_status tree_greedy_accept(const int32_t* target_argmax, const int32_t* cand
  *   node that times out sets TACO_DEVERR_WAIT_TIMEOUT. A block id that is already a node must not be
  *   passed for a block whose prefix is new.
  */
+/*
+ * Batched Lookahead Cache (53ai.com workshop page, "整体方案分为两大部分", item 1 "基于批处理的 Lookahead
+ * Cache" and the paragraphs after it: candidates for a whole batch from a per-sequence local cache and a
+ * shared global cache, queried by match length, a copied length adapted to batch size and hit rate, and
+ * a forest of branches).
+ *
+ * lookahead_propose: a candidate forest per sequence, ready for tree_mask_from_parents and the verify.
+ *   history        int32 [total]; sequence b's tokens (prompt plus generated) are
+ *                  history[hist_starts[b] .. hist_starts[b+1]), token ids >= 0 (the local cache)
+ *   hist_starts    int32 [batch + 1], non-decreasing (a decreasing pair sets TACO_DEVERR_CONTEXT_LEN
+ *                  and counts as empty)
+ *   global_tokens  int32 [global_len] shared by the batch (the global cache); values < 0 separate
+ *                  passages and never match. May be NULL when global_len is 0.
+ *   copy_len       int32 [batch]: at most this many tokens are copied per branch (<= 0: no candidates)
+ *   max_match      longest context matched, 1..16
+ *   Per cache: the longest m <= min(max_match, len_b) such that the sequence's last m tokens occur in
+ *   the cache ending at a position e with a following token (local: an earlier occurrence); the
+ *   occurrences of that m, most recent (largest e) first, each give the following tokens (at most
+ *   copy_len, stopping before a separator or the end) as a path. Local paths, then global ones, merge
+ *   into a trie of at most max_candidates (<= 32) nodes numbered in creation order (a parent precedes
+ *   its children); merging stops when the trie is full.
+ *   tokens_out, parents_out  int32 [batch, max_candidates]: node token and parent (-1 = root); -1 past
+ *                  the node count. num_candidates_out int32 [batch].
+ *
+ * lookahead_update_copy_len: after a verify step, per sequence
+ *   hit[b] <- (1 - alpha) * hit[b] + alpha * accept_len[b] / max(1, num_proposed[b])
+ *   copy_len[b] = clamp(floor(copy_max * hit[b] * min(1, batch_ref / batch) + 0.5), 1, copy_max)
+ *   each operation rounded to float32 in this order. hit float32 [batch] is updated in place.
+ */
+taco_status lookahead_propose(const int32_t* history, const int32_t* hist_starts, const int32_t* global_tokens,
+                              int64_t global_len, const int32_t* copy_len, int32_t max_match, int32_t batch,
+                              int32_t max_candidates, int32_t* tokens_out, int32_t* parents_out,
+                              int32_t* num_candidates_out, void* stream);
+
+taco_status lookahead_update_copy_len(const int32_t* accept_len, const int32_t* num_proposed, float* hit,
+                                      int32_t* copy_len, int32_t batch, int32_t copy_max, float alpha,
+                                      int32_t batch_ref, void* stream);
+
 taco_status prefix_cache_lookup(const int32_t* tokens, const int32_t* seq_starts, const uint64_t* slot_keys,
                                 const int32_t* slot_nodes, int64_t capacity, const int32_t* node_parent,
                                 const int32_t* node_depth, const int32_t* node_tokens, int32_t* out_blocks,

@@ -11,6 +11,8 @@ from ._lib import (  # noqa: F401
     check_device,
     load,
     logits_argmax,
+    lookahead_propose,
+    lookahead_update_copy_len,
     paged_kv_append,
     paged_kv_append_e4m3,
     paged_tree_attention,

@@ -44,6 +44,8 @@ EXPORTED = (
     "tree_greedy_accept",
     "prefix_cache_lookup",
     "prefix_cache_insert",
+    "lookahead_propose",
+    "lookahead_update_copy_len",
 )
 
 _lib = None
@@ -95,6 +97,10 @@ def load() -> ctypes.CDLL:
     lib.prefix_cache_lookup.restype = i32
     lib.prefix_cache_insert.argtypes = [vp] * 5 + [i64] + [vp] * 5 + [i32] * 4 + [vp]
     lib.prefix_cache_insert.restype = i32
+    lib.lookahead_propose.argtypes = [vp] * 3 + [i64, vp, i32, i32, i32] + [vp] * 3 + [vp]
+    lib.lookahead_propose.restype = i32
+    lib.lookahead_update_copy_len.argtypes = [vp] * 4 + [i32, i32, f32, i32, vp]
+    lib.lookahead_update_copy_len.restype = i32
     _lib = lib
     return lib
 
@@ -402,3 +408,42 @@ class PrefixCache:
             self.node_tokens.data_ptr(), out_blocks.data_ptr(), out_inserted.data_ptr(), B, self.block_size,
             self.num_blocks, max_blocks, _stream_handle(stream, tokens.device)))
         return out_blocks, out_inserted
+
+
+def lookahead_propose(history, hist_starts, global_tokens, copy_len, max_match: int, max_candidates: int,
+                      stream=None):
+    """Candidate forests (tokens [B, C], parents [B, C], num_candidates [B]) from each sequence's history
+    (int32 tokens, hist_starts [B + 1]) and a shared global token array (int32, may be empty)."""
+    _need_cuda("history", history, torch.int32, 1)
+    _need_cuda("hist_starts", hist_starts, torch.int32, 1)
+    _need_cuda("global_tokens", global_tokens, torch.int32, 1)
+    _need_cuda("copy_len", copy_len, torch.int32, 1)
+    B = hist_starts.shape[0] - 1
+    if B < 0 or copy_len.shape[0] != B:
+        raise ValueError("hist_starts must be [B + 1] and copy_len [B]")
+    if history.numel() == 0:
+        history = torch.zeros(1, dtype=torch.int32, device=history.device)
+    dev = history.device
+    tok = torch.empty((B, max_candidates), dtype=torch.int32, device=dev)
+    par = torch.empty((B, max_candidates), dtype=torch.int32, device=dev)
+    num = torch.empty((B,), dtype=torch.int32, device=dev)
+    g_ptr = global_tokens.data_ptr() if global_tokens.numel() > 0 else None
+    _check(load().lookahead_propose(history.data_ptr(), hist_starts.data_ptr(), g_ptr, global_tokens.numel(),
+                                    copy_len.data_ptr(), max_match, B, max_candidates, tok.data_ptr(), par.data_ptr(),
+                                    num.data_ptr(), _stream_handle(stream, dev)))
+    return tok, par, num
+
+
+def lookahead_update_copy_len(accept_len, num_proposed, hit, copy_len, copy_max: int, alpha: float = 0.5,
+                              batch_ref: int = 16, stream=None) -> None:
+    """Updates hit (float32 [B]) and copy_len (int32 [B]) in place from a verify step's accept lengths."""
+    _need_cuda("accept_len", accept_len, torch.int32, 1)
+    _need_cuda("num_proposed", num_proposed, torch.int32, 1)
+    _need_cuda("hit", hit, torch.float32, 1)
+    _need_cuda("copy_len", copy_len, torch.int32, 1)
+    B = accept_len.shape[0]
+    if num_proposed.shape[0] != B or hit.shape[0] != B or copy_len.shape[0] != B:
+        raise ValueError("all arrays must be [B]")
+    _check(load().lookahead_update_copy_len(accept_len.data_ptr(), num_proposed.data_ptr(), hit.data_ptr(),
+                                            copy_len.data_ptr(), B, copy_max, float(alpha), batch_ref,
+                                            _stream_handle(stream, accept_len.device)))

@@ -17,7 +17,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAbiVersion = 4;
+constexpr int kAbiVersion = 5;
 
 thread_local std::string g_last_error;
 
@@ -522,6 +522,43 @@ taco_status prefix_cache_insert(const int32_t* tokens, const int32_t* seq_starts
                                             node_parent, node_depth, node_tokens, out_blocks, out_inserted, err, batch,
                                             block_size, num_blocks, max_blocks_per_seq, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "prefix insert launch");
+  return TACO_OK;
+}
+
+taco_status lookahead_propose(const int32_t* history, const int32_t* hist_starts, const int32_t* global_tokens,
+                              int64_t global_len, const int32_t* copy_len, int32_t max_match, int32_t batch,
+                              int32_t max_candidates, int32_t* tokens_out, int32_t* parents_out,
+                              int32_t* num_candidates_out, void* stream) {
+  if (!history || !hist_starts || !copy_len || !tokens_out || !parents_out || !num_candidates_out)
+    return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (global_len < 0 || global_len > INT32_MAX) return fail(TACO_ERR_INVALID_ARG, "global_len must be in [0, 2^31)");
+  if (global_len > 0 && !global_tokens) return fail(TACO_ERR_INVALID_ARG, "null global_tokens with global_len > 0");
+  if (max_match < 1 || max_match > 16) return fail(TACO_ERR_UNSUPPORTED, "max_match must be in [1, 16]");
+  if (max_candidates < 1 || max_candidates > 32) return fail(TACO_ERR_UNSUPPORTED, "max_candidates must be in [1, 32]");
+  if (batch < 0) return fail(TACO_ERR_INVALID_ARG, "batch must be >= 0");
+  if (batch == 0) return TACO_OK;
+  uint32_t* err = nullptr;
+  taco_status st = device_error_word(&err);
+  if (st != TACO_OK) return st;
+  cudaError_t e = taco::launch_lookahead_propose(history, hist_starts, global_len > 0 ? global_tokens : nullptr,
+                                                 global_len, copy_len, max_match, batch, max_candidates, tokens_out,
+                                                 parents_out, num_candidates_out, err, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lookahead kernel launch");
+  return TACO_OK;
+}
+
+taco_status lookahead_update_copy_len(const int32_t* accept_len, const int32_t* num_proposed, float* hit,
+                                      int32_t* copy_len, int32_t batch, int32_t copy_max, float alpha,
+                                      int32_t batch_ref, void* stream) {
+  if (!accept_len || !num_proposed || !hit || !copy_len) return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (batch < 0) return fail(TACO_ERR_INVALID_ARG, "batch must be >= 0");
+  if (copy_max < 1) return fail(TACO_ERR_INVALID_ARG, "copy_max must be >= 1");
+  if (!(alpha >= 0.f && alpha <= 1.f)) return fail(TACO_ERR_INVALID_ARG, "alpha must be in [0, 1]");
+  if (batch_ref < 1) return fail(TACO_ERR_INVALID_ARG, "batch_ref must be >= 1");
+  if (batch == 0) return TACO_OK;
+  cudaError_t e = taco::launch_copy_len_update(accept_len, num_proposed, hit, copy_len, batch, copy_max, alpha,
+                                               batch_ref, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "copy_len kernel launch");
   return TACO_OK;
 }
 

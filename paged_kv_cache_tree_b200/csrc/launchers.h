@@ -68,6 +68,13 @@ cudaError_t launch_prefix_cache(bool insert, const int32_t* tokens, const int32_
                                 int32_t* node_depth, int32_t* node_tokens, int32_t* out_blocks, int32_t* out_count,
                                 uint32_t* error_word, int B, int bs, int num_blocks, int max_blocks,
                                 cudaStream_t stream);
+// Lookahead Cache candidate forests and the copy_len update.
+cudaError_t launch_lookahead_propose(const int32_t* history, const int32_t* hist_starts, const int32_t* global_tokens,
+                                     int64_t global_len, const int32_t* copy_len, int max_match, int B, int C,
+                                     int32_t* tokens_out, int32_t* parents_out, int32_t* num_out, uint32_t* error_word,
+                                     cudaStream_t stream);
+cudaError_t launch_copy_len_update(const int32_t* accept_len, const int32_t* proposed, float* hit, int32_t* copy_len,
+                                   int B, int copy_max, float alpha, int batch_ref, cudaStream_t stream);
 // Keys per work tile of the tcgen05 verify kernel.
 int tc_tile_keys();
 // Dynamic shared memory of the tcgen05 verify kernel.

@@ -30,7 +30,8 @@ sign and mantissa, exponent field mostly in 9..14, sometimes anywhere in 0..14),
 16-bit caches hold NaN, and per-KV-head scales uniform on [0.004, 0.012]; no quantisation happens here.
 
 Token streams for the prefix-tree lookup come from ``make_prefix_inputs`` (its docstring gives the
-recipe); they hold token ids only, no hashing or matching.
+recipe); they hold token ids only, no hashing or matching. Token streams for the Lookahead Cache come
+from ``make_lookahead_inputs`` (phrase-structured streams; its docstring gives the recipe).
 """
 from __future__ import annotations
 
@@ -418,6 +419,64 @@ def make_prefix_inputs(*, n_cached: int = 256, n_prompts: int = 64, bs: int = 16
     return PrefixInputs(bs=bs, num_blocks=NB, max_blocks=max_blocks, cached_tokens=torch.cat(cached),
                         cached_starts=starts(cached), cached_tables=tables, prompts=torch.cat(prompts),
                         prompt_starts=starts(prompts))
+
+
+@dataclasses.dataclass
+class LookaheadInputs:
+    """Host tensors for the Lookahead Cache: each sequence's token history, a shared global token array
+    (passages separated by -1) and per-sequence copy lengths."""
+
+    history: torch.Tensor       # int32 [total]
+    hist_starts: torch.Tensor   # int32 [B + 1]
+    global_tokens: torch.Tensor  # int32 [G]
+    copy_len: torch.Tensor      # int32 [B]
+    max_match: int
+    C: int
+
+    def histories(self) -> list:
+        h, st = self.history.tolist(), self.hist_starts.tolist()
+        return [h[st[i]:st[i + 1]] for i in range(len(st) - 1)]
+
+    def to(self, device) -> "LookaheadInputs":
+        out = dataclasses.replace(self)
+        for f in dataclasses.fields(self):
+            v = getattr(self, f.name)
+            if isinstance(v, torch.Tensor):
+                setattr(out, f.name, v.to(device))
+        return out
+
+
+def _phrase_stream(g: torch.Generator, n: int, bank: list, vocab: int, p_phrase: float) -> torch.Tensor:
+    parts, total = [], 0
+    while total < n:
+        if float(torch.rand(1, generator=g)) < p_phrase:
+            part = bank[int(torch.randint(0, len(bank), (1,), generator=g))]
+        else:
+            part = torch.randint(0, vocab, (int(torch.randint(1, 9, (1,), generator=g)),), generator=g, dtype=torch.int32)
+        parts.append(part)
+        total += part.numel()
+    return torch.cat(parts)[:n]
+
+
+def make_lookahead_inputs(*, B: int = 64, hist_len=(512, 4096), n_docs: int = 16, doc_len=(1024, 4096),
+                          n_phrases: int = 512, phrase_len=(2, 24), p_phrase: float = 0.8, vocab: int = 128256,
+                          copy_len=(1, 8), max_match: int = 4, C: int = 16, seed: int = 4242) -> LookaheadInputs:
+    """Seeded phrase-structured token streams (generated text repeats itself: the pages' premise). A bank
+    of random phrases is drawn first; every stream concatenates phrases from the bank (with probability
+    p_phrase) and short random runs. Sequence histories have lengths U[hist_len]; the global cache is
+    n_docs streams of U[doc_len] tokens separated by -1; copy lengths are uniform in copy_len."""
+    g = torch.Generator().manual_seed(int(seed))
+    rint = lambda lo, hi: int(torch.randint(int(lo), int(hi) + 1, (1,), generator=g))
+    bank = [torch.randint(0, vocab, (rint(*phrase_len),), generator=g, dtype=torch.int32) for _ in range(n_phrases)]
+    hists = [_phrase_stream(g, rint(*hist_len), bank, vocab, p_phrase) for _ in range(B)]
+    docs = []
+    for _ in range(n_docs):
+        docs += [_phrase_stream(g, rint(*doc_len), bank, vocab, p_phrase), torch.tensor([-1], dtype=torch.int32)]
+    glob = torch.cat(docs) if docs else torch.zeros(0, dtype=torch.int32)
+    cl = torch.randint(int(copy_len[0]), int(copy_len[1]) + 1, (B,), generator=g, dtype=torch.int32)
+    starts = torch.tensor([0] + list(itertools.accumulate(int(h.numel()) for h in hists)), dtype=torch.int32)
+    return LookaheadInputs(history=torch.cat(hists) if hists else torch.zeros(0, dtype=torch.int32),
+                           hist_starts=starts, global_tokens=glob, copy_len=cl, max_match=max_match, C=C)
 
 
 @dataclasses.dataclass

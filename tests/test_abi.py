@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.taco_attn_version() == 4
+    assert lib.taco_attn_version() == 5
 
 
 def _attn_args(**over):
@@ -206,3 +206,44 @@ def test_prefix_lookup_needs_out_matched_and_insert_needs_tables(lib):
 def test_prefix_calls_with_empty_batch_are_no_ops(lib):
     assert lib.prefix_cache_lookup(*_prefix_args(False, B=0)) == _lib.TACO_OK
     assert lib.prefix_cache_insert(*_prefix_args(True, B=0)) == _lib.TACO_OK
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(h=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(cl=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(g=None), _lib.TACO_ERR_INVALID_ARG),      # global_len > 0 needs tokens
+    (dict(glen=-1), _lib.TACO_ERR_INVALID_ARG),
+    (dict(M=0), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(M=17), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(C=33), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(C=0), _lib.TACO_ERR_UNSUPPORTED),
+    (dict(B=-1), _lib.TACO_ERR_INVALID_ARG),
+])
+def test_lookahead_propose_rejects_bad_arguments_on_host(lib, over, status):
+    a = dict(h=16, st=16, g=16, glen=100, cl=16, M=4, B=2, C=16, t=16, p=16, n=16, stream=None)
+    a.update(over)
+    args = [a["h"], a["st"], a["g"], ctypes.c_int64(a["glen"]), a["cl"], a["M"], a["B"], a["C"], a["t"], a["p"], a["n"],
+            a["stream"]]
+    assert lib.lookahead_propose(*args) == status
+    assert lib.taco_attn_last_error().decode()
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(acc=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(hit=None), _lib.TACO_ERR_INVALID_ARG),
+    (dict(cmax=0), _lib.TACO_ERR_INVALID_ARG),
+    (dict(alpha=1.5), _lib.TACO_ERR_INVALID_ARG),
+    (dict(alpha=float("nan")), _lib.TACO_ERR_INVALID_ARG),
+    (dict(bref=0), _lib.TACO_ERR_INVALID_ARG),
+    (dict(B=-3), _lib.TACO_ERR_INVALID_ARG),
+])
+def test_copy_len_update_rejects_bad_arguments_on_host(lib, over, status):
+    a = dict(acc=16, prop=16, hit=16, cl=16, B=4, cmax=8, alpha=0.5, bref=16, stream=None)
+    a.update(over)
+    args = [a["acc"], a["prop"], a["hit"], a["cl"], a["B"], a["cmax"], ctypes.c_float(a["alpha"]), a["bref"], a["stream"]]
+    assert lib.lookahead_update_copy_len(*args) == status
+
+
+def test_lookahead_calls_with_empty_batch_are_no_ops(lib):
+    assert lib.lookahead_propose(16, 16, None, ctypes.c_int64(0), 16, 4, 0, 16, 16, 16, 16, None) == _lib.TACO_OK
+    assert lib.lookahead_update_copy_len(16, 16, 16, 16, 0, 8, ctypes.c_float(0.5), 16, None) == _lib.TACO_OK
