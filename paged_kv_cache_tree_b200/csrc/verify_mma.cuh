@@ -3,7 +3,7 @@
 //
 // One CTA = 4 consumer warps + 2 producer warps, two CTAs per SM, persistent over a stream-K range of
 // key tiles (device_common.cuh). The producer warps walk the block table and stream each tile's
-// K chunks (first producer) and V chunks (second producer) (one chunk = min(bs, 64) consecutive
+// K chunks (first producer) and V chunks (second producer) (one chunk = min(bs, tile) consecutive
 // slots of one physical block and one KV head, contiguous in the [NB, Hkv, bs, D] cache) into a ring
 // of shared-memory stages with TMA, 128-byte swizzled so that ldmatrix reads are conflict-free. A
 // single warp can keep only so many TMA copies moving, so K and V are issued from separate warps;
@@ -11,7 +11,9 @@
 // (rows r = i * G + h' of candidate i and head g*G + h') and, when fewer than 4 row tiles exist,
 // split the tile's keys between them; S = Q K^T and O += P V run on mma.sync m16n8k16 with fp32
 // accumulators, and the softmax is the flash-style online form in base 2 (fp32 running max / sum).
-// The tree mask only enters the tiles that reach the candidates' positions.
+// The tree mask only enters the tiles that reach the candidates' positions. Units of at most 8 rows
+// use the swapped form (S^T = K Q^T, see MmaCfg), and e4m3 caches a variant that widens the codes to
+// f16 in registers (KV8).
 #pragma once
 
 #include "device_common.cuh"
