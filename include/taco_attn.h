@@ -112,6 +112,27 @@ taco_status paged_kv_append(const void* k_new, const void* v_new, const int32_t*
                             int32_t num_blocks, int32_t max_blocks_per_seq, void* stream);
 
 /*
+ * paged_tree_attention_append: paged_kv_append of the candidates followed by paged_tree_attention, in one
+ * call. Candidate i < n_b of sequence b goes to logical slot P_b + i (P_b = L_b - n_b; the layout
+ * paged_tree_attention assumes), so no slot array is needed; the caches are updated exactly as
+ * paged_kv_append would update them and `out` equals paged_tree_attention's result on the updated
+ * caches.
+ *   k_new, v_new  [B, C, Hkv, D] dtype, 16-byte aligned; rows i >= n_b are not read.
+ * Units of at most 16 packed query rows run the append inside the verify kernel: the CTA that loads the
+ * tile holding a candidate's key puts the new row into its shared-memory copy and into the cache, so no
+ * separate launch is needed. Other shapes launch the append kernel first on the same stream.
+ * Slot block ids outside [0, NB) are skipped and flagged (TACO_DEVERR_BLOCK_ID).
+ */
+taco_status paged_tree_attention_append(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                        void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                                        const int32_t* num_candidates, const uint32_t* tree_mask_bits,
+                                        float scale, void* out,
+                                        int32_t dtype, int32_t batch, int32_t max_candidates,
+                                        int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                        int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                        void* stream);
+
+/*
  * paged_tree_attention_noalloc: the same operation, arguments and results as paged_tree_attention,
  * for callers that cannot allocate device memory. The pages have no counterpart of this entry point;
  * it exists because paged_tree_attention grows a workspace with cudaMalloc on first use, which a

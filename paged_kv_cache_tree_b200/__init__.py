@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     paged_kv_append,
     paged_kv_append_e4m3,
     paged_tree_attention,
+    paged_tree_attention_append,
     paged_tree_attention_e4m3,
     paged_tree_attention_noalloc,
     release_workspace,

@@ -32,6 +32,7 @@ EXPORTED = (
     "paged_tree_attention",
     "paged_kv_append",
     "paged_tree_attention_noalloc",
+    "paged_tree_attention_append",
     "paged_tree_attention_e4m3",
     "paged_kv_append_e4m3",
     "taco_attn_last_error",
@@ -70,6 +71,8 @@ def load() -> ctypes.CDLL:
     lib.paged_tree_attention.restype = i32
     lib.paged_tree_attention_noalloc.argtypes = [vp] * 7 + [f32, vp] + [i32] * 9 + [vp]
     lib.paged_tree_attention_noalloc.restype = i32
+    lib.paged_tree_attention_append.argtypes = [vp] * 9 + [f32, vp] + [i32] * 9 + [vp]
+    lib.paged_tree_attention_append.restype = i32
     lib.paged_kv_append.argtypes = [vp] * 6 + [i32] * 8 + [vp]
     lib.paged_kv_append.restype = i32
     lib.paged_tree_attention_e4m3.argtypes = [vp] * 9 + [f32, vp] + [i32] * 9 + [vp]
@@ -176,6 +179,41 @@ def paged_tree_attention_noalloc(q, k_cache, v_cache, block_tables, context_lens
     scratch is a fixed array in the library; see include/taco_attn.h for its limits)."""
     return paged_tree_attention(q, k_cache, v_cache, block_tables, context_lens, num_candidates, tree_mask_bits,
                                 scale, out=out, stream=stream, _entry="paged_tree_attention_noalloc")
+
+
+def paged_tree_attention_append(q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, num_candidates,
+                                tree_mask_bits, scale: float, out: Optional[torch.Tensor] = None,
+                                stream=None) -> torch.Tensor:
+    """Append the candidates' K/V (k_new, v_new [B,C,Hkv,D]) at slots P_b + i, then attend; returns out."""
+    _need_cuda("k_new", k_new, q.dtype, 4)
+    _need_cuda("v_new", v_new, q.dtype, 4)
+    B, C, Hq, D = q.shape
+    if tuple(k_new.shape) != (B, C, k_cache.shape[1], D) or tuple(v_new.shape) != tuple(k_new.shape):
+        raise ValueError("k_new / v_new must be [B, C, Hkv, D]")
+    if out is None:
+        out = torch.empty_like(q)
+    # the shared checks of paged_tree_attention, then the fused entry point
+    _need_cuda("q", q, (torch.bfloat16, torch.float16), 4)
+    _need_cuda("k_cache", k_cache, q.dtype, 4)
+    _need_cuda("v_cache", v_cache, q.dtype, 4)
+    _need_cuda("block_tables", block_tables, torch.int32, 2)
+    _need_cuda("context_lens", context_lens, torch.int32, 1)
+    _need_cuda("num_candidates", num_candidates, torch.int32, 1)
+    _need_cuda("tree_mask_bits", tree_mask_bits, (torch.int32, torch.uint32), 2)
+    _need_cuda("out", out, q.dtype, 4)
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch")
+    if block_tables.shape[0] != B or context_lens.shape[0] != B or num_candidates.shape[0] != B:
+        raise ValueError("batch dimension mismatch")
+    if tuple(tree_mask_bits.shape) != (B, C):
+        raise ValueError("tree_mask_bits must be [B, C]")
+    _check(load().paged_tree_attention_append(
+        q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+        block_tables.data_ptr(), context_lens.data_ptr(), num_candidates.data_ptr(), tree_mask_bits.data_ptr(),
+        float(scale), out.data_ptr(), _dtype_code(q), B, C, Hq, Hkv, D, bs, NB, block_tables.shape[1],
+        _stream_handle(stream, q.device)))
+    return out
 
 
 def paged_kv_append(k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, stream=None) -> None:

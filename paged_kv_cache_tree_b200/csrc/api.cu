@@ -17,7 +17,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAbiVersion = 5;
+constexpr int kAbiVersion = 6;
 
 thread_local std::string g_last_error;
 
@@ -205,7 +205,8 @@ taco_status taco_attn_set_option(int32_t key, int64_t value) {
 
 // Both attention entry points; k_scale / v_scale non-null selects e4m3 caches.
 static taco_status attention_impl(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
-                                  const float* v_scale, const int32_t* block_tables, const int32_t* context_lens,
+                                  const float* v_scale, const void* k_new, const void* v_new,
+                                  const int32_t* block_tables, const int32_t* context_lens,
                                   const int32_t* num_candidates, const uint32_t* tree_mask_bits, float scale,
                                   void* out, int32_t dtype, int32_t batch, int32_t max_candidates,
                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
@@ -218,6 +219,8 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
     return fail(TACO_ERR_INVALID_ARG, "num_q_heads must be a positive multiple of num_kv_heads");
   if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !num_candidates || !tree_mask_bits || !out)
     return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
+  if (k_new && (!v_new || !aligned16(k_new) || !aligned16(v_new)))
+    return fail(TACO_ERR_INVALID_ARG, "k_new and v_new must be non-null and 16-byte aligned");
   if (kv8) {
     if (!v_scale) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (v_scale)");
     if (head_dim != 128) return fail(TACO_ERR_UNSUPPORTED, "e4m3 caches: head_dim must be 128");
@@ -311,6 +314,22 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
   p.tile_keys = tile;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
+  if (k_new) {
+    // fused append where the kernel supports it (mma.sync, <= 16 rows, 16-bit caches); otherwise the
+    // append kernel runs first on the same stream
+    if (!use_tc && rows <= 16 && !kv8) {
+      p.k_new = k_new;
+      p.v_new = v_new;
+      p.k_cache = const_cast<void*>(k_cache);
+      p.v_cache = const_cast<void*>(v_cache);
+    } else {
+      taco::AppendArgs a{k_new, v_new, block_tables, nullptr, const_cast<void*>(k_cache), const_cast<void*>(v_cache),
+                         w.error_word, batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks,
+                         max_blocks_per_seq, dtype, context_lens, num_candidates};
+      e = taco::launch_append(a, static_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+    }
+  }
 
   if (use_tc) {
     e = taco::launch_verify_tc(tk, tv, tq, p, dtype, grid, static_cast<cudaStream_t>(stream));
@@ -328,9 +347,22 @@ taco_status paged_tree_attention(const void* q, const void* k_cache, const void*
                                  void* out, int32_t dtype, int32_t batch, int32_t max_candidates,
                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                  int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
-  return attention_impl(q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens, num_candidates,
-                        tree_mask_bits, scale, out, dtype, batch, max_candidates, num_q_heads, num_kv_heads,
-                        head_dim, block_size, num_blocks, max_blocks_per_seq, stream);
+  return attention_impl(q, k_cache, v_cache, nullptr, nullptr, nullptr, nullptr, block_tables, context_lens,
+                        num_candidates, tree_mask_bits, scale, out, dtype, batch, max_candidates, num_q_heads,
+                        num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, stream);
+}
+
+taco_status paged_tree_attention_append(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                        void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                                        const int32_t* num_candidates, const uint32_t* tree_mask_bits, float scale,
+                                        void* out, int32_t dtype, int32_t batch, int32_t max_candidates,
+                                        int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                        int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                        void* stream) {
+  if (!k_new || !v_new) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (k_new / v_new)");
+  return attention_impl(q, k_cache, v_cache, nullptr, nullptr, k_new, v_new, block_tables, context_lens,
+                        num_candidates, tree_mask_bits, scale, out, dtype, batch, max_candidates, num_q_heads,
+                        num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, stream);
 }
 
 taco_status paged_tree_attention_e4m3(const void* q, const void* k_cache, const void* v_cache,
@@ -341,9 +373,9 @@ taco_status paged_tree_attention_e4m3(const void* q, const void* k_cache, const 
                                       int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                       int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
   if (!k_scale || !v_scale) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (k_scale / v_scale)");
-  return attention_impl(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_candidates,
-                        tree_mask_bits, scale, out, dtype, batch, max_candidates, num_q_heads, num_kv_heads,
-                        head_dim, block_size, num_blocks, max_blocks_per_seq, stream);
+  return attention_impl(q, k_cache, v_cache, k_scale, v_scale, nullptr, nullptr, block_tables, context_lens,
+                        num_candidates, tree_mask_bits, scale, out, dtype, batch, max_candidates, num_q_heads,
+                        num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, stream);
 }
 
 taco_status paged_kv_append(const void* k_new, const void* v_new, const int32_t* block_tables,

@@ -19,7 +19,14 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   const int h = static_cast<int>(row % a.Hkv);
   const int64_t bi = row / a.Hkv;                 // b * C + i
   const int b = static_cast<int>(bi / a.C);
-  const int s = __ldg(a.slot_offsets + bi);
+  int s;
+  if (a.slot_offsets != nullptr) {
+    s = __ldg(a.slot_offsets + bi);
+  } else {
+    const int i = static_cast<int>(bi % a.C);
+    const int n = __ldg(a.num_candidates + b), L = __ldg(a.context_lens + b);
+    s = (i < n && n <= L) ? L - n + i : -1;
+  }
   if (s < 0) return;
   if (s >= a.max_blocks * a.bs) {
     if (v == 0) atomicOr(a.error_word, TACO_DEVERR_SLOT);
@@ -69,7 +76,14 @@ __global__ void __launch_bounds__(256) append_e4m3_kernel(AppendArgs a, const fl
   const int h = static_cast<int>(row % a.Hkv);
   const int64_t bi = row / a.Hkv;
   const int b = static_cast<int>(bi / a.C);
-  const int s = __ldg(a.slot_offsets + bi);
+  int s;
+  if (a.slot_offsets != nullptr) {
+    s = __ldg(a.slot_offsets + bi);
+  } else {
+    const int i = static_cast<int>(bi % a.C);
+    const int n = __ldg(a.num_candidates + b), L = __ldg(a.context_lens + b);
+    s = (i < n && n <= L) ? L - n + i : -1;
+  }
   if (s < 0) return;
   if (s >= a.max_blocks * a.bs) {
     if (v == 0) atomicOr(a.error_word, TACO_DEVERR_SLOT);

@@ -37,6 +37,12 @@ struct VerifyParams {
   int tile_keys;         // keys per work tile of the kernel (64 or 128)
   const float* k_scale;  // e4m3 caches: per-KV-head scales (K value = code * k_scale[h]); else null
   const float* v_scale;
+  // fused append (16-bit caches, units of <= 16 rows): candidate i's new K/V rows [B, C, Hkv, D] go to
+  // logical slot P_b + i of these caches as the verify reads them; null = the caches are complete
+  const void* k_new;
+  const void* v_new;
+  void* k_cache;
+  void* v_cache;
 };
 
 // ---------------------------------------------------------------------------------------------

@@ -21,6 +21,9 @@ struct AppendArgs {
   uint32_t* error_word;
   int B, C, Hkv, D, bs, num_blocks, max_blocks;
   int dtype;  // of k_new / v_new (the quantising append converts them)
+  // with slot_offsets null: candidate i < n_b goes to logical slot L_b - n_b + i (the verify's layout)
+  const int32_t* context_lens;
+  const int32_t* num_candidates;
 };
 
 struct MaskArgs {

@@ -392,6 +392,39 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
         fence_proxy_async_smem();
         __syncwarp();
       }
+      if constexpr (!KV8 && MTS == 1) {
+        // fused append: the candidates' keys P .. L-1 that fall in this warp's key range were loaded
+        // from cache slots not yet written; put their new K/V rows into the stage (128-byte swizzle)
+        // and into the cache slots. One key group per warp and one row group per unit, so each
+        // candidate row has exactly one writer in the launch.
+        if (ready && p.k_new != nullptr && key0 + Cfg::kTile > P) {
+          const int p_lo = key0 + wkey0 > P ? key0 + wkey0 : P;
+          const int p_hi = key0 + wkey0 + KW < L ? key0 + wkey0 + KW : L;
+          constexpr int CH = D / 8;   // 16-byte chunks per row
+          uint8_t* kgen = stages + stage * Cfg::kStageBytes;
+          for (int idx = lane; idx < (p_hi - p_lo) * 2 * CH; idx += 32) {
+            const int pos = p_lo + idx / (2 * CH);
+            const int rem = idx % (2 * CH);
+            const bool is_v = rem >= CH;
+            const int c = rem % CH;
+            const int64_t src_row = (static_cast<int64_t>(b) * p.C + (pos - P)) * p.Hkv + g;
+            const uint4 val = __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(is_v ? p.v_new : p.k_new) +
+                                                                   src_row * D) + c);
+            const int r = pos - key0;
+            *reinterpret_cast<uint4*>(kgen + (is_v ? Cfg::kTensorBytes : 0) + (c / 8) * Cfg::kPanelBytes + r * 128 +
+                                      (((c % 8) ^ (r & 7)) << 4)) = val;
+            const int blk = __ldg(p.block_tables + static_cast<int64_t>(b) * p.max_blocks + pos / p.bs);
+            if (blk >= 0 && blk < p.num_blocks) {
+              T* cache = static_cast<T*>(is_v ? p.v_cache : p.k_cache);
+              reinterpret_cast<uint4*>(cache + ((static_cast<int64_t>(blk) * p.Hkv + g) * p.bs + pos % p.bs) * D)[c] = val;
+            } else if (c == 0 && !is_v) {
+              atomicOr(p.error_word, TACO_DEVERR_BLOCK_ID);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+      }
       if (ready) {
         if constexpr (SW) {
           // ---- swapped form. S^T = K Q^T: m tile m holds keys wkey0 + m*16 .. +15 (rows gq, gq+8 of the

@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.taco_attn_version() == 5
+    assert lib.taco_attn_version() == 6
 
 
 def _attn_args(**over):
@@ -247,3 +247,16 @@ def test_copy_len_update_rejects_bad_arguments_on_host(lib, over, status):
 def test_lookahead_calls_with_empty_batch_are_no_ops(lib):
     assert lib.lookahead_propose(16, 16, None, ctypes.c_int64(0), 16, 4, 0, 16, 16, 16, 16, None) == _lib.TACO_OK
     assert lib.lookahead_update_copy_len(16, 16, 16, 16, 0, 8, ctypes.c_float(0.5), 16, None) == _lib.TACO_OK
+
+
+def test_fused_append_attention_rejects_bad_arguments_on_host(lib):
+    def args(**over):
+        a = dict(kn=16, vn=16)
+        a.update({k: over.pop(k) for k in list(over) if k in a})
+        base = _attn_args(**over)
+        return [base[0], a["kn"], a["vn"]] + base[1:]
+    assert lib.paged_tree_attention_append(*args(kn=None)) == _lib.TACO_ERR_INVALID_ARG
+    assert lib.paged_tree_attention_append(*args(vn=None)) == _lib.TACO_ERR_INVALID_ARG
+    assert lib.paged_tree_attention_append(*args(kn=24)) == _lib.TACO_ERR_INVALID_ARG   # misaligned
+    assert lib.paged_tree_attention_append(*args(D=96)) == _lib.TACO_ERR_UNSUPPORTED
+    assert lib.paged_tree_attention_append(*args(B=0)) == _lib.TACO_OK
