@@ -141,3 +141,23 @@ def test_bad_parent_is_reported_not_faulted():
     with pytest.raises(taco.TacoError):
         taco.check_device()
     assert taco.check_device() == 0
+
+
+def test_argmax_signed_zeros_tie_and_maxima_anywhere_in_the_row():
+    """-0 and +0 are equal (the first wins); maxima planted across a full-vocabulary row, two per row
+    (the smaller index must win)."""
+    V = 128256
+    rows = 40
+    x = torch.full((rows, V), -1.0, dtype=torch.bfloat16)
+    x[0, :] = -0.0
+    x[0, 7] = 0.0
+    x[1, 5] = 0.0
+    x[1, 3] = -0.0
+    for r in range(2, rows):
+        x[r, (r * V) // (rows - 2) % V] = 2.0
+        x[r, ((r * 7919) % V)] = 2.0              # a second maximum: the smaller index must win
+    got = taco.logits_argmax(x.cuda()).cpu().numpy()
+    assert np.array_equal(got, oracle_argmax(x, "bf16"))
+    assert got[0] == 0 and got[1] == 3
+    # the scratch is left clean: the same call again gives the same answer
+    assert np.array_equal(taco.logits_argmax(x.cuda()).cpu().numpy(), got)
