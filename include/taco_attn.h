@@ -43,7 +43,7 @@ extern "C" {
 typedef int32_t taco_status;
 #define TACO_OK 0
 #define TACO_ERR_INVALID_ARG 1   /* null pointer, bad size, misaligned pointer */
-#define TACO_ERR_UNSUPPORTED 2   /* a size this build has no kernel for (D, bs, C) */
+#define TACO_ERR_UNSUPPORTED 2   /* a size the library has no kernel for (D, bs, C) */
 #define TACO_ERR_CUDA 3          /* a CUDA runtime call or launch failed */
 #define TACO_ERR_DEVICE_CHECK 4  /* taco_attn_check_device found a device-side range error */
 
