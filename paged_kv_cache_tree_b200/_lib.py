@@ -185,17 +185,16 @@ def paged_tree_attention_append(q, k_new, v_new, k_cache, v_cache, block_tables,
                                 tree_mask_bits, scale: float, out: Optional[torch.Tensor] = None,
                                 stream=None) -> torch.Tensor:
     """Append the candidates' K/V (k_new, v_new [B,C,Hkv,D]) at slots P_b + i, then attend; returns out."""
+    _need_cuda("q", q, (torch.bfloat16, torch.float16), 4)
     _need_cuda("k_new", k_new, q.dtype, 4)
     _need_cuda("v_new", v_new, q.dtype, 4)
+    _need_cuda("k_cache", k_cache, q.dtype, 4)
+    _need_cuda("v_cache", v_cache, q.dtype, 4)
     B, C, Hq, D = q.shape
     if tuple(k_new.shape) != (B, C, k_cache.shape[1], D) or tuple(v_new.shape) != tuple(k_new.shape):
         raise ValueError("k_new / v_new must be [B, C, Hkv, D]")
     if out is None:
         out = torch.empty_like(q)
-    # the shared checks of paged_tree_attention, then the fused entry point
-    _need_cuda("q", q, (torch.bfloat16, torch.float16), 4)
-    _need_cuda("k_cache", k_cache, q.dtype, 4)
-    _need_cuda("v_cache", v_cache, q.dtype, 4)
     _need_cuda("block_tables", block_tables, torch.int32, 2)
     _need_cuda("context_lens", context_lens, torch.int32, 1)
     _need_cuda("num_candidates", num_candidates, torch.int32, 1)
