@@ -305,10 +305,8 @@ __global__ void __launch_bounds__(256) prefix_insert_kernel(PrefixArgs a) {
     int found = -1;
     for (int64_t it = 0; it < a.cap && found < 0 && !stop; ++it) {
       uint64_t k = 0;
-      if (lane == 0) {
-        k = atomicAdd(reinterpret_cast<unsigned long long*>(a.slot_keys + slot), 0ull);
-        if (k == 0ull) k = atomicCAS(reinterpret_cast<unsigned long long*>(a.slot_keys + slot), 0ull, key);
-      }
+      // one compare-and-swap both reads the slot and, when it is empty, claims it (0 comes back)
+      if (lane == 0) k = atomicCAS(reinterpret_cast<unsigned long long*>(a.slot_keys + slot), 0ull, key);
       k = shfl_u64(k, 0);
       if (k == 0ull) {
         // claimed: write the node, then publish it
