@@ -98,3 +98,11 @@ def test_quantised_append_writes_only_the_slots():
         for sl in range(bs):
             if not touched[blk, sl]:
                 assert np.array_equal(k2[blk, :, sl], kc[blk, :, sl])
+
+
+def test_nan_encodes_to_the_positive_nan_code_and_both_nan_codes_decode_to_nan():
+    # the reading: NaN stays NaN, as 0x7F whatever its sign; 0x7F and 0xFF are e4m3's only NaN codes
+    codes = fp8.e4m3_encode(np.array([np.nan, -np.nan, np.float64("nan")]))
+    assert codes.tolist() == [0x7F, 0x7F, 0x7F]
+    vals = fp8.e4m3_decode(np.array([0x7F, 0xFF, 0x7E, 0xFE], dtype=np.uint8))
+    assert np.isnan(vals[0]) and np.isnan(vals[1]) and vals[2] == 448.0 and vals[3] == -448.0

@@ -119,3 +119,63 @@ def test_unmutated_oracles_pass_their_pins():
     assert not pins_fail(tl, lookahead_cache,
                          ["build_forest", "longest_match", "propose", "propose_batch", "update_copy_len"])
     assert not pins_fail(ta_pins, ta_pins.ta, [])
+
+
+ATTENTION_MUTATIONS = [
+    ("for h in range(g * G, (g + 1) * G)]", "for h in range(g, Hq, Hkv)]"),                       # wrong GQA map
+    ("s = scale * (keys @ q_row)", "s = (keys @ q_row)"),                                         # dropped scale
+    ("if (int(mask_word) >> j) & 1:", "if (int(mask_word) >> (n_cand - 1 - j)) & 1:"),            # reversed bits
+    ("vis = list(range(P))", "vis = list(range(P + 1))"),                                         # off-by-one prefix
+    ("kc[phys, h, s % bs, :] = k_new[b, i, h, :]", "kc[phys, h, (s + 1) % bs, :] = k_new[b, i, h, :]"),  # slot
+    ("vc[phys, h, s % bs, :] = v_new[b, i, h, :]", "vc[phys, h, s % bs, :] = v_new[b, i, 0, :]"),  # append head
+    ("return np.zeros(values.shape[-1], dtype=np.float64)", "return np.ones(values.shape[-1], dtype=np.float64)"),
+    ("phys = int(table_row[p // block_size])", "phys = int(table_row[p // block_size]) if p else 0"),  # table walk
+]
+
+FP8_MUTATIONS = [
+    ("c = lo if (lo & 1) == 0 else hi", "c = lo"),                                                 # ties down
+    ("a = min(abs(v), E4M3_MAX)", "a = abs(v)"),                                                   # no saturation
+    ("if np.signbit(v):", "if v < 0:"),                                                            # -0 loses its sign
+    ("sub = sign * (m / 8.0) * 2.0 ** -6", "sub = sign * (m / 8.0) * 2.0 ** -7"),                 # subnormal scale
+    ("flat_o[k] = 0x7F", "flat_o[k] = 0xFF"),                                                      # NaN code
+]
+
+_ATTN_NAMES = ("gather_sequence_kv", "paged_kv_append", "paged_tree_attention", "softmax_attend", "visible_positions",
+               "widen_to_f64", "within_tolerance")
+
+
+def _oracle_with(mod):
+    import oracle
+    ns = types.SimpleNamespace(**{k: getattr(oracle, k) for k in dir(oracle) if not k.startswith("__")})
+    for n in _ATTN_NAMES:
+        setattr(ns, n, getattr(mod, n))
+    return ns
+
+
+@pytest.mark.parametrize("old,new", ATTENTION_MUTATIONS)
+def test_attention_pins_catch(old, new):
+    import tests.test_oracle as t
+    saved = t.oracle
+    t.oracle = _oracle_with(mutant("paged_attention", old, new))
+    try:
+        assert pins_fail(t, None, [])
+    finally:
+        t.oracle = saved
+
+
+@pytest.mark.parametrize("old,new", FP8_MUTATIONS)
+def test_fp8_pins_catch(old, new):
+    import tests.test_oracle_fp8 as t
+    saved = t.fp8
+    t.fp8 = mutant("fp8", old, new)
+    try:
+        assert pins_fail(t, None, [])
+    finally:
+        t.fp8 = saved
+
+
+def test_unmutated_attention_and_fp8_oracles_pass_their_pins():
+    import tests.test_oracle as t_attn
+    import tests.test_oracle_fp8 as t_fp8
+    assert not pins_fail(t_attn, None, [])
+    assert not pins_fail(t_fp8, None, [])
