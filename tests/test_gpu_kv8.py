@@ -46,11 +46,11 @@ def gpu_attention_e4m3(w, c8):
 def special_rows(w):
     """Overwrite some new K/V rows with values that probe the rounding: exact midpoints between e4m3
     neighbours (ties go to the even code), values past 448 (saturation), +-inf, tiny values
-    (subnormal codes and underflow to zero) and signed zeros."""
+    (subnormal codes and underflow to zero), signed zeros and NaN (both signs, through V = -row)."""
     k, v = w.k_new.clone(), w.v_new.clone()
     D = w.D
     probe = torch.tensor([1.0625, 1.1875, -1.0625, 0.3125 * 1.0625, 500.0, -1e4, float("inf"), float("-inf"),
-                          2.0 ** -10, -(2.0 ** -10) * 1.5, 2.0 ** -12, 0.0, -0.0, 448.0, 464.0, 480.0])
+                          2.0 ** -10, -(2.0 ** -10) * 1.5, 2.0 ** -12, 0.0, -0.0, 448.0, 464.0, 480.0, float("nan")])
     reps = (D + len(probe) - 1) // len(probe)
     row = probe.repeat(reps)[:D].to(k.dtype)
     k[0, 0, 0] = row
@@ -84,7 +84,7 @@ def test_quantising_append_bit_exact(dtype, D, bs):
     codes = g["kc"][blk, 0, P0 % bs].cpu().numpy()
     if dtype == "bf16":                            # scale 1: 1.0625 is a tie between 1.0 and 1.125
         assert codes[0] == 0x38 and codes[2] == 0xB8 and codes[4] == 0x7E and codes[6] == 0x7E
-        assert codes[7] == 0xFE and codes[11] == 0x00 and codes[12] == 0x80
+        assert codes[7] == 0xFE and codes[11] == 0x00 and codes[12] == 0x80 and codes[16] == 0x7F
 
 
 @pytest.mark.parametrize("grid", [0, 1, 3, 50])
