@@ -46,7 +46,10 @@ from paged_kv_cache_tree_b200 import workloads as wl  # noqa: E402
 METRIC = "paged tree-attn KV GB/s & % of B200 HBM peak; candidate-tokens/s vs CPU oracle"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-DEFAULT_WORKLOAD = "decode"
+DEFAULT_WORKLOAD = "long"
+# the other full-size workloads, each measured in the same run under "per_config"
+PER_CONFIG = ("decode", "chain", "tree", "long")
+CLOCK_WINDOW_S = 1.5
 KERNEL_SOURCES = ("device_common.cuh", "verify_mma.cuh", "verify_mma.cu", "verify_tc.cuh", "verify_tc.cu")
 
 
@@ -210,6 +213,15 @@ def oracle_sample(w, budget_s: float):
     return nbytes, ncand, spent, f"{done_b} of {w.B} sequences (all their KV heads and candidates), append + attention"
 
 
+def host_cores() -> dict:
+    """Host CPU counts: all logical CPUs, the ones this process may run on, and the BLAS pool."""
+    try:
+        aff = len(os.sched_getaffinity(0))
+    except Exception:
+        aff = os.cpu_count() or 1
+    return {"host_cpus": os.cpu_count() or 1, "affinity_cpus": aff, "blas_threads": blas_threads()}
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -236,7 +248,8 @@ def run_reference(args, world, rank):
         tot_cand += ncnd
         tot_s += s
     gbs = tot_bytes / tot_s / 1e9
-    cores = blas_threads()
+    hc = host_cores()
+    cores = hc["blas_threads"]
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
@@ -245,7 +258,7 @@ def run_reference(args, world, rank):
                    "l2": "not applicable (host)"},
         "candidate_tokens_per_s": tot_cand / tot_s,
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: {desc}"},
+                         "sample": f"each step: {desc}", **hc},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     return line
@@ -425,6 +438,83 @@ def measure_lookahead(taco, dev, stream, args):
     }
 
 
+def sustain(step, seconds: float, dev) -> int:
+    """Run `step` back to back for about `seconds` (untimed), so that clock samples see the kernel under
+    load for longer than one nvidia-smi period. Returns the number of steps run."""
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(50):
+            step()
+        torch.cuda.synchronize(dev)
+        n += 50
+    return n
+
+
+def measure_config(taco, name, world, rank, dev, stream, args, peak, peak_kind):
+    """One full-size workload's verify step (paged_tree_attention_append), timed on its own with CUDA events
+    on its stream: 200 steps after the warm-up, max over ranks, then an untimed window of the same step
+    for the clock record; plus the step over e4m3 caches where that kernel exists."""
+    w = wl.make_workload(name, seed=1000 + wl.WORKLOADS[name]["k"] + 7919 * rank, fill="zero")
+    d = w.to(dev)
+    out = torch.empty_like(d.q)
+    nbytes = step_bytes(w)
+    fused = w.G * w.C <= 16
+
+    def step(ev_pair=None):
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        taco.paged_tree_attention_append(d.q, d.k_new, d.v_new, d.k_cache, d.v_cache, d.block_tables, d.context_lens,
+                                         d.num_candidates, d.tree_mask, w.scale, out=out, stream=stream)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    n = 200
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for k in range(n):
+        step(pairs[k])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    sustain(step, CLOCK_WINDOW_S, dev)
+    clocks = sampler.stop() if sampler else None
+    barrier(world)
+    taco.check_device(stream)
+    ms_per_step = max_over_ranks(t0.elapsed_time(t1) / n, world)
+    launch_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in pairs) / n, world)
+    achieved = nbytes / (launch_ms * 1e-3) / 1e9
+    kv8 = measure_kv8(taco, w, d, dev, stream, args)
+    if kv8 is not None:
+        kv8["attention_frac"] = kv8["attention_GBps"] / peak
+        kv8["traffic"] = recorded_traffic(f"{name}_e4m3")
+        kv8["attention_speedup_vs_16bit"] = launch_ms / (kv8["attention_us"] * 1e-3)
+    res = {
+        "workload": wl.WORKLOAD_DESCRIPTIONS[name], "steps": n,
+        "value": world * nbytes / (ms_per_step * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_per_step,
+        "step_bytes": nbytes, "candidate_tokens_per_step": w.candidate_tokens(),
+        "candidate_tokens_per_s": world * w.candidate_tokens() / (ms_per_step * 1e-3),
+        "candidate_tokens_per_s_at_roofline": world * w.candidate_tokens() * peak * 1e9 / nbytes,
+        "hbm_frac_of_nominal_8tbs": nbytes / (ms_per_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(name), "algorithmic_bytes": nbytes, "launch_ms": launch_ms,
+                     "peak_source": f"{peak_kind} hbm_gbs",
+                     "kernel": "paged_tree_attention_append (append fused into the verify)" if fused else
+                               "paged_tree_attention_append (append kernel, then the verify)"},
+        "gpu_launches": (1 if fused else 2) * n,
+        "clocks": clocks,
+        "kv8": kv8,
+    }
+    del d, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, world, rank, local):
     import paged_kv_cache_tree_b200 as taco
 
@@ -466,8 +556,14 @@ def run_ours(args, world, rank, local):
         step(pairs[k])
     t_stop.record(stream)
     torch.cuda.synchronize(dev)
-    barrier(world)
+    # the timed region is shorter than one nvidia-smi sample: keep the same step running, untimed, for
+    # a while longer so that the clock record covers the kernel under load
+    sustained_steps = sustain(step, CLOCK_WINDOW_S, dev)
     clocks = sampler.stop() if sampler else None
+    if clocks is not None:
+        clocks["window"] = (f"the timed region plus {sustained_steps} more steps of the same call right after it "
+                            f"(untimed, about {CLOCK_WINDOW_S} s)")
+    barrier(world)
     taco.check_device(stream)
     region_ms = t_start.elapsed_time(t_stop)
     attn_ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
@@ -534,10 +630,17 @@ def run_ours(args, world, rank, local):
     kv8 = measure_kv8(taco, w, d, dev, stream, args)
     prefix = measure_prefix(taco, dev, stream, args)
     lookahead = measure_lookahead(taco, dev, stream, args)
+    del d, out, dev_in, out_dev
+    torch.cuda.empty_cache()
+    peak, peak_kind = measured_peaks()
+    per_config = {}
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            if name != args.workload:
+                per_config[name] = measure_config(taco, name, world, rank, dev, stream, args, peak, peak_kind)
 
     if rank != 0:
         return None
-    peak, peak_kind = measured_peaks()
     achieved = nbytes / (attn_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -566,7 +669,18 @@ def run_ours(args, world, rank, local):
         "kv8": kv8,
         "prefix_cache": prefix,
         "lookahead_cache": lookahead,
+        "per_config": per_config,
     }
+    if not args.no_per_config:
+        # the headline workload's own entry, from the timed region above
+        per_config[args.workload] = {
+            "workload": wl.WORKLOAD_DESCRIPTIONS[args.workload], "steps": args.steps, "value": value, "unit": "GB/s",
+            "ms_per_step": ms_per_step, "step_bytes": nbytes, "candidate_tokens_per_step": w.candidate_tokens(),
+            "candidate_tokens_per_s": line["candidate_tokens_per_s"],
+            "candidate_tokens_per_s_at_roofline": line["candidate_tokens_per_s_at_roofline"],
+            "hbm_frac_of_nominal_8tbs": line["hbm_frac_of_nominal_8tbs"], "roofline": line["roofline"],
+            "gpu_launches": line["gpu_launches"], "clocks": clocks, "kv8": kv8, "headline": True}
+        line["per_config"] = {k: per_config[k] for k in PER_CONFIG if k in per_config}
     if kv8 is not None:
         kv8["attention_frac"] = kv8["attention_GBps"] / peak
         kv8["traffic"] = recorded_traffic(f"{args.workload}_e4m3")
@@ -575,8 +689,10 @@ def run_ours(args, world, rank, local):
     accept["argmax_roofline"]["frac"] = accept["argmax_roofline"]["achieved"] / peak
     if world == 1 and not args.no_cpu_baseline:
         nb, ncnd, secs, desc = oracle_sample(w, args.cpu_budget)
-        line["cpu_baseline"] = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"{desc}; {secs:.1f} s", "candidate_tokens_per_s": ncnd / secs}
+        hc = host_cores()
+        line["cpu_baseline"] = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": hc["blas_threads"],
+                                "kind": "oracle", "sample": f"{desc}; {secs:.1f} s",
+                                "candidate_tokens_per_s": ncnd / secs, **hc}
     return line
 
 
@@ -589,6 +705,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the other workloads' per_config entries")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

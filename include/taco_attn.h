@@ -24,8 +24,14 @@
  *  - Host-side validation runs before any launch; a non-OK status means nothing was enqueued, and
  *    taco_attn_last_error() gives a message (thread-local).
  *  - Values inside device arrays (block ids, lengths, slots) are checked on the device: an
- *    out-of-range value sets a bit in a per-device error word and the offending access is skipped
- *    (it never faults or traps). taco_attn_check_device() reads and clears that word.
+ *    out-of-range value sets a bit in an error word and the offending access is skipped (it never
+ *    faults or traps). Each (device, stream) pair has its own word; taco_attn_check_device(stream)
+ *    reads and clears the word of the current device and that stream.
+ *  - Library-owned device memory (the error word and the split-KV workspace) is kept per (device,
+ *    stream handle). Calls on different streams may therefore run concurrently; calls on one stream
+ *    are ordered by the stream. A stream handle that is destroyed while its work is still queued and
+ *    then reused by a new stream shares the old workspace: let such work finish first.
+ *    paged_tree_attention_noalloc is the exception: it uses one fixed array per device (see there).
  *
  * Shapes: B batch, C max candidates per sequence (1..32), Hq / Hkv query / KV heads (Hq % Hkv == 0,
  * G = Hq / Hkv), D head dim (64 or 128), bs block size (power of two, 8..256), NB physical blocks,
@@ -81,9 +87,10 @@ typedef int32_t taco_status;
  *                   see no key are zeros. Must not alias any input.
  *   query head h reads KV head h / G.
  * Softmax state (max, sum) and the output accumulator are fp32; the result is rounded once to
- * `dtype` (round to nearest even). The library keeps a per-device workspace for split-KV partial
- * results; the first call on a device (or one that needs a larger workspace) allocates it with
- * cudaMalloc and therefore synchronises the device.
+ * `dtype` (round to nearest even). The library keeps a workspace for split-KV partial results per
+ * (device, stream); the first call on a stream (or one that needs a larger workspace) allocates it
+ * with cudaMalloc and therefore synchronises the device. Calls on different streams use different
+ * workspaces and may overlap on the GPU.
  */
 taco_status paged_tree_attention(const void* q, const void* k_cache, const void* v_cache,
                                  const int32_t* block_tables, const int32_t* context_lens,
@@ -133,8 +140,9 @@ taco_status paged_tree_attention_append(const void* q, const void* k_new, const 
                                         void* stream);
 
 /*
- * paged_tree_attention_noalloc: the same operation, arguments and results as paged_tree_attention,
- * for callers that cannot allocate device memory. The pages have no counterpart of this entry point;
+ * paged_tree_attention_noalloc: the same arguments and result (within the tolerance that holds for
+ * every kernel of this library) as paged_tree_attention, for callers that cannot allocate device
+ * memory. The pages have no counterpart of this entry point;
  * it exists because paged_tree_attention grows a workspace with cudaMalloc on first use, which a
  * caller cannot allow when it runs under a fixed memory-pool budget (e.g. a server that has handed
  * all free HBM to its KV cache), when an implicit device synchronisation mid-step is not acceptable,
@@ -144,12 +152,17 @@ taco_status paged_tree_attention_append(const void* q, const void* k_new, const 
  *   - Limit: at most 65536 work units (batch * num_kv_heads * row groups of up to 64 packed query
  *     rows); larger calls return TACO_ERR_UNSUPPORTED with a message and enqueue nothing. The grid is
  *     capped so that the split-KV partials fit the scratch.
+ *   - Kernel: always the mma.sync verify kernel (at most 64 packed rows per work unit), never the
+ *     tcgen05 kernel paged_tree_attention uses for G * C >= 48, whose partials would not fit the
+ *     array; for 64-row units the grid is also capped (121 CTAs at D = 128) so that the partials fit.
+ *     Wide calls (chain- and tree-shaped verifies) therefore run slower here.
  *   - All calls on a device share the array and it keeps the last call's contents; each call clears
  *     what must start at zero on `stream` first. Calls whose work overlaps on the GPU race: order them
  *     on one stream.
- *   - The first call on a device looks up the array's address (cudaGetSymbolAddress, that device
- *     current); make it before any stream capture.
- *   - Device-side range violations are skipped but are not visible to taco_attn_check_device.
+ *   - The first call on a device (of this function or of taco_attn_check_noalloc) looks up the
+ *     array's address (cudaGetSymbolAddress, that device current); make it before any stream capture.
+ *   - Device-side range violations and wait timeouts are skipped and recorded in the array's own
+ *     error word, which accumulates until taco_attn_check_noalloc reads and clears it.
  */
 taco_status paged_tree_attention_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                          const int32_t* block_tables, const int32_t* context_lens,
@@ -159,6 +172,15 @@ taco_status paged_tree_attention_noalloc(const void* q, const void* k_cache, con
                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                          int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
                                          void* stream);
+
+/*
+ * taco_attn_check_noalloc: synchronise `stream`, then read and clear the error word of
+ * paged_tree_attention_noalloc's fixed array on the current device (TACO_DEVERR_* bits). Returns
+ * TACO_OK if it was zero, TACO_ERR_DEVICE_CHECK otherwise (bits in the message and in *bits_out when
+ * bits_out is not NULL). Allocates nothing. The pages have no counterpart of this function: it only
+ * reports the errors of the allocation-free entry point above.
+ */
+taco_status taco_attn_check_noalloc(void* stream, uint32_t* bits_out);
 
 /*
  * 8-bit KV cache. The 53ai.com workshop page (section "5. 支持 Quantization（模型量化）") lists 8-bit
@@ -354,18 +376,22 @@ taco_status prefix_cache_insert(const int32_t* tokens, const int32_t* seq_starts
 const char* taco_attn_last_error(void);
 
 /*
- * Synchronise `stream`, then read and clear the current device's error word. Returns TACO_OK if it
+ * Synchronise `stream`, then read and clear the error word of (the current device, `stream`): the
+ * bits set by calls enqueued on that stream, and by no other stream's calls. Returns TACO_OK if it
  * was zero, TACO_ERR_DEVICE_CHECK otherwise (the bits are in the message and in *bits_out when
- * bits_out is not NULL). After a wait timeout it also clears the split-KV arrival counters.
+ * bits_out is not NULL). After a wait timeout it also clears that stream's split-KV arrival
+ * counters. paged_tree_attention_noalloc has its own word: taco_attn_check_noalloc reads it.
  */
 taco_status taco_attn_check_device(void* stream, uint32_t* bits_out);
 
-/* Free the per-device workspaces (call only when no work using them is in flight). */
+/* Free every (device, stream) workspace (call only when no work using them is in flight). */
 void taco_attn_release_workspace(void);
 
 /* Tuning / test knobs (process-wide). */
 #define TACO_OPT_GRID_CTAS 1   /* verify grid size in CTAs; 0 = automatic (2 per SM). */
 #define TACO_OPT_KERNEL 2      /* 0 = automatic, 1 = mma.sync path, 2 = tcgen05 path (where built) */
+#define TACO_OPT_L2_PREFETCH 3 /* key tiles of K/V the verify asks L2 to fetch ahead of its shared-memory
+                                  loads: -1 = the kernel's default, 0 = none, up to 64 */
 taco_status taco_attn_set_option(int32_t key, int64_t value);
 
 /* ABI version of this header (bumped on any signature change). */

@@ -7,8 +7,10 @@ from ._lib import (  # noqa: F401
     PrefixCache,
     TACO_OPT_GRID_CTAS,
     TACO_OPT_KERNEL,
+    TACO_OPT_L2_PREFETCH,
     TacoError,
     check_device,
+    check_noalloc,
     load,
     logits_argmax,
     lookahead_propose,

@@ -27,6 +27,7 @@ TACO_DTYPE_BF16 = 1
 
 TACO_OPT_GRID_CTAS = 1
 TACO_OPT_KERNEL = 2
+TACO_OPT_L2_PREFETCH = 3
 
 EXPORTED = (
     "paged_tree_attention",
@@ -37,6 +38,7 @@ EXPORTED = (
     "paged_kv_append_e4m3",
     "taco_attn_last_error",
     "taco_attn_check_device",
+    "taco_attn_check_noalloc",
     "taco_attn_release_workspace",
     "taco_attn_set_option",
     "taco_attn_version",
@@ -83,6 +85,8 @@ def load() -> ctypes.CDLL:
     lib.taco_attn_last_error.restype = ctypes.c_char_p
     lib.taco_attn_check_device.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.taco_attn_check_device.restype = i32
+    lib.taco_attn_check_noalloc.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.taco_attn_check_noalloc.restype = i32
     lib.taco_attn_release_workspace.argtypes = []
     lib.taco_attn_release_workspace.restype = None
     lib.taco_attn_set_option.argtypes = [i32, ctypes.c_int64]
@@ -365,6 +369,17 @@ def check_device(stream=None, device=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     bits = ctypes.c_uint32(0)
     st = lib.taco_attn_check_device(_stream_handle(stream, dev), ctypes.byref(bits))
+    _check(st)
+    return int(bits.value)
+
+
+def check_noalloc(stream=None, device=None) -> int:
+    """Synchronise the stream and return the error bits of paged_tree_attention_noalloc's fixed scratch
+    (raises TacoError if any are set); the word is cleared."""
+    lib = load()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    bits = ctypes.c_uint32(0)
+    st = lib.taco_attn_check_noalloc(_stream_handle(stream, dev), ctypes.byref(bits))
     _check(st)
     return int(bits.value)
 

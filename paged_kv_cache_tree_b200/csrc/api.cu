@@ -7,8 +7,10 @@
 #include <cstdio>
 #include <algorithm>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "device_common.cuh"
 #include "launchers.h"
@@ -35,7 +37,8 @@ taco_status cuda_fail(cudaError_t e, const char* what) {
   return fail(TACO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-// Workspace of one device: [error word | counters | partial lse | partial O].
+// Workspace of one (device, stream): [error word | counters | partial lse | partial O]. Calls on
+// different streams never share one, so they may overlap on the GPU.
 struct Workspace {
   uint8_t* base = nullptr;
   size_t bytes = 0;
@@ -46,23 +49,33 @@ struct Workspace {
   size_t lse_cap = 0;  // floats
   float* part_o = nullptr;
   size_t o_cap = 0;    // floats
-  int sm_count = 0;
 };
 
 std::mutex g_mu;
-Workspace g_ws[kMaxDevices];
+std::map<std::pair<int, uintptr_t>, Workspace> g_ws;  // keyed by (device, stream handle)
+int g_sm_count[kMaxDevices];
 int64_t g_opt_grid = 0;
 int64_t g_opt_kernel = 0;
+int64_t g_opt_prefetch = -1;  // -1 = the kernel's default distance
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Make sure device `dev`'s workspace has room; returns a status. Caller holds g_mu.
-taco_status ensure_workspace(int dev, size_t counters, size_t lse_floats, size_t o_floats) {
-  Workspace& w = g_ws[dev];
-  if (w.sm_count == 0) {
-    cudaError_t e = cudaDeviceGetAttribute(&w.sm_count, cudaDevAttrMultiProcessorCount, dev);
+// SM count of device `dev`. Caller holds g_mu.
+taco_status sm_count_of(int dev, int* out) {
+  if (g_sm_count[dev] == 0) {
+    cudaError_t e = cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   }
+  *out = g_sm_count[dev];
+  return TACO_OK;
+}
+
+// Make sure the workspace of (device `dev`, `stream`) has room and return it in *out; returns a status.
+// Caller holds g_mu.
+taco_status ensure_workspace(int dev, void* stream, size_t counters, size_t lse_floats, size_t o_floats,
+                             Workspace** out) {
+  Workspace& w = g_ws[std::make_pair(dev, reinterpret_cast<uintptr_t>(stream))];
+  *out = &w;
   if (w.base && counters <= w.counters_cap && lse_floats <= w.lse_cap && o_floats <= w.o_cap) return TACO_OK;
   // grow (keeping at least the old capacities); the old buffer may still be in use by queued
   // work, so wait for the device before freeing it
@@ -79,7 +92,7 @@ taco_status ensure_workspace(int dev, size_t counters, size_t lse_floats, size_t
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize (workspace grow)");
     cudaMemcpy(&old_err, w.error_word, 4, cudaMemcpyDeviceToHost);
     cudaFree(w.base);
-    w = Workspace{nullptr, 0, nullptr, nullptr, 0, nullptr, 0, nullptr, 0, w.sm_count};
+    w = Workspace{};
   }
   void* p = nullptr;
   cudaError_t e = cudaMalloc(&p, total);
@@ -200,6 +213,11 @@ taco_status taco_attn_set_option(int32_t key, int64_t value) {
     g_opt_kernel = value;
     return TACO_OK;
   }
+  if (key == TACO_OPT_L2_PREFETCH) {
+    if (value < -1 || value > 64) return fail(TACO_ERR_INVALID_ARG, "prefetch distance must be in [-1, 64]");
+    g_opt_prefetch = value;
+    return TACO_OK;
+  }
   return fail(TACO_ERR_INVALID_ARG, "unknown option key %d", key);
 }
 
@@ -262,16 +280,16 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
   }
   const int64_t units = static_cast<int64_t>(batch) * num_kv_heads * row_groups;
 
-  if (g_ws[dev].sm_count == 0) {
-    e = cudaDeviceGetAttribute(&g_ws[dev].sm_count, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-  }
-  int grid = static_cast<int>(g_opt_grid);
-  if (grid == 0) grid = (use_tc ? 1 : taco::mma_ctas_per_sm(rows)) * g_ws[dev].sm_count;
-  const size_t slots = 2 * static_cast<size_t>(grid);
-  st = ensure_workspace(dev, static_cast<size_t>(units), slots * rows, slots * rows * head_dim);
+  int sms = 0;
+  st = sm_count_of(dev, &sms);
   if (st != TACO_OK) return st;
-  Workspace& w = g_ws[dev];
+  int grid = static_cast<int>(g_opt_grid);
+  if (grid == 0) grid = (use_tc ? 1 : taco::mma_ctas_per_sm(rows)) * sms;
+  const size_t slots = 2 * static_cast<size_t>(grid);
+  Workspace* wp = nullptr;
+  st = ensure_workspace(dev, stream, static_cast<size_t>(units), slots * rows, slots * rows * head_dim, &wp);
+  if (st != TACO_OK) return st;
+  Workspace& w = *wp;
 
   const int tile = use_tc ? taco::tc_tile_keys() : taco::mma_tile_keys(rows, kv8);
   const int rpc = block_size < tile ? block_size : tile;
@@ -312,6 +330,8 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
   p.row_groups = row_groups;
   p.cands_per_group = cands_per_group;
   p.tile_keys = tile;
+  p.l2_prefetch_tiles = static_cast<int>(
+      g_opt_prefetch >= 0 ? g_opt_prefetch : (use_tc ? taco::kTcPrefetchTiles : taco::kMmaPrefetchTiles));
   p.k_scale = k_scale;
   p.v_scale = v_scale;
   if (k_new) {
@@ -397,9 +417,10 @@ taco_status paged_kv_append(const void* k_new, const void* v_new, const int32_t*
   uint32_t* err = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    st = ensure_workspace(dev, 0, 0, 0);
+    Workspace* wp = nullptr;
+    st = ensure_workspace(dev, stream, 0, 0, 0, &wp);
     if (st != TACO_OK) return st;
-    err = g_ws[dev].error_word;
+    err = wp->error_word;
   }
   taco::AppendArgs a{k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, err,
                      batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq};
@@ -429,9 +450,10 @@ taco_status paged_kv_append_e4m3(const void* k_new, const void* v_new, const int
   uint32_t* err = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    st = ensure_workspace(dev, 0, 0, 0);
+    Workspace* wp = nullptr;
+    st = ensure_workspace(dev, stream, 0, 0, 0, &wp);
     if (st != TACO_OK) return st;
-    err = g_ws[dev].error_word;
+    err = wp->error_word;
   }
   taco::AppendArgs a{k_new, v_new, block_tables, slot_offsets, k_cache, v_cache, err,
                      batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
@@ -441,16 +463,17 @@ taco_status paged_kv_append_e4m3(const void* k_new, const void* v_new, const int
   return TACO_OK;
 }
 
-// Error word of the current device (creates the workspace's header on first use).
-static taco_status device_error_word(uint32_t** out) {
+// Error word of (the current device, `stream`) (creates the workspace's header on first use).
+static taco_status stream_error_word(void* stream, uint32_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(TACO_ERR_UNSUPPORTED, "device index %d too large", dev);
   std::lock_guard<std::mutex> lk(g_mu);
-  taco_status st = ensure_workspace(dev, 0, 0, 0);
+  Workspace* wp = nullptr;
+  taco_status st = ensure_workspace(dev, stream, 0, 0, 0, &wp);
   if (st != TACO_OK) return st;
-  *out = g_ws[dev].error_word;
+  *out = wp->error_word;
   return TACO_OK;
 }
 
@@ -462,7 +485,7 @@ taco_status tree_mask_from_parents(const int32_t* parents, const int32_t* num_ca
   if (!parents || !num_candidates || !mask_out) return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
   if (batch == 0) return TACO_OK;
   uint32_t* err = nullptr;
-  taco_status st = device_error_word(&err);
+  taco_status st = stream_error_word(stream, &err);
   if (st != TACO_OK) return st;
   taco::MaskArgs a{parents, num_candidates, mask_out, err, batch, max_candidates};
   cudaError_t e = taco::launch_tree_masks(a, static_cast<cudaStream_t>(stream));
@@ -494,7 +517,7 @@ taco_status tree_greedy_accept(const int32_t* target_argmax, const int32_t* cand
     return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
   if (batch == 0) return TACO_OK;
   uint32_t* err = nullptr;
-  taco_status st = device_error_word(&err);
+  taco_status st = stream_error_word(stream, &err);
   if (st != TACO_OK) return st;
   taco::AcceptArgs a{target_argmax, candidate_tokens, parents, num_candidates, context_lens, accept_len,
                      accepted_path, bonus_token, slot_offsets_out, err, batch, max_candidates};
@@ -507,7 +530,7 @@ static taco_status prefix_common(const int32_t* tokens, const int32_t* seq_start
                                  const void* slot_nodes, int64_t capacity, const void* node_parent,
                                  const void* node_depth, const void* node_tokens, const void* out_blocks,
                                  int32_t batch, int32_t block_size, int32_t num_blocks, int32_t max_blocks,
-                                 uint32_t** err) {
+                                 void* stream, uint32_t** err) {
   if (!tokens || !seq_starts || !slot_keys || !slot_nodes || !node_parent || !node_depth || !node_tokens ||
       !out_blocks)
     return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
@@ -518,7 +541,7 @@ static taco_status prefix_common(const int32_t* tokens, const int32_t* seq_start
   if (num_blocks < 1) return fail(TACO_ERR_INVALID_ARG, "num_blocks must be >= 1");
   if (max_blocks < 1) return fail(TACO_ERR_INVALID_ARG, "max_blocks_per_seq must be >= 1");
   if (batch == 0) return TACO_OK;
-  return device_error_word(err);
+  return stream_error_word(stream, err);
 }
 
 taco_status prefix_cache_lookup(const int32_t* tokens, const int32_t* seq_starts, const uint64_t* slot_keys,
@@ -529,7 +552,8 @@ taco_status prefix_cache_lookup(const int32_t* tokens, const int32_t* seq_starts
   if (!out_matched) return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
   uint32_t* err = nullptr;
   taco_status st = prefix_common(tokens, seq_starts, slot_keys, slot_nodes, capacity, node_parent, node_depth,
-                                 node_tokens, out_blocks, batch, block_size, num_blocks, max_blocks_per_seq, &err);
+                                 node_tokens, out_blocks, batch, block_size, num_blocks, max_blocks_per_seq, stream,
+                                 &err);
   if (st != TACO_OK || batch == 0) return st;
   cudaError_t e = taco::launch_prefix_cache(false, tokens, seq_starts, nullptr, const_cast<uint64_t*>(slot_keys),
                                             const_cast<int32_t*>(slot_nodes), capacity, const_cast<int32_t*>(node_parent),
@@ -548,7 +572,8 @@ taco_status prefix_cache_insert(const int32_t* tokens, const int32_t* seq_starts
   if (!block_tables) return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
   uint32_t* err = nullptr;
   taco_status st = prefix_common(tokens, seq_starts, slot_keys, slot_nodes, capacity, node_parent, node_depth,
-                                 node_tokens, out_blocks, batch, block_size, num_blocks, max_blocks_per_seq, &err);
+                                 node_tokens, out_blocks, batch, block_size, num_blocks, max_blocks_per_seq, stream,
+                                 &err);
   if (st != TACO_OK || batch == 0) return st;
   cudaError_t e = taco::launch_prefix_cache(true, tokens, seq_starts, block_tables, slot_keys, slot_nodes, capacity,
                                             node_parent, node_depth, node_tokens, out_blocks, out_inserted, err, batch,
@@ -570,7 +595,7 @@ taco_status lookahead_propose(const int32_t* history, const int32_t* hist_starts
   if (batch < 0) return fail(TACO_ERR_INVALID_ARG, "batch must be >= 0");
   if (batch == 0) return TACO_OK;
   uint32_t* err = nullptr;
-  taco_status st = device_error_word(&err);
+  taco_status st = stream_error_word(stream, &err);
   if (st != TACO_OK) return st;
   cudaError_t e = taco::launch_lookahead_propose(history, hist_starts, global_len > 0 ? global_tokens : nullptr,
                                                  global_len, copy_len, max_match, batch, max_candidates, tokens_out,
@@ -603,8 +628,9 @@ taco_status taco_attn_check_device(void* stream, uint32_t* bits_out) {
   e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
   std::lock_guard<std::mutex> lk(g_mu);
-  Workspace& w = g_ws[dev];
-  if (!w.base) return TACO_OK;
+  auto it = g_ws.find(std::make_pair(dev, reinterpret_cast<uintptr_t>(stream)));
+  if (it == g_ws.end() || !it->second.base) return TACO_OK;
+  Workspace& w = it->second;
   uint32_t bits = 0;
   e = cudaMemcpy(&bits, w.error_word, 4, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy (error word)");
@@ -626,12 +652,12 @@ void taco_attn_release_workspace(void) {
   std::lock_guard<std::mutex> lk(g_mu);
   int cur = 0;
   cudaGetDevice(&cur);
-  for (int d = 0; d < kMaxDevices; ++d) {
-    if (!g_ws[d].base) continue;
-    cudaSetDevice(d);
-    cudaFree(g_ws[d].base);
-    g_ws[d] = Workspace{};
+  for (auto& kv : g_ws) {
+    if (!kv.second.base) continue;
+    cudaSetDevice(kv.first.first);
+    cudaFree(kv.second.base);
   }
+  g_ws.clear();
   cudaSetDevice(cur);
 }
 

@@ -17,6 +17,9 @@ namespace taco {
 constexpr int kTileKeys = 64;                 // keys per pipeline stage
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a pipeline wait gives up after 2 s
+// default L2 prefetch distances (key tiles past the latest load) of the two verify kernels
+constexpr int kTcPrefetchTiles = 0;
+constexpr int kMmaPrefetchTiles = 0;
 
 struct VerifyParams {
   const void* q;
@@ -35,6 +38,7 @@ struct VerifyParams {
   int row_groups;        // number of row groups per (sequence, KV head)
   int cands_per_group;   // tensor-core path: candidates per row group (rows = cands_per_group * G)
   int tile_keys;         // keys per work tile of the kernel (64 or 128)
+  int l2_prefetch_tiles; // key tiles whose K/V the producer asks L2 to fetch ahead of its loads (0 = none)
   const float* k_scale;  // e4m3 caches: per-KV-head scales (K value = code * k_scale[h]); else null
   const float* v_scale;
   // fused append (16-bit caches, units of <= 16 rows): candidate i's new K/V rows [B, C, Hkv, D] go to
@@ -134,6 +138,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
       : "memory");
+}
+
+// L2 prefetch of one TMA tile: no shared memory, no completion. The later tile load of the same
+// coordinates then finds its lines in L2 (or already on their way), so HBM latency is covered by
+// requests that hold no shared-memory stage.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
@@ -478,6 +492,80 @@ struct SegCursor {
         L = clamp_context(p, b, report);
         Tb = tiles_of(L, p.tile_keys);
       }
+    }
+  }
+};
+
+// Walks a CTA's tiles like its producers do and asks L2 to fetch each tile's K and V chunks, a set
+// number of tiles before the producer loads them (tma_prefetch_2d). A shared-memory ring can only
+// hold a few tiles while HBM latency under load is several microseconds; these requests keep more of
+// the stream in flight without holding any stage. Run by one whole warp; prefetch() issues every tile
+// whose CTA-local ordinal is below `upto` and has not been issued yet. Lanes take one chunk each,
+// exactly as the loads do, and chunks with a bad block id are skipped (the loads report them).
+template <int kPanels, int kColsPerPanel>
+struct TilePrefetcher {
+  SegCursor c;
+  int tl, tend, g, nblk, win;
+  int32_t win_val;
+  const int32_t* bt_row;
+  int64_t next;  // CTA-local ordinal of the next tile to prefetch
+  bool have;
+
+  __device__ __forceinline__ void start_segment(const VerifyParams& p) {
+    tl = c.tile;
+    tend = c.seg_end();
+    g = c.j / p.row_groups;
+    nblk = (c.L + p.bs - 1) / p.bs;
+    bt_row = p.block_tables + static_cast<int64_t>(c.b) * p.max_blocks;
+    win = -1000000;
+    win_val = -1;
+  }
+  __device__ __forceinline__ void step(const VerifyParams& p) {
+    ++next;
+    if (++tl == tend) {
+      c.next_segment(p, false);
+      have = c.valid();
+      if (have) start_segment(p);
+    }
+  }
+  // `skip` leading tiles are passed over (the producer's first loads find an empty ring anyway)
+  __device__ __forceinline__ void init(const VerifyParams& p, int b0, int64_t base_b0, int64_t lo, int64_t hi,
+                                       int skip) {
+    c.init(p, b0, base_b0, lo, hi, false);
+    next = 0;
+    have = c.valid();
+    if (have) start_segment(p);
+    while (have && next < skip) step(p);
+  }
+  __device__ __forceinline__ void prefetch(const VerifyParams& p, int64_t upto, const CUtensorMap* mk,
+                                           const CUtensorMap* mv) {
+    const int lane = threadIdx.x & 31;
+    const int tk = p.tile_keys;
+    const int rpc = p.bs < tk ? p.bs : tk;
+    const int chunks_per_tile = tk / rpc;
+    while (have && next < upto) {
+      const int L = c.L;
+      const int key0 = tl * tk;
+      int nvalid = L > key0 ? (L - key0 + rpc - 1) / rpc : 0;
+      if (nvalid > chunks_per_tile) nvalid = chunks_per_tile;
+      const int lb_first = key0 / p.bs;
+      if (nvalid > 0 && (lb_first < win || (key0 + (nvalid - 1) * rpc) / p.bs >= win + 32)) {
+        win = lb_first;
+        const int lb = win + lane;
+        win_val = lb < nblk ? __ldg(bt_row + lb) : -1;
+      }
+      const int my_lb = (key0 + lane * rpc) / p.bs;
+      const int32_t blk = __shfl_sync(0xffffffffu, win_val, (my_lb - win) & 31);
+      if (lane < nvalid && blk >= 0 && blk < p.num_blocks) {
+        const int row = (blk * p.Hkv + g) * p.bs + (key0 + lane * rpc) % p.bs;
+#pragma unroll
+        for (int pn = 0; pn < kPanels; ++pn) {
+          tma_prefetch_2d(mk, pn * kColsPerPanel, row);
+          tma_prefetch_2d(mv, pn * kColsPerPanel, row);
+        }
+      }
+      __syncwarp();
+      step(p);
     }
   }
 };

@@ -1,13 +1,18 @@
 // paged_tree_attention_noalloc: the verify entry point for callers that must not allocate device
 // memory.
 //
-// paged_tree_attention keeps a per-device workspace for its split-KV partial results and grows it
-// with cudaMalloc on first use. Some callers cannot allow that: code running under a fixed
-// memory-pool budget (an inference server that reserves all free HBM for its KV cache up front),
-// callers that must not trigger the implicit device synchronisation of cudaMalloc/cudaFree in the
-// middle of a pipelined step, and hosts that forbid allocation after start-up. This variant runs the
-// same verify kernel but takes its scratch (split-KV partials, arrival counters, error word) from a
-// fixed array that lives in the library's device image instead of calling cudaMalloc.
+// paged_tree_attention keeps a workspace for its split-KV partial results and grows it with
+// cudaMalloc on first use. Some callers cannot allow that: code running under a fixed memory-pool
+// budget (an inference server that reserves all free HBM for its KV cache up front), callers that
+// must not trigger the implicit device synchronisation of cudaMalloc/cudaFree in the middle of a
+// pipelined step, and hosts that forbid allocation after start-up. This variant computes the same
+// result but takes its scratch (split-KV partials, arrival counters, error word) from a fixed array
+// that lives in the library's device image instead of calling cudaMalloc.
+//
+// Kernel: it always runs the mma.sync verify kernel, with at most 64 packed query rows per work unit,
+// and never the tcgen05 kernel that paged_tree_attention picks for wide tiles (G * C >= 48): that
+// kernel's partials (128 rows per slot, two slots per SM) would not fit the fixed array. Wide calls
+// (the chain and tree verify shapes) are therefore slower here than through paged_tree_attention.
 //
 // Limits and rules:
 //  - The scratch is kNoAllocScratchBytes = 8 MiB per device. Every GPU that loads the library holds
@@ -17,13 +22,15 @@
 //    anything is enqueued. The kernel's grid is capped so that its partials fit in the scratch; for
 //    wide row groups (G * C > 32) this means fewer CTAs than paged_tree_attention uses.
 //  - All calls on a device share the one array, and it keeps the previous call's contents. Each call
-//    clears the arrival counters and the error word it needs on `stream` before its kernel runs. Two
-//    calls whose work overlaps on the GPU (different streams without ordering between them) race on
-//    the scratch and give wrong results: serialise them.
-//  - The first call on a device looks up the array's device address with cudaGetSymbolAddress, with
-//    that device current; make that first call before any stream capture begins.
-//  - Device-side range violations (bad block ids, lengths) are skipped as in paged_tree_attention, but
-//    they are recorded in this scratch's own error word, which taco_attn_check_device does not read.
+//    clears the arrival counters it needs on `stream` before its kernel runs. Two calls whose work
+//    overlaps on the GPU (different streams without ordering between them) race on the scratch and
+//    give wrong results: serialise them.
+//  - The first call on a device (of this entry point or of taco_attn_check_noalloc) looks up the
+//    array's device address with cudaGetSymbolAddress, with that device current; make that first call
+//    before any stream capture begins.
+//  - Device-side range violations (bad block ids, lengths) and wait timeouts are skipped as in
+//    paged_tree_attention and recorded in this scratch's own error word. The word accumulates over
+//    calls until taco_attn_check_noalloc reads and clears it (taco_attn_check_device does not see it).
 //  - No cudaMalloc, cudaFree or other allocating call is made.
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -64,6 +71,21 @@ taco_status fail(taco_status st, const char* fmt, ...) {
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Device address of the scratch on the current device `dev`, looked up once per device (with `dev`
+// current) and cached. Caller holds g_mu.
+taco_status scratch_of(int dev, unsigned char** out) {
+  if (!g_scratch_addr[dev]) {
+    void* addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+    if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    e = cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    g_scratch_addr[dev] = static_cast<unsigned char*>(addr);
+  }
+  *out = g_scratch_addr[dev];
+  return TACO_OK;
+}
 
 }  // namespace
 
@@ -112,16 +134,8 @@ extern "C" taco_status paged_tree_attention_noalloc(
   int sms = 0;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_addr[dev]) {
-      // one-time set-up on this device (the current one): the array's device address
-      void* addr = nullptr;
-      e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
-      if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-      e = cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
-      if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
-      g_scratch_addr[dev] = static_cast<unsigned char*>(addr);
-    }
-    base = g_scratch_addr[dev];
+    taco_status st = scratch_of(dev, &base);  // one-time set-up on this device (the current one)
+    if (st != TACO_OK) return st;
     sms = g_sm_count[dev];
   }
 
@@ -137,8 +151,9 @@ extern "C" taco_status paged_tree_attention_noalloc(
   float* part_lse = reinterpret_cast<float*>(base + kErrWordBytes + kCounterBytes);
   float* part_o = reinterpret_cast<float*>(base + kErrWordBytes + kCounterBytes + round_up(slots * rows * 4, 256));
 
-  // the counters of this call's units and the error word must start at zero
-  e = cudaMemsetAsync(base, 0, kErrWordBytes + static_cast<size_t>(units) * 4, static_cast<cudaStream_t>(stream));
+  // the counters of this call's units must start at zero; the error word keeps earlier calls' bits
+  // until taco_attn_check_noalloc reads it
+  e = cudaMemsetAsync(counters, 0, static_cast<size_t>(units) * 4, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaMemsetAsync(scratch): %s", cudaGetErrorString(e));
 
   // TMA descriptors of the two caches: rows of D elements, 64-column boxes of min(bs, 64) rows
@@ -192,7 +207,37 @@ extern "C" taco_status paged_tree_attention_noalloc(
   p.rows_per_unit = rows;
   p.row_groups = row_groups;
   p.tile_keys = taco::kTileKeys;
+  p.l2_prefetch_tiles = taco::kMmaPrefetchTiles;
   e = taco::launch_verify_mma(maps[0], maps[1], p, dtype, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "verify kernel launch: %s", cudaGetErrorString(e));
   return TACO_OK;
+}
+
+// Reads and clears the scratch's error word (see the rules at the top of this file).
+extern "C" taco_status taco_attn_check_noalloc(void* stream, uint32_t* bits_out) {
+  if (bits_out) *bits_out = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(TACO_ERR_UNSUPPORTED, "device index %d too large", dev);
+  e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  unsigned char* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    taco_status st = scratch_of(dev, &base);
+    if (st != TACO_OK) return st;
+  }
+  uint32_t bits = 0;
+  e = cudaMemcpy(&bits, base, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaMemcpy (noalloc error word): %s", cudaGetErrorString(e));
+  if (bits_out) *bits_out = bits;
+  if (bits == 0) return TACO_OK;
+  e = cudaMemset(base, 0, 4);
+  if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaMemset (noalloc error word): %s", cudaGetErrorString(e));
+  return fail(TACO_ERR_DEVICE_CHECK, "paged_tree_attention_noalloc device check failed: bits 0x%x%s%s%s%s", bits,
+              (bits & TACO_DEVERR_BLOCK_ID) ? " [block id out of range]" : "",
+              (bits & TACO_DEVERR_CONTEXT_LEN) ? " [context length out of range]" : "",
+              (bits & TACO_DEVERR_NUM_CAND) ? " [candidate count out of range]" : "",
+              (bits & TACO_DEVERR_WAIT_TIMEOUT) ? " [pipeline wait timed out]" : "");
 }

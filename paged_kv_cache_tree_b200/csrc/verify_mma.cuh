@@ -173,6 +173,11 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
     int64_t t = lo;
     int j = static_cast<int>((t - base_b) / Tb);
     int tile = static_cast<int>((t - base_b) % Tb);
+    // the V producer also asks L2 for both tensors of the tile pf_ahead tiles past its latest load
+    const int pf_ahead = is_k ? 0 : p.l2_prefetch_tiles;
+    TilePrefetcher<Cfg::kPanels, Cfg::kColsPerPanel> pf;
+    if (pf_ahead > 0) pf.init(p, b, base_b, lo, hi, Cfg::kStages);
+    int64_t kt = 0;  // tile ordinal within the CTA
     while (t < hi) {
       const int g = j / p.row_groups;
       const int tend = static_cast<int>(Tb < tile + (hi - t) ? Tb : tile + (hi - t));
@@ -216,6 +221,8 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
           for (int pn = 0; pn < Cfg::kPanels; ++pn) tma_load_2d(dst + pn * Cfg::kPanelBytes, tmap, fb, pn * Cfg::kColsPerPanel, row, policy);
         }
         __syncwarp();
+        ++kt;
+        if (go && pf_ahead > 0) pf.prefetch(p, kt + pf_ahead, &tmap_k, &tmap_v);
         if (++stage == Cfg::kStages) {
           stage = 0;
           phase ^= 1u;

@@ -163,6 +163,10 @@ __global__ void __launch_bounds__(352, 1)
     SegCursor cur;
     cur.init(p, sh->b, sh->base_b, lo, hi, true);
     int64_t k = 0;  // tile ordinal within the CTA
+    // the V producer also asks L2 for both tensors of the tile pf_ahead tiles past its latest load
+    const int pf_ahead = is_k ? 0 : p.l2_prefetch_tiles;
+    TilePrefetcher<Cfg::kPanels, 64> pf;
+    if (pf_ahead > 0) pf.init(p, sh->b, sh->base_b, lo, hi, SV);
     while (cur.valid()) {
       const int g = cur.j / p.row_groups;
       const int rg = cur.j % p.row_groups;
@@ -252,6 +256,7 @@ __global__ void __launch_bounds__(352, 1)
               tma_load_2d(dst + pn * Cfg::kPanelBytes, &tmap_v, smem_addr(&sh->v_full[st]), pn * 64, row, policy);
           }
           __syncwarp();
+          if (go && pf_ahead > 0) pf.prefetch(p, k + 1 + pf_ahead, &tmap_k, &tmap_v);
         }
       }
       cur.next_segment(p, true);

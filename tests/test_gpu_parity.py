@@ -197,3 +197,35 @@ def test_append_skips_negative_slots_and_touches_nothing_else():
     assert np.array_equal(wl.to_numpy_bits(d.v_cache.cpu()), rvc)
     changed = (d.k_cache.view(torch.int16) != before_k.view(torch.int16)).any(dim=-1).sum().item()
     assert changed <= (4 + 2) * 2
+
+
+def test_two_streams_overlap_without_sharing_a_workspace():
+    """Two verifies of different shapes, both with split units, enqueued on two streams with no order
+    between them: each (device, stream) pair has its own workspace and error word, so both results
+    match the oracle and each stream's error check sees only its own calls."""
+    specs = [dict(dtype="bf16", B=2, Hq=32, Hkv=8, D=128, bs=16, C=1, tree="chain", ctx=("uniform", 3000, 6000)),
+             dict(dtype="bf16", B=2, Hq=64, Hkv=8, D=128, bs=32, C=8, tree="forest", ctx=("uniform", 3000, 6000))]
+    ws = [wl.make_workload(s, seed=300 + k) for k, s in enumerate(specs)]
+    ds = [w.to("cuda") for w in ws]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [torch.full_like(d.q, float("nan")) for d in ds]
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for k in range(2):
+            taco.paged_tree_attention(ds[k].q, ds[k].k_cache, ds[k].v_cache, ds[k].block_tables, ds[k].context_lens,
+                                      ds[k].num_candidates, ds[k].tree_mask, ws[k].scale, out=outs[k],
+                                      stream=streams[k])
+    # a bad block id on stream 1 only: stream 0's word stays clean
+    bt = ds[1].block_tables.clone()
+    bt[0, 1] = ws[1].num_blocks + 3
+    bad_out = torch.empty_like(ds[1].q)
+    taco.paged_tree_attention(ds[1].q, ds[1].k_cache, ds[1].v_cache, bt, ds[1].context_lens, ds[1].num_candidates,
+                              ds[1].tree_mask, ws[1].scale, out=bad_out, stream=streams[1])
+    assert taco.check_device(streams[0]) == 0
+    with pytest.raises(taco.TacoError) as ei:
+        taco.check_device(streams[1])
+    assert "block id" in str(ei.value)
+    torch.cuda.synchronize()
+    for k in range(2):
+        want, _, _ = oracle_step(ws[k], append=False)
+        assert_parity(outs[k].cpu(), want, ws[k])

@@ -177,3 +177,36 @@ def test_device_errors_are_reported_not_faulted():
         taco.check_device()
     assert matched.cpu().tolist() == [0]
     assert taco.check_device() == 0
+
+
+def test_insert_wait_for_an_unpublished_slot_times_out_and_reports_it():
+    """A slot holding a block's key whose node was never published (a claim by a writer that never
+    finished) makes the inserting warp wait; the wait is bounded, so the call returns, reports
+    TACO_DEVERR_WAIT_TIMEOUT, inserts nothing past that block, and the next clean call is exact.
+    Nothing else runs in the kernel (no copy is in flight), so running out of the wait faults nothing."""
+    bs = 4
+    s = [7, 1, 7, 2, 5, 5, 3, 3]                             # two full blocks
+    tree = PrefixTree(bs)
+    cache = taco.PrefixCache(16, bs, 64)
+    got, cnt = cache.insert(flat([s]).cuda(), starts_of([s]).cuda(), torch.tensor([[3, 9]], dtype=torch.int32).cuda())
+    assert taco.check_device() == 0
+    assert got.cpu().tolist()[0][:2] == tree.insert(s, [3, 9]) == [3, 9]
+    # un-publish the first block's node: its slot keeps the key, its node index goes back to -1
+    keys, nodes = cache.slot_keys.cpu(), cache.slot_nodes.cpu()
+    first = [i for i in range(cache.capacity) if int(keys[i]) != 0 and int(nodes[i]) == 3]
+    assert len(first) == 1
+    cache.slot_nodes[first[0]] = -1
+    got, cnt = cache.insert(flat([s]).cuda(), starts_of([s]).cuda(), torch.tensor([[5, 6]], dtype=torch.int32).cuda())
+    with pytest.raises(taco.TacoError) as ei:
+        taco.check_device()
+    assert "wait timed out" in str(ei.value)
+    assert int(cnt[0]) == 0 and got.cpu().tolist() == [[-1, -1]]
+    assert taco.check_device() == 0                          # the word was cleared by the read above
+    # a clean cache afterwards behaves exactly like the oracle
+    cache = taco.PrefixCache(16, bs, 64)
+    tree = PrefixTree(bs)
+    for table in ([3, 9], [5, 6]):
+        got, cnt = cache.insert(flat([s]).cuda(), starts_of([s]).cuda(), torch.tensor([table], dtype=torch.int32).cuda())
+        assert taco.check_device() == 0
+        want = tree.insert(s, table)
+        assert got.cpu().tolist()[0][:len(want)] == want and int(cnt[0]) == len(want)
