@@ -8,9 +8,13 @@
 //               every 64-key tile's K chunks (warp 0) and V chunks (warp 10) reached through the block
 //               table, into separate K and V rings (K is released as soon as its Q K^T is done, V
 //               after its P V);
-//   warp 1      MMA issuer (one thread): S = Q K^T into one of four tensor-memory S buffers
-//               (64 fp32 columns each), up to three tiles ahead; O += P V with P read back from
-//               tensor memory (A operand) and V from shared memory (MN-major B operand);
+//   warp 1      Q K^T issuer (one thread): S = Q K^T into one of four tensor-memory S buffers
+//               (64 fp32 columns each), up to four tiles ahead of the P V issuer;
+//   warp 11     P V issuer (one thread): O += P V with P read back from tensor memory (A operand)
+//               and V from shared memory (MN-major B operand). Two issuing threads, each waiting
+//               only for its own inputs in tile order, because issuing one tcgen05.mma or commit
+//               costs a single thread tens of cycles and one thread doing both products plus the
+//               polling between them became the bound of the whole kernel;
 //   warps 2..9  two softmax warpgroups; tile k belongs to warpgroup k % 2, which owns its own O
 //               accumulator in tensor memory. Thread r of a warpgroup owns query row r (lane r):
 //               base-2 online softmax in fp32 whose reference max only moves when a row's max grows
@@ -31,7 +35,7 @@ constexpr int kTcTileKeys = 64;   // keys per work tile of this kernel (QK^T is 
 
 template <int D>
 struct TcCfg {
-  static constexpr int kThreads = 352;
+  static constexpr int kThreads = 384;
   static constexpr int kTK = kTcTileKeys;
   static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = kTK * 128;            // kTK keys x 128 bytes
@@ -49,8 +53,11 @@ struct TcCfg {
 };
 
 struct TcShared {
+  // k_empty[s]: Q K^T of the tile in K stage s is done (its K slot is free; with as many K stages as
+  // S buffers it also means the tile's S is ready). v_empty[s]: P V of the tile in V stage s is done
+  // (its V slot and its S buffer are free, and its warpgroup's O holds it).
   uint64_t k_full[8], k_empty[8], v_full[14], v_empty[14];
-  uint64_t q_full, q_empty, s_full[4], p_full[4], pv_done[4], o_free;
+  uint64_t q_full, q_empty, s_full[4], p_full[4], o_free;
   uint32_t tmem_base;
   int merge_flag, abort_flag;
   long long W, lo, hi, base_b;
@@ -70,7 +77,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const __grid_constant__ CUtensorMap tmap_q, const VerifyParams p) {
   using Cfg = TcCfg<D>;
@@ -109,7 +116,6 @@ __global__ void __launch_bounds__(352, 1)
     for (int j = 0; j < NS; ++j) {
       mbar_init(smem_addr(&sh->s_full[j]), 1);
       mbar_init(smem_addr(&sh->p_full[j]), 4);
-      mbar_init(smem_addr(&sh->pv_done[j]), 1);
     }
     mbar_init(smem_addr(&sh->o_free), 4);
     sh->merge_flag = 0;
@@ -145,6 +151,15 @@ __global__ void __launch_bounds__(352, 1)
   }
   const int64_t lo = sh->lo, hi = sh->hi;
   volatile int* abort_flag = &sh->abort_flag;
+  // barrier (and parity) that completes when S of tile k is in tensor memory
+  constexpr bool kMergedS = (SK == NS);
+  auto s_bar = [&](int64_t kk) -> uint32_t {
+    return kMergedS ? smem_addr(&sh->k_empty[kk % SK]) : smem_addr(&sh->s_full[kk % NS]);
+  };
+  auto s_par = [&](int64_t kk) -> uint32_t { return static_cast<uint32_t>((kk / (kMergedS ? SK : NS)) & 1); };
+  // barrier (and parity) that completes when P V of tile k is done
+  auto pv_bar = [&](int64_t kk) -> uint32_t { return smem_addr(&sh->v_empty[kk % SV]); };
+  auto pv_par = [&](int64_t kk) -> uint32_t { return static_cast<uint32_t>((kk / SV) & 1); };
   const int cpg = p.cands_per_group;
   const int qrows = cpg * p.G;
 
@@ -278,123 +293,97 @@ __global__ void __launch_bounds__(352, 1)
     return;
   }
 
-  if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    // One thread issues all tensor-core work: S = Q K^T up to kLookahead tiles ahead of the oldest
-    // tile whose P has not been consumed, and O += P V for that tile once its P is in tensor memory
-    // and its V has landed. S buffer (tile % 4) is reused only after the PV of the tile four earlier
-    // has completed. It suspends on barriers (short time hints) instead of spinning, since it shares
-    // its scheduler with two softmax warps.
-    constexpr int kLookahead = NS - 1;
+  if (warp == 1 || warp == 11) {
+    // ------------------------------------------------------------------ MMA issuers
+    // Warp 1 issues S = Q K^T, warp 11 issues O += P V, one thread each, tile by tile. Q K^T of tile
+    // k needs its K landed, its S buffer (k % NS) free (P V of tile k - NS done) and, on a segment's
+    // first tile, the segment's Q; P V of tile k needs its P written, its V landed and, on a
+    // segment's first tile, O released by the previous segment's epilogue. Every wait is bounded;
+    // a wait that gives up aborts the CTA and the issuer commits the rest of its barriers so that
+    // nobody waits on it.
     if (lane == 0) {
-      TileWalker wq, wp;
-      wq.init(p, sh->b, sh->base_b, lo, hi);
-      wp.init(p, sh->b, sh->base_b, lo, hi);
-      TileInfo tq, tp;
-      bool have_q = wq.next(p, tq);
-      bool have_p = wp.next(p, tp);
-      int64_t kq = 0, kp = 0;
+      const bool is_qk = (warp == 1);
+      TileWalker wk;
+      wk.init(p, sh->b, sh->base_b, lo, hi);
+      TileInfo ti;
+      bool have = wk.next(p, ti);
+      int64_t k = 0;
       // descriptor bases; every K step only adds a constant to the 14-bit start-address field
       const uint64_t q_desc = tc::smem_desc_sw128(smem_addr(qbuf), 16, 1024);
       const uint64_t k_desc = tc::smem_desc_sw128(smem_addr(kring), 16, 1024);
       const uint64_t v_desc = tc::smem_desc_sw128(smem_addr(vring), Cfg::kPanelBytes, 1024);
-      const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
       bool ok = true;
-      auto qk_ready = [&]() -> bool {
-        return mbar_test(smem_addr(&sh->k_full[kq % SK]), static_cast<uint32_t>((kq / SK) & 1)) &&
-               (kq < NS ||
-                mbar_test(smem_addr(&sh->pv_done[kq % NS]), static_cast<uint32_t>(((kq / NS) - 1) & 1))) &&
-               (!tq.first || mbar_test(smem_addr(&sh->q_full), static_cast<uint32_t>(tq.ui & 1)));
+      auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (*abort_flag != 0) return false;
+        return mbar_wait(bar, parity, p.error_word);
       };
-      auto issue_qk = [&]() {
-        tc::fence_after_sync();
-        const int kst = static_cast<int>(kq % SK);
-        const int sb = static_cast<int>(kq % NS);
-        const uint64_t kd = k_desc + static_cast<uint64_t>((kst * Cfg::kTensorBytes) >> 4);
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(sb * TK);
+      if (is_qk) {
+        for (; have; ++k, have = wk.next(p, ti)) {
+          const int kst = static_cast<int>(k % SK);
+          const int sb = static_cast<int>(k % NS);
+          ok = wait(smem_addr(&sh->k_full[kst]), static_cast<uint32_t>((k / SK) & 1)) &&
+               (k < NS || wait(pv_bar(k - NS), pv_par(k - NS))) &&
+               (!ti.first || wait(smem_addr(&sh->q_full), static_cast<uint32_t>(ti.ui & 1)));
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint64_t kd = k_desc + static_cast<uint64_t>((kst * Cfg::kTensorBytes) >> 4);
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>(sb * TK);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          // panel (ks / 4), then 16 elements = 32 bytes along the 128-byte swizzled row
-          const uint64_t qoff = static_cast<uint64_t>(((ks >> 2) * Cfg::kQPanelBytes + (ks & 3) * 32) >> 4);
-          const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kPanelBytes + (ks & 3) * 32) >> 4);
-          tc::mma_ss(d_tmem, q_desc + qoff, kd + koff, kIdescQK, ks > 0 ? 1u : 0u);
-        }
-        tc::commit(smem_addr(&sh->s_full[sb]));
-        tc::commit(smem_addr(&sh->k_empty[kst]));
-        if (tq.last) tc::commit(smem_addr(&sh->q_empty));
-        ++kq;
-        have_q = wq.next(p, tq);
-      };
-      auto pv_ready = [&]() -> bool {
-        return mbar_test(smem_addr(&sh->p_full[kp % NS]), static_cast<uint32_t>((kp / NS) & 1)) &&
-               mbar_test(smem_addr(&sh->v_full[kp % SV]), static_cast<uint32_t>((kp / SV) & 1)) &&
-               (!tp.first || tp.ui == 0 || mbar_test(smem_addr(&sh->o_free), static_cast<uint32_t>((tp.ui - 1) & 1)));
-      };
-      while (have_p && ok) {
-        // S = Q K^T for every tile that is ready, up to the lookahead; the tile whose P comes next
-        // must have its S before we wait for that P, so that one is waited for
-        while (have_q && kq <= kp + kLookahead) {
-          if (!qk_ready()) {
-            if (kq != kp) break;
-            while (ok && !qk_ready()) {
-              mbar_try_wait_hint(smem_addr(&sh->k_full[kq % SK]), static_cast<uint32_t>((kq / SK) & 1), 200);
-              ok = (*abort_flag == 0) && global_timer_ns() < deadline;
-            }
-            if (!ok) break;
+          for (int ks = 0; ks < D / 16; ++ks) {
+            // panel (ks / 4), then 16 elements = 32 bytes along the 128-byte swizzled row
+            const uint64_t qoff = static_cast<uint64_t>(((ks >> 2) * Cfg::kQPanelBytes + (ks & 3) * 32) >> 4);
+            const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kPanelBytes + (ks & 3) * 32) >> 4);
+            tc::mma_ss(d_tmem, q_desc + qoff, kd + koff, kIdescQK, ks > 0 ? 1u : 0u);
           }
-          issue_qk();
+          if constexpr (!kMergedS) tc::commit(smem_addr(&sh->s_full[sb]));
+          tc::commit(smem_addr(&sh->k_empty[kst]));
+          if (ti.last) tc::commit(smem_addr(&sh->q_empty));
         }
-        if (!ok) break;
-        // O += P V for tile kp: suspend on its P, issuing any S that becomes ready meanwhile
-        while (ok && !pv_ready()) {
-          mbar_try_wait_hint(smem_addr(&sh->p_full[kp % NS]), static_cast<uint32_t>((kp / NS) & 1), 200);
-          if (have_q && kq <= kp + kLookahead && qk_ready()) issue_qk();
-          ok = (*abort_flag == 0) && global_timer_ns() < deadline;
-        }
-        if (!ok) break;
-        tc::fence_after_sync();
-        const int sb = static_cast<int>(kp % NS);
-        const int vs = static_cast<int>(kp % SV);
-        const uint64_t vd = v_desc + static_cast<uint64_t>((vs * Cfg::kTensorBytes) >> 4);
-        const uint32_t a_tmem = tmem + static_cast<uint32_t>(sb * TK);
-        const uint32_t o_tmem = tmem + Cfg::kOCol + static_cast<uint32_t>((kp & 1) * 128);
-        const bool fresh = tp.jl < 2;  // first tile of this segment for its warpgroup
+      } else {
+        for (; have; ++k, have = wk.next(p, ti)) {
+          const int sb = static_cast<int>(k % NS);
+          const int vs = static_cast<int>(k % SV);
+          ok = wait(smem_addr(&sh->p_full[sb]), static_cast<uint32_t>((k / NS) & 1)) &&
+               wait(smem_addr(&sh->v_full[vs]), static_cast<uint32_t>((k / SV) & 1)) &&
+               (!ti.first || ti.ui == 0 || wait(smem_addr(&sh->o_free), static_cast<uint32_t>((ti.ui - 1) & 1)));
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint64_t vd = v_desc + static_cast<uint64_t>((vs * Cfg::kTensorBytes) >> 4);
+          const uint32_t a_tmem = tmem + static_cast<uint32_t>(sb * TK);
+          const uint32_t o_tmem = tmem + Cfg::kOCol + static_cast<uint32_t>((k & 1) * 128);
+          const bool fresh = ti.jl < 2;  // first tile of this segment for its warpgroup
 #pragma unroll
-        for (int ks = 0; ks < TK / 16; ++ks) {
-          // V as the MN-major B operand: 64-column panels kPanelBytes apart (LBO), 8-key groups 1024
-          // bytes apart (SBO); 16 keys per step = 2048 bytes; P: 16 keys = 8 packed columns
-          tc::mma_ts(o_tmem, a_tmem + ks * 8, vd + static_cast<uint64_t>((ks * 2048) >> 4), kIdescPV,
-                     (fresh && ks == 0) ? 0u : 1u);
+          for (int ks = 0; ks < TK / 16; ++ks) {
+            // V as the MN-major B operand: 64-column panels kPanelBytes apart (LBO), 8-key groups 1024
+            // bytes apart (SBO); 16 keys per step = 2048 bytes; P: 16 keys = 8 packed columns
+            tc::mma_ts(o_tmem, a_tmem + ks * 8, vd + static_cast<uint64_t>((ks * 2048) >> 4), kIdescPV,
+                       (fresh && ks == 0) ? 0u : 1u);
+          }
+          tc::commit(smem_addr(&sh->v_empty[vs]));
         }
-        tc::commit(smem_addr(&sh->v_empty[vs]));
-        tc::commit(smem_addr(&sh->pv_done[sb]));
-        ++kp;
-        have_p = wp.next(p, tp);
       }
       if (!ok) {
-        // gave up (2 s without finishing, or another role aborted): release everyone still waiting
+        // gave up (a wait ran out, or another role aborted): release everyone still waiting on us
         if (*abort_flag == 0) atomicOr(p.error_word, TACO_DEVERR_WAIT_TIMEOUT);
         *abort_flag = 1;
-        while (have_q) {
-          tc::commit(smem_addr(&sh->s_full[kq % NS]));
-          tc::commit(smem_addr(&sh->k_empty[kq % SK]));
-          if (tq.last) tc::commit(smem_addr(&sh->q_empty));
-          ++kq;
-          have_q = wq.next(p, tq);
-        }
-        while (have_p) {
-          tc::commit(smem_addr(&sh->v_empty[kp % SV]));
-          tc::commit(smem_addr(&sh->pv_done[kp % NS]));
-          ++kp;
-          have_p = wp.next(p, tp);
+        for (; have; ++k, have = wk.next(p, ti)) {
+          if (is_qk) {
+            if constexpr (!kMergedS) tc::commit(smem_addr(&sh->s_full[k % NS]));
+            tc::commit(smem_addr(&sh->k_empty[k % SK]));
+            if (ti.last) tc::commit(smem_addr(&sh->q_empty));
+          } else {
+            tc::commit(smem_addr(&sh->v_empty[k % SV]));
+          }
         }
       }
     }
     __syncwarp();
     tc::fence_before_sync();
-    named_bar_sync(2, 288);
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, Cfg::kTmemCols);
+    named_bar_sync(2, 320);
+    if (warp == 1) {
+      tc::fence_after_sync();
+      tc::tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
     return;
   }
 
@@ -434,7 +423,7 @@ __global__ void __launch_bounds__(352, 1)
       const int sb = static_cast<int>(k % NS);
       const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(sb * TK);
       bool ok = (*abort_flag == 0);
-      if (ok) ok = mbar_wait(smem_addr(&sh->s_full[sb]), static_cast<uint32_t>((k / NS) & 1), p.error_word);
+      if (ok) ok = mbar_wait(s_bar(k), s_par(k), p.error_word);
       if (!ok) *abort_flag = 1;
       tc::fence_after_sync();
       uint32_t sraw[2][32];
@@ -532,7 +521,7 @@ __global__ void __launch_bounds__(352, 1)
         const int64_t kprev = k_mine_last;
         bool okw = (*abort_flag == 0);
         if (okw)
-          okw = mbar_wait(smem_addr(&sh->pv_done[kprev % NS]), static_cast<uint32_t>((kprev / NS) & 1), p.error_word);
+          okw = mbar_wait(pv_bar(kprev), pv_par(kprev), p.error_word);
         if (!okw) *abort_flag = 1;
         tc::fence_after_sync();
 #pragma unroll 1
@@ -557,8 +546,7 @@ __global__ void __launch_bounds__(352, 1)
     if (k_mine_last >= 0) {
       bool ok = (*abort_flag == 0);
       if (ok)
-        ok = mbar_wait(smem_addr(&sh->pv_done[k_mine_last % NS]), static_cast<uint32_t>((k_mine_last / NS) & 1),
-                       p.error_word);
+        ok = mbar_wait(pv_bar(k_mine_last), pv_par(k_mine_last), p.error_word);
       if (!ok) *abort_flag = 1;
     }
     if (wg == 1) {
@@ -654,7 +642,7 @@ __global__ void __launch_bounds__(352, 1)
     cur.next_segment(p, false);
   }
   tc::fence_before_sync();
-  named_bar_sync(2, 288);
+  named_bar_sync(2, 320);
 }
 
 }  // namespace taco
