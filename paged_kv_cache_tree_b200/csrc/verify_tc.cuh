@@ -31,39 +31,50 @@
 
 namespace taco {
 
-constexpr int kTcTileKeys = 64;   // keys per work tile of this kernel (QK^T is M=128 x N=64)
+// Keys per work tile of this kernel: Q K^T is one M = 128 x N = 128 product per k step. A
+// tcgen05.mma with both operands in shared memory occupies the tensor core for about the same time
+// at N = 64 as at N = 128 (measured on B200: about 120 cycles either way), so 64-key products spent
+// half of the tensor core's time on nothing. Softmax warpgroup w takes keys [64 w, 64 w + 64) of
+// every tile.
+constexpr int kTcTileKeys = 128;
 
 template <int D>
 struct TcCfg {
   static constexpr int kThreads = 384;
   static constexpr int kTK = kTcTileKeys;
+  static constexpr int kHalf = kTK / 2;                    // keys per softmax warpgroup and tile
   static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = kTK * 128;            // kTK keys x 128 bytes
   static constexpr int kTensorBytes = kPanels * kPanelBytes;
-  static constexpr int kKStages = (D == 128) ? 4 : 8;
-  static constexpr int kVStages = (D == 128) ? 7 : 14;
+  static constexpr int kKStages = (D == 128) ? 3 : 6;
+  static constexpr int kVStages = (D == 128) ? 3 : 6;
   static constexpr int kQPanelBytes = 128 * 128;           // 128 rows x 128 bytes
   static constexpr int kQBytes = kPanels * kQPanelBytes;
-  static constexpr int kSBufs = 4;                         // S/P buffers of kTK columns at 0, 64, 128, 192
+  static constexpr int kSBufs = 2;                         // S/P buffers of kTK columns at 0, 128
   static constexpr int kTmemCols = 512;
   static constexpr int kOCol = 256;                        // O of warpgroup w at kOCol + w * 128
-  static constexpr int kSharedBytes = 4096;
+  static constexpr int kSharedBytes = 1536;
   static constexpr int kSmemBytes =
       1024 + (kKStages + kVStages) * kTensorBytes + kQBytes + kSharedBytes;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 struct TcShared {
   // k_empty[s]: Q K^T of the tile in K stage s is done (its K slot is free; with as many K stages as
   // S buffers it also means the tile's S is ready). v_empty[s]: P V of the tile in V stage s is done
   // (its V slot and its S buffer are free, and its warpgroup's O holds it).
-  uint64_t k_full[8], k_empty[8], v_full[14], v_empty[14];
-  uint64_t q_full, q_empty, s_full[4], p_full[4], o_free;
+  // p_full[2 sb + w]: warpgroup w wrote its half of P into S buffer sb.
+  uint64_t k_full[6], k_empty[6], v_full[6], v_empty[6];
+  uint64_t q_full, q_empty, s_full[2], p_full[4], o_free;
   uint32_t tmem_base;
   int merge_flag, abort_flag;
   long long W, lo, hi, base_b;
   int nC, b;
-  float xm[2][128];  // warpgroup 1's reference max per row, double-buffered by segment
-  float xl[2][128];  // warpgroup 1's running sum per row
+  // warpgroup 1's reference max and running sum per row at a segment's end. One buffer suffices:
+  // warpgroup 1 writes the next segment's values only after that segment's last P V, which waits
+  // for O to be released, which warpgroup 0 does after reading these.
+  float xm[128];
+  float xl[128];
 };
 
 // 3-D TMA tile load (Q tile: x = column, y = head, z = sequence * C + candidate).
@@ -87,6 +98,7 @@ __global__ void __launch_bounds__(384, 1)
   constexpr int NS = Cfg::kSBufs;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr int TK = Cfg::kTK;
+  constexpr int TH = Cfg::kHalf;
   constexpr uint32_t kIdescQK = tc::idesc_f16(kBf16 ? 1 : 0, 128, TK, 0);
   constexpr uint32_t kIdescPV = tc::idesc_f16(kBf16 ? 1 : 0, 128, D, 1);
   static_assert(sizeof(TcShared) <= Cfg::kSharedBytes, "shared bookkeeping too large");
@@ -113,10 +125,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(smem_addr(&sh->q_full), 1);
     mbar_init(smem_addr(&sh->q_empty), 1);
-    for (int j = 0; j < NS; ++j) {
-      mbar_init(smem_addr(&sh->s_full[j]), 1);
-      mbar_init(smem_addr(&sh->p_full[j]), 4);
-    }
+    for (int j = 0; j < NS; ++j) mbar_init(smem_addr(&sh->s_full[j]), 1);
+    for (int j = 0; j < 2 * NS; ++j) mbar_init(smem_addr(&sh->p_full[j]), 4);
     mbar_init(smem_addr(&sh->o_free), 4);
     sh->merge_flag = 0;
     sh->abort_flag = 0;
@@ -343,22 +353,27 @@ __global__ void __launch_bounds__(384, 1)
         for (; have; ++k, have = wk.next(p, ti)) {
           const int sb = static_cast<int>(k % NS);
           const int vs = static_cast<int>(k % SV);
-          ok = wait(smem_addr(&sh->p_full[sb]), static_cast<uint32_t>((k / NS) & 1)) &&
-               wait(smem_addr(&sh->v_full[vs]), static_cast<uint32_t>((k / SV) & 1)) &&
+          ok = wait(smem_addr(&sh->v_full[vs]), static_cast<uint32_t>((k / SV) & 1)) &&
                (!ti.first || ti.ui == 0 || wait(smem_addr(&sh->o_free), static_cast<uint32_t>((ti.ui - 1) & 1)));
           if (!ok) break;
-          tc::fence_after_sync();
-          const uint64_t vd = v_desc + static_cast<uint64_t>((vs * Cfg::kTensorBytes) >> 4);
-          const uint32_t a_tmem = tmem + static_cast<uint32_t>(sb * TK);
-          const uint32_t o_tmem = tmem + Cfg::kOCol + static_cast<uint32_t>((k & 1) * 128);
-          const bool fresh = ti.jl < 2;  // first tile of this segment for its warpgroup
+          // each warpgroup's half as soon as its P is written: O_w += P_w V[64 w, 64 w + 64)
+#pragma unroll 1
+          for (int w = 0; w < 2; ++w) {
+            ok = wait(smem_addr(&sh->p_full[2 * sb + w]), static_cast<uint32_t>((k / NS) & 1));
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint64_t vd = v_desc + static_cast<uint64_t>((vs * Cfg::kTensorBytes + w * TH * 128) >> 4);
+            const uint32_t a_tmem = tmem + static_cast<uint32_t>(sb * TK + w * TH);
+            const uint32_t o_tmem = tmem + Cfg::kOCol + static_cast<uint32_t>(w * 128);
 #pragma unroll
-          for (int ks = 0; ks < TK / 16; ++ks) {
-            // V as the MN-major B operand: 64-column panels kPanelBytes apart (LBO), 8-key groups 1024
-            // bytes apart (SBO); 16 keys per step = 2048 bytes; P: 16 keys = 8 packed columns
-            tc::mma_ts(o_tmem, a_tmem + ks * 8, vd + static_cast<uint64_t>((ks * 2048) >> 4), kIdescPV,
-                       (fresh && ks == 0) ? 0u : 1u);
+            for (int ks = 0; ks < TH / 16; ++ks) {
+              // V as the MN-major B operand: 64-column panels kPanelBytes apart (LBO), 8-key groups
+              // 1024 bytes apart (SBO); 16 keys per step = 2048 bytes; P: 16 keys = 8 packed columns
+              tc::mma_ts(o_tmem, a_tmem + ks * 8, vd + static_cast<uint64_t>((ks * 2048) >> 4), kIdescPV,
+                         (ti.first && ks == 0) ? 0u : 1u);
+            }
           }
+          if (!ok) break;
           tc::commit(smem_addr(&sh->v_empty[vs]));
         }
       }
@@ -418,10 +433,9 @@ __global__ void __launch_bounds__(384, 1)
     float l_run = 0.f;
     int64_t k_mine_last = -1;
     for (int tl = tbegin; tl < tend; ++tl, ++k) {
-      if (static_cast<int>(k & 1) != wg) continue;
-      const int key0 = tl * TK;
+      const int key0 = tl * TK + wg * TH;   // this warpgroup's half of the tile
       const int sb = static_cast<int>(k % NS);
-      const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(sb * TK);
+      const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(sb * TK + wg * TH);
       bool ok = (*abort_flag == 0);
       if (ok) ok = mbar_wait(s_bar(k), s_par(k), p.error_word);
       if (!ok) *abort_flag = 1;
@@ -429,8 +443,8 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t sraw[2][32];
       tc::ld_32x32b_x32(s_col, sraw[0]);
       tc::ld_32x32b_x32(s_col + 32, sraw[1]);
-      if (key0 + TK > L) {
-        // keys >= L in this tile: their V rows may be stale or NaN-poisoned; zero them once V landed
+      if (key0 + TH > L) {
+        // keys >= L in this half: their V rows may be stale or NaN-poisoned; zero them once V landed
         const int vs = static_cast<int>(k % SV);
         bool okv = (*abort_flag == 0);
         if (okv) okv = mbar_wait(smem_addr(&sh->v_full[vs]), static_cast<uint32_t>((k / SV) & 1), p.error_word);
@@ -439,8 +453,8 @@ __global__ void __launch_bounds__(384, 1)
         if (z0 < 0) z0 = 0;
         uint8_t* vgen = vring + vs * Cfg::kTensorBytes;
         const int per_row = Cfg::kPanels * 8;
-        for (int idx = r; idx < (TK - z0) * per_row; idx += 128) {
-          const int row = z0 + idx / per_row;
+        for (int idx = r; idx < (TH - z0) * per_row; idx += 128) {
+          const int row = wg * TH + z0 + idx / per_row;
           const int rem = idx % per_row;
           *reinterpret_cast<uint4*>(vgen + (rem / 8) * Cfg::kPanelBytes + row * 128 + (rem % 8) * 16) =
               make_uint4(0u, 0u, 0u, 0u);
@@ -448,10 +462,10 @@ __global__ void __launch_bounds__(384, 1)
         fence_proxy_async_smem();
       }
       tc::wait_ld();
-      static_assert(TK == 64, "the softmax below holds one 64-column tile per thread");
+      static_assert(TH == 64, "the softmax below holds one 64-column half tile per thread");
       // Row max of the raw scores (a positive scale_log2 commutes with max; otherwise the scaled
       // values are used). Masked keys become -inf; only the tiles that reach the candidates mask.
-      const bool need_mask = key0 + TK > P;
+      const bool need_mask = key0 + TH > P;
       const bool pos_scale = p.scale_log2 > 0.f;
       float v[64];
 #pragma unroll
@@ -537,7 +551,7 @@ __global__ void __launch_bounds__(384, 1)
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&sh->p_full[sb]));
+      if (lane == 0) mbar_arrive(smem_addr(&sh->p_full[2 * sb + wg]));
       k_mine_last = k;
     }
 
@@ -550,15 +564,15 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) *abort_flag = 1;
     }
     if (wg == 1) {
-      sh->xm[cur.ui & 1][r] = k_mine_last >= 0 ? m_ref : -INFINITY;
-      sh->xl[cur.ui & 1][r] = k_mine_last >= 0 ? l_run : 0.f;
+      sh->xm[r] = k_mine_last >= 0 ? m_ref : -INFINITY;
+      sh->xl[r] = k_mine_last >= 0 ? l_run : 0.f;
       tc::fence_before_sync();
       named_bar_sync(3, 256);
     } else {
       named_bar_sync(3, 256);
       tc::fence_after_sync();
-      const float m1 = sh->xm[cur.ui & 1][r];
-      const float l1 = sh->xl[cur.ui & 1][r];
+      const float m1 = sh->xm[r];
+      const float l1 = sh->xl[r];
       const float m0 = k_mine_last >= 0 ? m_ref : -INFINITY;
       const float l0 = k_mine_last >= 0 ? l_run : 0.f;
       const float M = fmaxf(m0, m1);
