@@ -70,11 +70,10 @@ struct TcShared {
   int merge_flag, abort_flag;
   long long W, lo, hi, base_b;
   int nC, b;
-  // warpgroup 1's reference max and running sum per row at a segment's end. One buffer suffices:
-  // warpgroup 1 writes the next segment's values only after that segment's last P V, which waits
-  // for O to be released, which warpgroup 0 does after reading these.
-  float xm[128];
-  float xl[128];
+  // per-row values the two softmax warpgroups exchange at a segment's end (log-sum-exp, then scale);
+  // the next segment's exchange comes after that segment's last P V, which waits for O to be
+  // released, which both warpgroups do only after their reads here.
+  float xs[2][128];
 };
 
 // 3-D TMA tile load (Q tile: x = column, y = head, z = sequence * C + candidate).
@@ -85,6 +84,63 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+// Combines the split-KV partials of one unit for row r, head dims [w D/2, (w + 1) D/2): one thread per
+// (row, half), pieces s = 0 .. c_last - c_first in CTA order (slots as in merge_split_unit):
+//   out = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s,
+// pieces with lse = -inf (no visible key) weigh 0. Two pieces at a time, every load of a 32-column
+// chunk issued before any is used.
+template <typename T, int D>
+__device__ __forceinline__ void merge_split_row_half(const VerifyParams& p, int r, int w, int c_first, int c_last,
+                                                     bool first_odd, T* dst, bool active) {
+  constexpr int H = D / 2;
+  const int nsl = c_last - c_first + 1;
+  auto slot_of = [&](int s) -> int64_t {
+    const int c = c_first + s;
+    return (s == 0 && first_odd) ? 2 * c + 1 : 2 * c;
+  };
+  float M = -INFINITY;
+  for (int s = 0; s < nsl; ++s) M = fmaxf(M, __ldcg(p.part_lse + slot_of(s) * 128 + r));
+#pragma unroll 1
+  for (int c0 = 0; c0 < H; c0 += 32) {
+    float acc[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+    float l = 0.f;
+    for (int s0 = 0; s0 < nsl; s0 += 2) {
+      float wt[2];
+      float4 v[2][8];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const bool have = s0 + j < nsl;
+        const int64_t sl = have ? slot_of(s0 + j) : 0;
+        const float ls = have ? __ldcg(p.part_lse + sl * 128 + r) : -INFINITY;
+        wt[j] = (ls == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ls - M);
+        const float4* src = reinterpret_cast<const float4*>(p.part_o + (sl * 128 + r) * D + w * H + c0);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[j][e] = wt[j] > 0.f ? __ldcg(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        l += wt[j];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          acc[4 * e] = fmaf(wt[j], v[j][e].x, acc[4 * e]);
+          acc[4 * e + 1] = fmaf(wt[j], v[j][e].y, acc[4 * e + 1]);
+          acc[4 * e + 2] = fmaf(wt[j], v[j][e].z, acc[4 * e + 2]);
+          acc[4 * e + 3] = fmaf(wt[j], v[j][e].w, acc[4 * e + 3]);
+        }
+      }
+    }
+    const float inv = (active && l > 0.f) ? 1.f / l : 0.f;
+    uint32_t wv[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) wv[e] = active ? MmaOp<T>::pack(acc[2 * e] * inv, acc[2 * e + 1] * inv) : 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      *reinterpret_cast<uint4*>(dst + w * H + c0 + e * 8) = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+  }
 }
 
 template <typename T, int D>
@@ -127,7 +183,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(smem_addr(&sh->q_empty), 1);
     for (int j = 0; j < NS; ++j) mbar_init(smem_addr(&sh->s_full[j]), 1);
     for (int j = 0; j < 2 * NS; ++j) mbar_init(smem_addr(&sh->p_full[j]), 4);
-    mbar_init(smem_addr(&sh->o_free), 4);
+    mbar_init(smem_addr(&sh->o_free), 8);
     sh->merge_flag = 0;
     sh->abort_flag = 0;
     fence_mbar_init();
@@ -556,101 +612,94 @@ __global__ void __launch_bounds__(384, 1)
     }
 
     // ---------------------------------------------------------------- segment epilogue
-    // wait for this warpgroup's last PV (each S buffer has its own completion barrier)
+    // Both warpgroups finish the segment together, each on half of the head dims of both O
+    // accumulators: O = s_0 O_0 + s_1 O_1 with s_w = 2^(m_w - LSE) and LSE = log2(l_0 2^m_0 + l_1 2^m_1)
+    // (the base-2 log-sum-exp of the segment; m_w, l_w are warpgroup w's reference max and sum).
+    // Each warpgroup publishes its own log-sum-exp, then its scale, through shared memory.
     if (k_mine_last >= 0) {
       bool ok = (*abort_flag == 0);
-      if (ok)
-        ok = mbar_wait(pv_bar(k_mine_last), pv_par(k_mine_last), p.error_word);
+      if (ok) ok = mbar_wait(pv_bar(k_mine_last), pv_par(k_mine_last), p.error_word);
       if (!ok) *abort_flag = 1;
     }
-    if (wg == 1) {
-      sh->xm[r] = k_mine_last >= 0 ? m_ref : -INFINITY;
-      sh->xl[r] = k_mine_last >= 0 ? l_run : 0.f;
-      tc::fence_before_sync();
-      named_bar_sync(3, 256);
-    } else {
-      named_bar_sync(3, 256);
-      tc::fence_after_sync();
-      const float m1 = sh->xm[r];
-      const float l1 = sh->xl[r];
-      const float m0 = k_mine_last >= 0 ? m_ref : -INFINITY;
-      const float l0 = k_mine_last >= 0 ? l_run : 0.f;
-      const float M = fmaxf(m0, m1);
-      const float f0 = l0 > 0.f ? fast_exp2(m0 - M) : 0.f;
-      const float f1 = l1 > 0.f ? fast_exp2(m1 - M) : 0.f;
-      const float ltot = f0 * l0 + f1 * l1;
-      const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-      const float w0 = f0 * inv, w1 = f1 * inv;
-      const bool use0 = f0 > 0.f, use1 = f1 > 0.f;
-      const bool whole_unit = (tbegin == 0 && tend == Tb);
-      const int slot = 2 * static_cast<int>(blockIdx.x) + (first_segment ? 0 : 1);
-      T* dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D;
-      float* pdst = p.part_o + (static_cast<int64_t>(slot) * 128 + r) * D;
-      const uint32_t o0 = tmem + lane_base + Cfg::kOCol;
-      const uint32_t o1 = o0 + 128;
+    const bool have_keys = k_mine_last >= 0 && l_run > 0.f;
+    const float lse_mine = have_keys ? m_ref + __log2f(l_run) : -INFINITY;
+    sh->xs[wg][r] = lse_mine;
+    named_bar_sync(3, 256);
+    const float lse_other = sh->xs[wg ^ 1][r];
+    const float lmax = fmaxf(lse_mine, lse_other);
+    const float LSE =
+        lmax == -INFINITY ? -INFINITY : lmax + __log2f(fast_exp2(lse_mine - lmax) + fast_exp2(lse_other - lmax));
+    const float s_mine = have_keys ? fast_exp2(m_ref - LSE) : 0.f;
+    named_bar_sync(3, 256);
+    sh->xs[wg][r] = s_mine;
+    named_bar_sync(3, 256);
+    const float s_other = sh->xs[wg ^ 1][r];
+    const float s0 = wg == 0 ? s_mine : s_other;
+    const float s1 = wg == 0 ? s_other : s_mine;
+    const bool use0 = s0 > 0.f, use1 = s1 > 0.f;
+    tc::fence_after_sync();
+    const bool whole_unit = (tbegin == 0 && tend == Tb);
+    const int slot = 2 * static_cast<int>(blockIdx.x) + (first_segment ? 0 : 1);
+    T* dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D;
+    float* pdst = p.part_o + (static_cast<int64_t>(slot) * 128 + r) * D;
+    const uint32_t o0 = tmem + lane_base + Cfg::kOCol;
+    const uint32_t o1 = o0 + 128;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t a[32], bb[32];
-        tc::ld_32x32b_x32(o0 + c * 32, a);
-        tc::ld_32x32b_x32(o1 + c * 32, bb);
-        tc::wait_ld();
-        float x[32];
+    for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
+      uint32_t a[32], bb[32];
+      tc::ld_32x32b_x32(o0 + c * 32, a);
+      tc::ld_32x32b_x32(o1 + c * 32, bb);
+      tc::wait_ld();
+      float x[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          x[e] = (use0 ? w0 * __uint_as_float(a[e]) : 0.f) + (use1 ? w1 * __uint_as_float(bb[e]) : 0.f);
-        if (whole_unit) {
-          if (row_real) {
-            uint32_t wv[16];
+      for (int e = 0; e < 32; ++e)
+        x[e] = (use0 ? s0 * __uint_as_float(a[e]) : 0.f) + (use1 ? s1 * __uint_as_float(bb[e]) : 0.f);
+      if (whole_unit) {
+        if (row_real) {
+          uint32_t wv[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) wv[e] = active ? Op::pack(x[2 * e], x[2 * e + 1]) : 0u;
+          for (int e = 0; e < 16; ++e) wv[e] = active ? Op::pack(x[2 * e], x[2 * e + 1]) : 0u;
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              *reinterpret_cast<uint4*>(dst + c * 32 + e * 8) =
-                  make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            __stcg(reinterpret_cast<float4*>(pdst + c * 32 + e * 4),
-                   make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]));
+          for (int e = 0; e < 4; ++e)
+            *reinterpret_cast<uint4*>(dst + c * 32 + e * 8) =
+                make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
         }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          __stcg(reinterpret_cast<float4*>(pdst + c * 32 + e * 4),
+                 make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]));
       }
-      if (!whole_unit)
-        __stcg(p.part_lse + static_cast<int64_t>(slot) * 128 + r, ltot > 0.f ? M + __log2f(ltot) : -INFINITY);
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&sh->o_free));
+    }
+    if (!whole_unit && wg == 0) __stcg(p.part_lse + static_cast<int64_t>(slot) * 128 + r, LSE);
+    tc::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sh->o_free));
 
-      if (!whole_unit) {
-        __threadfence();
-        named_bar_sync(1, 128);
-        const int64_t unit_base = cur.unit_base();
-        const int c_first = cta_of_tile(unit_base, W, nC);
-        const int c_last = cta_of_tile(unit_base + Tb - 1, W, nC);
-        const int u = (b * p.Hkv + g) * p.row_groups + rg;
-        if (warp == 2 && lane == 0) {
-          const uint32_t prev = atomicAdd(p.counters + u, 1u);
-          const bool last = prev == static_cast<uint32_t>(c_last - c_first);
-          if (last) {
-            p.counters[u] = 0u;
-            __threadfence();
-          }
-          sh->merge_flag = last ? 1 : 0;
+    if (!whole_unit) {
+      // the CTA that arrives last on the unit's counter combines every piece's partial
+      __threadfence();
+      named_bar_sync(1, 256);
+      const int64_t unit_base = cur.unit_base();
+      const int c_first = cta_of_tile(unit_base, W, nC);
+      const int c_last = cta_of_tile(unit_base + Tb - 1, W, nC);
+      const int u = (b * p.Hkv + g) * p.row_groups + rg;
+      if (warp == 2 && lane == 0) {
+        const uint32_t prev = atomicAdd(p.counters + u, 1u);
+        const bool last = prev == static_cast<uint32_t>(c_last - c_first);
+        if (last) {
+          p.counters[u] = 0u;
+          __threadfence();
         }
-        named_bar_sync(1, 128);
-        if (sh->merge_flag) {
-          const int64_t lo_first = static_cast<int64_t>(c_first) * W / nC;
-          const int64_t row0 = static_cast<int64_t>(b) * p.C;
-          merge_split_unit<T, D>(p, qrows, 128, c_first, c_last, lo_first < unit_base, warp - 2, lane,
-                                 [&](int rr) -> MergeRow<T> {
-                                   const int ii = rg * cpg + rr / p.G;
-                                   if (ii >= p.C) return MergeRow<T>{nullptr, false};
-                                   T* d = static_cast<T*>(p.out) + ((row0 + ii) * p.Hq + g * p.G + rr % p.G) * D;
-                                   return MergeRow<T>{d, ii < n};
-                                 });
-        }
-        named_bar_sync(1, 128);
+        sh->merge_flag = last ? 1 : 0;
       }
+      named_bar_sync(1, 256);
+      if (sh->merge_flag) {
+        const int64_t lo_first = static_cast<int64_t>(c_first) * W / nC;
+        if (row_real)
+          merge_split_row_half<T, D>(p, r, wg, c_first, c_last, lo_first < unit_base, dst, active);
+      }
+      named_bar_sync(1, 256);
     }
     first_segment = false;
     cur.next_segment(p, false);
