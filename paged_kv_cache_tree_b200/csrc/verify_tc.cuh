@@ -86,11 +86,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Combines the split-KV partials of one unit for row r, head dims [w D/2, (w + 1) D/2): one thread per
-// (row, half), pieces s = 0 .. c_last - c_first in CTA order (slots as in merge_split_unit):
+// Split-KV partials of this kernel are stored transposed, [slot][head dim][128 rows] fp32, so that the
+// 32 row-threads of a warp store and load one contiguous 128-byte line per instruction (a row-major
+// layout made every warp instruction touch 32 lines, and the merge and epilogue ran at a fraction of
+// L2's request rate).
+//
+// Combines the partials of one unit for row r, head dims [w D/2, (w + 1) D/2): one thread per
+// (row, half), pieces s = 0 .. c_last - c_first in CTA order (slot of piece 0 is 2 c_first + 1 when it
+// is not c_first's first segment, every other piece's is 2 c):
 //   out = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s,
-// pieces with lse = -inf (no visible key) weigh 0. Two pieces at a time, every load of a 32-column
-// chunk issued before any is used.
+// pieces with lse = -inf (no visible key) weigh 0. The pieces' log-sum-exp and a 32-column chunk of
+// two pieces are loaded together (unconditionally; a zero weight then selects 0); further pieces are
+// folded in pairs with an online rescale.
 template <typename T, int D>
 __device__ __forceinline__ void merge_split_row_half(const VerifyParams& p, int r, int w, int c_first, int c_last,
                                                      bool first_odd, T* dst, bool active) {
@@ -100,38 +107,40 @@ __device__ __forceinline__ void merge_split_row_half(const VerifyParams& p, int 
     const int c = c_first + s;
     return (s == 0 && first_odd) ? 2 * c + 1 : 2 * c;
   };
-  float M = -INFINITY;
-  for (int s = 0; s < nsl; ++s) M = fmaxf(M, __ldcg(p.part_lse + slot_of(s) * 128 + r));
 #pragma unroll 1
   for (int c0 = 0; c0 < H; c0 += 32) {
     float acc[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) acc[e] = 0.f;
-    float l = 0.f;
+    float M = -INFINITY, l = 0.f;
     for (int s0 = 0; s0 < nsl; s0 += 2) {
-      float wt[2];
-      float4 v[2][8];
+      float ls[2];
+      float v[2][32];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const bool have = s0 + j < nsl;
-        const int64_t sl = have ? slot_of(s0 + j) : 0;
-        const float ls = have ? __ldcg(p.part_lse + sl * 128 + r) : -INFINITY;
-        wt[j] = (ls == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ls - M);
-        const float4* src = reinterpret_cast<const float4*>(p.part_o + (sl * 128 + r) * D + w * H + c0);
+        const int64_t sl = slot_of(have ? s0 + j : s0);
+        ls[j] = __ldcg(p.part_lse + sl * 128 + r);
+        const float* src = p.part_o + (sl * D + w * H + c0) * 128 + r;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[j][e] = wt[j] > 0.f ? __ldcg(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e = 0; e < 32; ++e) v[j][e] = __ldcg(src + e * 128);
+        if (!have) ls[j] = -INFINITY;
       }
+      const float mn = fmaxf(M, fmaxf(ls[0], ls[1]));
+      if (mn == -INFINITY) continue;
+      const float f = M == -INFINITY ? 0.f : exp2f(M - mn);
+      float wt[2];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        l += wt[j];
+      for (int j = 0; j < 2; ++j) wt[j] = ls[j] == -INFINITY ? 0.f : exp2f(ls[j] - mn);
+      l = l * f + wt[0] + wt[1];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          acc[4 * e] = fmaf(wt[j], v[j][e].x, acc[4 * e]);
-          acc[4 * e + 1] = fmaf(wt[j], v[j][e].y, acc[4 * e + 1]);
-          acc[4 * e + 2] = fmaf(wt[j], v[j][e].z, acc[4 * e + 2]);
-          acc[4 * e + 3] = fmaf(wt[j], v[j][e].w, acc[4 * e + 3]);
-        }
+      for (int e = 0; e < 32; ++e) {
+        float t = acc[e] * f;
+        if (wt[0] > 0.f) t = fmaf(wt[0], v[0][e], t);
+        if (wt[1] > 0.f) t = fmaf(wt[1], v[1][e], t);
+        acc[e] = t;
       }
+      M = mn;
     }
     const float inv = (active && l > 0.f) ? 1.f / l : 0.f;
     uint32_t wv[16];
@@ -641,7 +650,7 @@ __global__ void __launch_bounds__(384, 1)
     const bool whole_unit = (tbegin == 0 && tend == Tb);
     const int slot = 2 * static_cast<int>(blockIdx.x) + (first_segment ? 0 : 1);
     T* dst = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * p.C + i) * p.Hq + g * p.G + hh) * D;
-    float* pdst = p.part_o + (static_cast<int64_t>(slot) * 128 + r) * D;
+    float* pdst = p.part_o + static_cast<int64_t>(slot) * D * 128 + r;  // transposed: [D][128] per slot
     const uint32_t o0 = tmem + lane_base + Cfg::kOCol;
     const uint32_t o1 = o0 + 128;
 #pragma unroll 1
@@ -666,9 +675,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          __stcg(reinterpret_cast<float4*>(pdst + c * 32 + e * 4),
-                 make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]));
+        for (int e = 0; e < 32; ++e) __stcg(pdst + (c * 32 + e) * 128, x[e]);
       }
     }
     if (!whole_unit && wg == 0) __stcg(p.part_lse + static_cast<int64_t>(slot) * 128 + r, LSE);
