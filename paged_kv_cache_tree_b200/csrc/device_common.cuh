@@ -265,8 +265,7 @@ struct MmaOp<__half> {
 // last on the unit's counter combines them. Since each CTA's range is contiguous, only its first
 // and last piece can be partial, so CTA c owns two partial slots: 2c (its first piece) and 2c+1.
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ int clamp_context(const VerifyParams& p, int b, bool report) {
-  int L = __ldg(p.context_lens + b);
+__device__ __forceinline__ int clamp_context_value(const VerifyParams& p, int L, bool report) {
   const int cap = p.max_blocks * p.bs;
   if (L < 0 || L > cap) {
     if (report) atomicOr(p.error_word, TACO_DEVERR_CONTEXT_LEN);
@@ -275,14 +274,21 @@ __device__ __forceinline__ int clamp_context(const VerifyParams& p, int b, bool 
   return L;
 }
 
-__device__ __forceinline__ int clamp_candidates(const VerifyParams& p, int b, int L, bool report) {
-  int n = __ldg(p.num_candidates + b);
+__device__ __forceinline__ int clamp_context(const VerifyParams& p, int b, bool report) {
+  return clamp_context_value(p, __ldg(p.context_lens + b), report);
+}
+
+__device__ __forceinline__ int clamp_candidates_value(const VerifyParams& p, int n, int L, bool report) {
   const int cap = L < p.C ? L : p.C;
   if (n < 0 || n > cap) {
     if (report) atomicOr(p.error_word, TACO_DEVERR_NUM_CAND);
     n = n < 0 ? 0 : cap;
   }
   return n;
+}
+
+__device__ __forceinline__ int clamp_candidates(const VerifyParams& p, int b, int L, bool report) {
+  return clamp_candidates_value(p, __ldg(p.num_candidates + b), L, report);
 }
 
 __device__ __forceinline__ int tiles_of(int L, int tile) { return L <= 0 ? 1 : (L + tile - 1) / tile; }
@@ -454,11 +460,13 @@ __device__ __forceinline__ void merge_split_unit(const VerifyParams& p, int rows
 }
 
 // Walks one CTA's work as segments: a segment is the part of one unit (b, j = g * RG + rg) that
-// falls into the CTA's tile range; tiles [tile, seg_end()) of the unit.
+// falls into the CTA's tile range; tiles [tile, seg_end()) of the unit. The next sequence's context
+// length is loaded one sequence ahead, so that moving on does not wait for it.
 struct SegCursor {
   int b;
   int64_t base_b;  // first global tile of sequence b's units
   int L, Tb, j, tile;
+  int L_next_raw;  // context_lens[b + 1] as loaded (0 past the batch)
   int64_t t, hi;
   int HR;
   int ui;          // segment ordinal within the CTA
@@ -469,6 +477,7 @@ struct SegCursor {
     base_b = base_b0;
     HR = p.Hkv * p.row_groups;
     L = clamp_context(p, b, report);
+    L_next_raw = b + 1 < p.B ? __ldg(p.context_lens + b + 1) : 0;
     Tb = tiles_of(L, p.tile_keys);
     t = lo;
     hi = hi_;
@@ -489,7 +498,8 @@ struct SegCursor {
       j = 0;
       base_b += static_cast<int64_t>(Tb) * HR;
       if (++b < p.B) {
-        L = clamp_context(p, b, report);
+        L = clamp_context_value(p, L_next_raw, report);
+        L_next_raw = b + 1 < p.B ? __ldg(p.context_lens + b + 1) : 0;
         Tb = tiles_of(L, p.tile_keys);
       }
     }

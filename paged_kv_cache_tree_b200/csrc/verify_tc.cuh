@@ -477,6 +477,20 @@ __global__ void __launch_bounds__(384, 1)
   cur.init(p, sh->b, sh->base_b, lo, hi, false);
   int64_t k = 0;
   bool first_segment = true;
+  // a segment's candidate count and this row's mask word, as loaded (the next segment's are loaded
+  // at the start of the current one, so that a segment switch does not wait for them)
+  auto load_seg_inputs = [&](int bb, int jj, int& n_raw, uint32_t& mw_raw) {
+    n_raw = 0;
+    mw_raw = 0u;
+    if (bb < p.B) {
+      n_raw = __ldg(p.num_candidates + bb);
+      const int ii = (jj % p.row_groups) * cpg + r / p.G;
+      if (r < qrows && ii < p.C) mw_raw = __ldg(p.tree_mask_bits + static_cast<int64_t>(bb) * p.C + ii);
+    }
+  };
+  int n_raw_cur;
+  uint32_t mw_raw_cur;
+  load_seg_inputs(cur.b, cur.j, n_raw_cur, mw_raw_cur);
   while (cur.valid()) {
     const int b = cur.b;
     const int g = cur.j / p.row_groups;
@@ -485,14 +499,18 @@ __global__ void __launch_bounds__(384, 1)
     const int tbegin = cur.tile;
     const int tend = cur.seg_end();
     const int Tb = cur.Tb;
-    const int n = clamp_candidates(p, b, L, false);
+    const int n = clamp_candidates_value(p, n_raw_cur, L, false);
     const int P = L - n;
     const uint32_t nmask = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
     const int i = rg * cpg + r / p.G;            // candidate of this row
     const int hh = r % p.G;
     const bool row_real = r < qrows && i < p.C;  // a row of the output
     const bool active = row_real && i < n;       // a row with a query
-    const uint32_t mw = active ? (__ldg(p.tree_mask_bits + static_cast<int64_t>(b) * p.C + i) & nmask) : 0u;
+    const uint32_t mw = active ? (mw_raw_cur & nmask) : 0u;
+    {
+      const bool same_b = cur.j + 1 < cur.HR;
+      load_seg_inputs(same_b ? b : b + 1, same_b ? cur.j + 1 : 0, n_raw_cur, mw_raw_cur);
+    }
 
     float m_ref = -INFINITY;
     float l_run = 0.f;
@@ -508,24 +526,6 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t sraw[2][32];
       tc::ld_32x32b_x32(s_col, sraw[0]);
       tc::ld_32x32b_x32(s_col + 32, sraw[1]);
-      if (key0 + TH > L) {
-        // keys >= L in this half: their V rows may be stale or NaN-poisoned; zero them once V landed
-        const int vs = static_cast<int>(k % SV);
-        bool okv = (*abort_flag == 0);
-        if (okv) okv = mbar_wait(smem_addr(&sh->v_full[vs]), static_cast<uint32_t>((k / SV) & 1), p.error_word);
-        if (!okv) *abort_flag = 1;
-        int z0 = L - key0;
-        if (z0 < 0) z0 = 0;
-        uint8_t* vgen = vring + vs * Cfg::kTensorBytes;
-        const int per_row = Cfg::kPanels * 8;
-        for (int idx = r; idx < (TH - z0) * per_row; idx += 128) {
-          const int row = wg * TH + z0 + idx / per_row;
-          const int rem = idx % per_row;
-          *reinterpret_cast<uint4*>(vgen + (rem / 8) * Cfg::kPanelBytes + row * 128 + (rem % 8) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
-      }
       tc::wait_ld();
       static_assert(TH == 64, "the softmax below holds one 64-column half tile per thread");
       // Row max of the raw scores (a positive scale_log2 commutes with max; otherwise the scaled
@@ -595,6 +595,26 @@ __global__ void __launch_bounds__(384, 1)
         l_run += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
       }
       tc::st_32x32b_x32(s_col, pk);
+      if (key0 + TH > L) {
+        // keys >= L in this half: their V rows may be stale or NaN-poisoned; zero them once V has
+        // landed (after P is written, so that the wait for V overlaps the softmax above; P V reads
+        // them only after this warpgroup's p_full arrival below)
+        const int vs = static_cast<int>(k % SV);
+        bool okv = (*abort_flag == 0);
+        if (okv) okv = mbar_wait(smem_addr(&sh->v_full[vs]), static_cast<uint32_t>((k / SV) & 1), p.error_word);
+        if (!okv) *abort_flag = 1;
+        int z0 = L - key0;
+        if (z0 < 0) z0 = 0;
+        uint8_t* vgen = vring + vs * Cfg::kTensorBytes;
+        const int per_row = Cfg::kPanels * 8;
+        for (int idx = r; idx < (TH - z0) * per_row; idx += 128) {
+          const int row = wg * TH + z0 + idx / per_row;
+          const int rem = idx % per_row;
+          *reinterpret_cast<uint4*>(vgen + (rem / 8) * Cfg::kPanelBytes + row * 128 + (rem % 8) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
       if (__any_sync(0xffffffffu, rescale)) {
         // this warpgroup's O must be stable: the PV of its previous tile has to be complete
         const int64_t kprev = k_mine_last;
@@ -624,12 +644,8 @@ __global__ void __launch_bounds__(384, 1)
     // Both warpgroups finish the segment together, each on half of the head dims of both O
     // accumulators: O = s_0 O_0 + s_1 O_1 with s_w = 2^(m_w - LSE) and LSE = log2(l_0 2^m_0 + l_1 2^m_1)
     // (the base-2 log-sum-exp of the segment; m_w, l_w are warpgroup w's reference max and sum).
-    // Each warpgroup publishes its own log-sum-exp, then its scale, through shared memory.
-    if (k_mine_last >= 0) {
-      bool ok = (*abort_flag == 0);
-      if (ok) ok = mbar_wait(pv_bar(k_mine_last), pv_par(k_mine_last), p.error_word);
-      if (!ok) *abort_flag = 1;
-    }
+    // Each warpgroup publishes its own log-sum-exp, then its scale, through shared memory; this needs
+    // only the softmax state, so it runs while the segment's last P V is still in flight.
     const bool have_keys = k_mine_last >= 0 && l_run > 0.f;
     const float lse_mine = have_keys ? m_ref + __log2f(l_run) : -INFINITY;
     sh->xs[wg][r] = lse_mine;
@@ -646,6 +662,11 @@ __global__ void __launch_bounds__(384, 1)
     const float s0 = wg == 0 ? s_mine : s_other;
     const float s1 = wg == 0 ? s_other : s_mine;
     const bool use0 = s0 > 0.f, use1 = s1 > 0.f;
+    if (k_mine_last >= 0) {
+      bool ok = (*abort_flag == 0);
+      if (ok) ok = mbar_wait(pv_bar(k_mine_last), pv_par(k_mine_last), p.error_word);
+      if (!ok) *abort_flag = 1;
+    }
     tc::fence_after_sync();
     const bool whole_unit = (tbegin == 0 && tend == Tb);
     const int slot = 2 * static_cast<int>(blockIdx.x) + (first_segment ? 0 : 1);
@@ -653,12 +674,20 @@ __global__ void __launch_bounds__(384, 1)
     float* pdst = p.part_o + static_cast<int64_t>(slot) * D * 128 + r;  // transposed: [D][128] per slot
     const uint32_t o0 = tmem + lane_base + Cfg::kOCol;
     const uint32_t o1 = o0 + 128;
-#pragma unroll 1
-    for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
-      uint32_t a[32], bb[32];
-      tc::ld_32x32b_x32(o0 + c * 32, a);
-      tc::ld_32x32b_x32(o1 + c * 32, bb);
-      tc::wait_ld();
+    // this warpgroup's D / 64 chunks of 32 head dims from both accumulators, loads issued together
+    constexpr int NCH = D / 64;
+    uint32_t oa[NCH][32], ob[NCH][32];
+#pragma unroll
+    for (int cc = 0; cc < NCH; ++cc) {
+      tc::ld_32x32b_x32(o0 + (wg * NCH + cc) * 32, oa[cc]);
+      tc::ld_32x32b_x32(o1 + (wg * NCH + cc) * 32, ob[cc]);
+    }
+    tc::wait_ld();
+#pragma unroll
+    for (int cc = 0; cc < NCH; ++cc) {
+      const int c = wg * NCH + cc;
+      const uint32_t(&a)[32] = oa[cc];
+      const uint32_t(&bb)[32] = ob[cc];
       float x[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e)
