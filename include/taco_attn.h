@@ -209,10 +209,13 @@ taco_status paged_kv_append_e4m3(const void* k_new, const void* v_new, const int
 /*
  * paged_tree_attention_e4m3: paged_tree_attention over e4m3 caches (layout and scales as above): the
  * result is that of paged_tree_attention with K = decode(k_cache) * k_scale[h] and V = decode(v_cache) *
- * v_scale[h]. q and out are `dtype` (F16 / BF16). Supported: head_dim 128 and packed query rows
- * (num_q_heads / num_kv_heads) * max_candidates <= 64; other sizes return TACO_ERR_UNSUPPORTED. The
- * workspace rules of paged_tree_attention apply. k_scale, v_scale: device float32 [Hkv], finite and
- * nonzero (not checked).
+ * v_scale[h]. q and out are `dtype` (F16 / BF16). Every size paged_tree_attention takes is supported
+ * (head_dim 64 or 128, any packed query rows). Narrow tiles (head_dim 128, fewer than 48 packed rows)
+ * run a warp-MMA kernel that widens the codes in registers; every other shape runs the tensor-core
+ * (tcgen05) kernel, which widens each tile of codes once, exactly, to f16 in shared memory. For bf16
+ * queries that kernel multiplies each query row by a power of two and rounds it to f16 (exact for every
+ * element down to 2^-29 of the row's largest magnitude) in the workspace first. The workspace rules of
+ * paged_tree_attention apply. k_scale, v_scale: device float32 [Hkv], finite and nonzero (not checked).
  */
 taco_status paged_tree_attention_e4m3(const void* q, const void* k_cache, const void* v_cache,
                                       const float* k_scale, const float* v_scale,
@@ -223,6 +226,22 @@ taco_status paged_tree_attention_e4m3(const void* q, const void* k_cache, const 
                                       int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                       int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
                                       void* stream);
+
+/*
+ * paged_tree_attention_append_e4m3: paged_kv_append_e4m3 of each sequence's candidates into logical
+ * slots P_b .. L_b - 1 (slot_offsets derived as for paged_tree_attention_append), then
+ * paged_tree_attention_e4m3 over the updated caches, in one call: the quantising append kernel runs
+ * first on `stream` and the verify waits for it on the device. k_new, v_new: [B, C, Hkv, D] `dtype`.
+ * Every other argument, rule and error is that of the two calls.
+ */
+taco_status paged_tree_attention_append_e4m3(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                             void* v_cache, const float* k_scale, const float* v_scale,
+                                             const int32_t* block_tables, const int32_t* context_lens,
+                                             const int32_t* num_candidates, const uint32_t* tree_mask_bits,
+                                             float scale, void* out, int32_t dtype, int32_t batch,
+                                             int32_t max_candidates, int32_t num_q_heads, int32_t num_kv_heads,
+                                             int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                             int32_t max_blocks_per_seq, void* stream);
 
 /*
  * The step after the verify. The pages ("大模型倍速推理引擎 TACO-LLM 的设计与实践", sections

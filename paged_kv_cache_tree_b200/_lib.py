@@ -35,6 +35,7 @@ EXPORTED = (
     "paged_tree_attention_noalloc",
     "paged_tree_attention_append",
     "paged_tree_attention_e4m3",
+    "paged_tree_attention_append_e4m3",
     "paged_kv_append_e4m3",
     "taco_attn_last_error",
     "taco_attn_check_device",
@@ -79,6 +80,8 @@ def load() -> ctypes.CDLL:
     lib.paged_kv_append.restype = i32
     lib.paged_tree_attention_e4m3.argtypes = [vp] * 9 + [f32, vp] + [i32] * 9 + [vp]
     lib.paged_tree_attention_e4m3.restype = i32
+    lib.paged_tree_attention_append_e4m3.argtypes = [vp] * 11 + [f32, vp] + [i32] * 9 + [vp]
+    lib.paged_tree_attention_append_e4m3.restype = i32
     lib.paged_kv_append_e4m3.argtypes = [vp] * 8 + [i32] * 8 + [vp]
     lib.paged_kv_append_e4m3.restype = i32
     lib.taco_attn_last_error.argtypes = []
@@ -249,9 +252,11 @@ def _need_scales(k_scale, v_scale, Hkv: int) -> None:
 
 def paged_tree_attention_e4m3(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_candidates,
                               tree_mask_bits, scale: float, out: Optional[torch.Tensor] = None,
-                              stream=None) -> torch.Tensor:
+                              stream=None, k_new=None, v_new=None) -> torch.Tensor:
     """Attention over e4m3 caches: q [B,C,Hq,D] bf16/fp16; k/v_cache uint8 [NB,Hkv,bs,D] e4m3 codes;
-    k_scale / v_scale float32 [Hkv] (value = decode(code) * scale[h]). Returns ``out`` (q's dtype)."""
+    k_scale / v_scale float32 [Hkv] (value = decode(code) * scale[h]). Returns ``out`` (q's dtype).
+    With ``k_new`` / ``v_new`` ([B,C,Hkv,D], q's dtype) the candidates are first appended (quantised)
+    at slots P_b .. L_b - 1 in the same call (paged_tree_attention_append_e4m3)."""
     _need_cuda("q", q, (torch.bfloat16, torch.float16), 4)
     _need_cuda("k_cache", k_cache, torch.uint8, 4)
     _need_cuda("v_cache", v_cache, torch.uint8, 4)
@@ -273,6 +278,17 @@ def paged_tree_attention_e4m3(q, k_cache, v_cache, k_scale, v_scale, block_table
     _need_cuda("out", out, q.dtype, 4)
     if tuple(out.shape) != tuple(q.shape):
         raise ValueError("out must have q's shape")
+    if k_new is not None or v_new is not None:
+        for name, t in (("k_new", k_new), ("v_new", v_new)):
+            _need_cuda(name, t, q.dtype, 4)
+            if tuple(t.shape) != (B, C, Hkv, D):
+                raise ValueError(f"{name} must be [B, C, Hkv, D]")
+        _check(load().paged_tree_attention_append_e4m3(
+            q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+            k_scale.data_ptr(), v_scale.data_ptr(), block_tables.data_ptr(), context_lens.data_ptr(),
+            num_candidates.data_ptr(), tree_mask_bits.data_ptr(), float(scale), out.data_ptr(), _dtype_code(q), B, C,
+            Hq, Hkv, D, bs, NB, block_tables.shape[1], _stream_handle(stream, q.device)))
+        return out
     _check(load().paged_tree_attention_e4m3(
         q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(),
         block_tables.data_ptr(), context_lens.data_ptr(), num_candidates.data_ptr(), tree_mask_bits.data_ptr(),

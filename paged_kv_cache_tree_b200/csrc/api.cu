@@ -19,7 +19,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAbiVersion = 6;
+constexpr int kAbiVersion = 7;
 
 thread_local std::string g_last_error;
 
@@ -49,6 +49,8 @@ struct Workspace {
   size_t lse_cap = 0;  // floats
   float* part_o = nullptr;
   size_t o_cap = 0;    // floats
+  uint8_t* qbuf = nullptr;  // e4m3 tcgen05 path: f16 query rows, then one float scale per row
+  size_t q_cap = 0;         // bytes
 };
 
 std::mutex g_mu;
@@ -73,19 +75,22 @@ taco_status sm_count_of(int dev, int* out) {
 // Make sure the workspace of (device `dev`, `stream`) has room and return it in *out; returns a status.
 // Caller holds g_mu.
 taco_status ensure_workspace(int dev, void* stream, size_t counters, size_t lse_floats, size_t o_floats,
-                             Workspace** out) {
+                             Workspace** out, size_t q_bytes = 0) {
   Workspace& w = g_ws[std::make_pair(dev, reinterpret_cast<uintptr_t>(stream))];
   *out = &w;
-  if (w.base && counters <= w.counters_cap && lse_floats <= w.lse_cap && o_floats <= w.o_cap) return TACO_OK;
+  if (w.base && counters <= w.counters_cap && lse_floats <= w.lse_cap && o_floats <= w.o_cap && q_bytes <= w.q_cap)
+    return TACO_OK;
   // grow (keeping at least the old capacities); the old buffer may still be in use by queued
   // work, so wait for the device before freeing it
   counters = std::max(counters, w.counters_cap);
   lse_floats = std::max(lse_floats, w.lse_cap);
   o_floats = std::max(o_floats, w.o_cap);
+  q_bytes = std::max(q_bytes, w.q_cap);
   const size_t off_counters = 256;
   const size_t off_lse = off_counters + round_up(counters * 4, 256);
   const size_t off_o = off_lse + round_up(lse_floats * 4, 256);
-  const size_t total = off_o + round_up(o_floats * 4, 256);
+  const size_t off_q = off_o + round_up(o_floats * 4, 256);
+  const size_t total = off_q + round_up(q_bytes, 256);
   uint32_t old_err = 0;
   if (w.base) {
     cudaError_t e = cudaDeviceSynchronize();
@@ -112,6 +117,8 @@ taco_status ensure_workspace(int dev, void* stream, size_t counters, size_t lse_
   w.lse_cap = lse_floats;
   w.part_o = reinterpret_cast<float*>(w.base + off_o);
   w.o_cap = o_floats;
+  w.qbuf = w.base + off_q;
+  w.q_cap = q_bytes;
   return TACO_OK;
 }
 
@@ -131,20 +138,22 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // [NB * Hkv * bs rows, D columns] view of a cache; box = one 128-byte swizzle row (64 16-bit values,
 // or 128 e4m3 codes when kv8) x rows_per_chunk rows.
+// raw_rows (e4m3 only): whole D-byte rows, no swizzle (the tcgen05 path widens them in shared memory).
 taco_status make_cache_map(CUtensorMap* map, const void* base, int dtype, int D, int64_t rows, int rows_per_chunk,
-                           bool kv8 = false) {
+                           bool kv8 = false, bool raw_rows = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int elt = kv8 ? 1 : 2;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * elt};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elt), static_cast<cuuint32_t>(rows_per_chunk)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(raw_rows ? D : 128 / elt), static_cast<cuuint32_t>(rows_per_chunk)};
   cuuint32_t estr[2] = {1, 1};
   const CUtensorMapDataType ty = kv8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                      : (dtype == TACO_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   CUresult r = enc(map, ty, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   raw_rows ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return TACO_OK;
 }
@@ -239,36 +248,42 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
     return fail(TACO_ERR_INVALID_ARG, "null pointer argument");
   if (k_new && (!v_new || !aligned16(k_new) || !aligned16(v_new)))
     return fail(TACO_ERR_INVALID_ARG, "k_new and v_new must be non-null and 16-byte aligned");
-  if (kv8) {
-    if (!v_scale) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (v_scale)");
-    if (head_dim != 128) return fail(TACO_ERR_UNSUPPORTED, "e4m3 caches: head_dim must be 128");
-    if ((num_q_heads / num_kv_heads) * max_candidates > 64)
-      return fail(TACO_ERR_UNSUPPORTED, "e4m3 caches: (num_q_heads / num_kv_heads) * max_candidates must be <= 64");
-    if (g_opt_kernel == 2) return fail(TACO_ERR_UNSUPPORTED, "e4m3 caches have no tensor-core (tcgen05) kernel");
-  }
+  if (kv8 && !v_scale) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (v_scale)");
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return fail(TACO_ERR_INVALID_ARG, "q, k_cache, v_cache and out must be 16-byte aligned");
   if (!(scale == scale)) return fail(TACO_ERR_INVALID_ARG, "scale is NaN");
   if (batch == 0) return TACO_OK;
+  const int G = num_q_heads / num_kv_heads;
+  const int packed = G * max_candidates;
+  int64_t opt_kernel = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    opt_kernel = g_opt_kernel;
+  }
+  // kernel choice: the tcgen05 kernel once the packed (GQA group x candidates) tile is wide enough to
+  // keep the tensor cores busy, the mma.sync kernel for narrow tiles. e4m3 caches: the mma.sync kernel
+  // exists for head_dim 128 and <= 64 packed rows; everything else goes to the tcgen05 kernel, which
+  // widens the codes to f16 once per tile
+  const bool tc_possible = G <= 128;
+  const bool mma_possible = !kv8 || (head_dim == 128 && packed <= 64);
+  bool use_tc = tc_possible && (packed >= 48 || !mma_possible);
+  if (opt_kernel == 1) {
+    if (!mma_possible)
+      return fail(TACO_ERR_UNSUPPORTED, "e4m3 caches on the mma.sync path need head_dim 128 and G * C <= 64");
+    use_tc = false;
+  }
+  if (opt_kernel == 2) use_tc = true;
+  if (use_tc && !tc_possible)
+    return fail(TACO_ERR_UNSUPPORTED, "tensor-core path needs num_q_heads / num_kv_heads <= 128");
+  if (!use_tc && !mma_possible)
+    return fail(TACO_ERR_UNSUPPORTED, "e4m3 caches: no kernel for num_q_heads / num_kv_heads > 128 with this shape");
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(TACO_ERR_UNSUPPORTED, "device index %d too large", dev);
 
-  const int G = num_q_heads / num_kv_heads;
-  const int packed = G * max_candidates;
-
   std::lock_guard<std::mutex> lk(g_mu);
-  // kernel choice: the tcgen05 path once the packed (GQA group x candidates) tile is wide enough to
-  // keep tensor cores busy; the mma.sync path for narrow tiles
-  const bool tc_possible = G <= 128;
-  bool use_tc = tc_possible && packed >= 48 && !kv8;
-  if (g_opt_kernel == 1) use_tc = false;
-  if (g_opt_kernel == 2) {
-    if (!tc_possible) return fail(TACO_ERR_UNSUPPORTED, "tensor-core path needs num_q_heads / num_kv_heads <= 128");
-    use_tc = true;
-  }
   int rows, row_groups, cands_per_group = 0;
   if (use_tc) {
     cands_per_group = std::min(max_candidates, 128 / G);
@@ -286,21 +301,29 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
   int grid = static_cast<int>(g_opt_grid);
   if (grid == 0) grid = (use_tc ? 1 : taco::mma_ctas_per_sm(rows)) * sms;
   const size_t slots = 2 * static_cast<size_t>(grid);
+  // e4m3 caches with bf16 queries on the tcgen05 path: f16 query rows and their scales in the workspace
+  const bool q_convert = use_tc && kv8 && dtype == TACO_DTYPE_BF16;
+  const int64_t q_rows = static_cast<int64_t>(batch) * max_candidates * num_q_heads;
+  const size_t q16_bytes = q_convert ? round_up(static_cast<size_t>(q_rows) * head_dim * 2, 256) : 0;
+  const size_t q_ws = q_convert ? q16_bytes + static_cast<size_t>(q_rows) * 4 : 0;
   Workspace* wp = nullptr;
-  st = ensure_workspace(dev, stream, static_cast<size_t>(units), slots * rows, slots * rows * head_dim, &wp);
+  st = ensure_workspace(dev, stream, static_cast<size_t>(units), slots * rows, slots * rows * head_dim, &wp, q_ws);
   if (st != TACO_OK) return st;
   Workspace& w = *wp;
 
   const int tile = use_tc ? taco::tc_tile_keys() : taco::mma_tile_keys(rows, kv8);
   const int rpc = block_size < tile ? block_size : tile;
   const int64_t cache_rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
+  const bool raw_rows = use_tc && kv8;
   CUtensorMap tk, tv, tq;
-  st = make_cache_map(&tk, k_cache, dtype, head_dim, cache_rows, rpc, kv8);
+  st = make_cache_map(&tk, k_cache, dtype, head_dim, cache_rows, rpc, kv8, raw_rows);
   if (st != TACO_OK) return st;
-  st = make_cache_map(&tv, v_cache, dtype, head_dim, cache_rows, rpc, kv8);
+  st = make_cache_map(&tv, v_cache, dtype, head_dim, cache_rows, rpc, kv8, raw_rows);
   if (st != TACO_OK) return st;
   if (use_tc) {
-    st = make_query_map(&tq, q, dtype, head_dim, num_q_heads, static_cast<int64_t>(batch) * max_candidates, G,
+    const void* qsrc = q_convert ? static_cast<const void*>(w.qbuf) : q;
+    const int qdtype = kv8 ? TACO_DTYPE_F16 : dtype;
+    st = make_query_map(&tq, qsrc, qdtype, head_dim, num_q_heads, static_cast<int64_t>(batch) * max_candidates, G,
                         cands_per_group);
     if (st != TACO_OK) return st;
   }
@@ -334,6 +357,7 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
       g_opt_prefetch >= 0 ? g_opt_prefetch : (use_tc ? taco::kTcPrefetchTiles : taco::kMmaPrefetchTiles));
   p.k_scale = k_scale;
   p.v_scale = v_scale;
+  p.q_scale = q_convert ? reinterpret_cast<const float*>(w.qbuf + q16_bytes) : nullptr;
   if (k_new) {
     // fused append where the kernel supports it (mma.sync, <= 16 rows, 16-bit caches); otherwise the
     // append kernel runs first on the same stream
@@ -346,9 +370,17 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
       taco::AppendArgs a{k_new, v_new, block_tables, nullptr, const_cast<void*>(k_cache), const_cast<void*>(v_cache),
                          w.error_word, batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks,
                          max_blocks_per_seq, dtype, context_lens, num_candidates};
-      e = taco::launch_append(a, static_cast<cudaStream_t>(stream));
+      e = kv8 ? taco::launch_append_e4m3(a, k_scale, v_scale, static_cast<cudaStream_t>(stream))
+              : taco::launch_append(a, static_cast<cudaStream_t>(stream));
       if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
     }
+  }
+  // after the append (a plain launch: it starts once the append has finished, and the verify's
+  // dependency wait then covers both)
+  if (q_convert) {
+    e = taco::launch_q_to_f16(q, w.qbuf, reinterpret_cast<float*>(w.qbuf + q16_bytes), q_rows, head_dim,
+                              static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "query conversion launch");
   }
 
   if (use_tc) {
@@ -394,6 +426,21 @@ taco_status paged_tree_attention_e4m3(const void* q, const void* k_cache, const 
                                       int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
   if (!k_scale || !v_scale) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (k_scale / v_scale)");
   return attention_impl(q, k_cache, v_cache, k_scale, v_scale, nullptr, nullptr, block_tables, context_lens,
+                        num_candidates, tree_mask_bits, scale, out, dtype, batch, max_candidates, num_q_heads,
+                        num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, stream);
+}
+
+taco_status paged_tree_attention_append_e4m3(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                             void* v_cache, const float* k_scale, const float* v_scale,
+                                             const int32_t* block_tables, const int32_t* context_lens,
+                                             const int32_t* num_candidates, const uint32_t* tree_mask_bits,
+                                             float scale, void* out, int32_t dtype, int32_t batch,
+                                             int32_t max_candidates, int32_t num_q_heads, int32_t num_kv_heads,
+                                             int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                             int32_t max_blocks_per_seq, void* stream) {
+  if (!k_new || !v_new) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (k_new / v_new)");
+  if (!k_scale || !v_scale) return fail(TACO_ERR_INVALID_ARG, "null pointer argument (k_scale / v_scale)");
+  return attention_impl(q, k_cache, v_cache, k_scale, v_scale, k_new, v_new, block_tables, context_lens,
                         num_candidates, tree_mask_bits, scale, out, dtype, batch, max_candidates, num_q_heads,
                         num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, stream);
 }

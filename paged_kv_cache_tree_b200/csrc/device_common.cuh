@@ -41,6 +41,7 @@ struct VerifyParams {
   int l2_prefetch_tiles; // key tiles whose K/V the producer asks L2 to fetch ahead of its loads (0 = none)
   const float* k_scale;  // e4m3 caches: per-KV-head scales (K value = code * k_scale[h]); else null
   const float* v_scale;
+  const float* q_scale;  // e4m3 caches on the tcgen05 path: the f16 query rows' scale per row, or null
   // fused append (16-bit caches, units of <= 16 rows): candidate i's new K/V rows [B, C, Hkv, D] go to
   // logical slot P_b + i of these caches as the verify reads them; null = the caches are complete
   const void* k_new;
@@ -580,7 +581,73 @@ struct TilePrefetcher {
   }
 };
 
+// A producer's walk over its CTA's tiles, one tile at a time, with the block-table window of the
+// current segment; chunk() gives a lane's chunk of the current tile the way the 16-bit producers
+// compute it (lane l takes rows [l rpc, (l + 1) rpc) of the tile; chunks past the context or with a
+// bad block id are not loaded).
+struct TileLoadCursor {
+  SegCursor c;
+  int tl, tend, g, nblk, win;
+  int32_t win_val;
+  const int32_t* bt_row;
+  int64_t k;  // CTA-local ordinal of the current tile
+  bool have, report;
+
+  __device__ __forceinline__ void start_segment(const VerifyParams& p) {
+    tl = c.tile;
+    tend = c.seg_end();
+    g = c.j / p.row_groups;
+    nblk = (c.L + p.bs - 1) / p.bs;
+    bt_row = p.block_tables + static_cast<int64_t>(c.b) * p.max_blocks;
+    win = -1000000;
+    win_val = -1;
+  }
+  __device__ __forceinline__ void init(const VerifyParams& p, int b0, int64_t base_b0, int64_t lo, int64_t hi,
+                                       bool report_) {
+    report = report_;
+    c.init(p, b0, base_b0, lo, hi, report);
+    k = 0;
+    have = c.valid();
+    if (have) start_segment(p);
+  }
+  __device__ __forceinline__ void step(const VerifyParams& p) {
+    ++k;
+    if (++tl == tend) {
+      c.next_segment(p, report);
+      have = c.valid();
+      if (have) start_segment(p);
+    }
+  }
+  // Whole warp. Returns whether this lane loads a chunk; *row is its first cache row, *nloaded the
+  // number of chunks the warp loads.
+  __device__ __forceinline__ bool chunk(const VerifyParams& p, int tk, int rpc, int* row, int* nloaded) {
+    const int lane = threadIdx.x & 31;
+    const int chunks_per_tile = tk / rpc;
+    const int L = c.L;
+    const int key0 = tl * tk;
+    int nvalid = L > key0 ? (L - key0 + rpc - 1) / rpc : 0;
+    if (nvalid > chunks_per_tile) nvalid = chunks_per_tile;
+    const int lb_first = key0 / p.bs;
+    if (nvalid > 0 && (lb_first < win || (key0 + (nvalid - 1) * rpc) / p.bs >= win + 32)) {
+      win = lb_first;
+      const int lb = win + lane;
+      win_val = lb < nblk ? __ldg(bt_row + lb) : -1;
+    }
+    const int my_lb = (key0 + lane * rpc) / p.bs;
+    const int32_t blk = __shfl_sync(0xffffffffu, win_val, (my_lb - win) & 31);
+    bool ok = lane < nvalid;
+    if (ok && (blk < 0 || blk >= p.num_blocks)) {
+      if (report) atomicOr(p.error_word, TACO_DEVERR_BLOCK_ID);
+      ok = false;
+    }
+    *nloaded = __popc(__ballot_sync(0xffffffffu, ok));
+    *row = (blk * p.Hkv + g) * p.bs + (key0 + lane * rpc) % p.bs;
+    return ok;
+  }
+};
+
 struct TileInfo {
+  int b, j;    // the tile's sequence and unit within it (j = kv head * row groups + row group)
   int ui;      // segment ordinal within the CTA
   int tl;      // tile index within the unit
   int jl;      // tile index within the segment
@@ -603,6 +670,8 @@ struct TileWalker {
   }
   __device__ __forceinline__ bool next(const VerifyParams& p, TileInfo& ti) {
     if (!have) return false;
+    ti.b = c.b;
+    ti.j = c.j;
     ti.ui = c.ui;
     ti.tl = tl;
     ti.jl = tl - c.tile;

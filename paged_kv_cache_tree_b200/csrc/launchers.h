@@ -81,7 +81,10 @@ cudaError_t launch_copy_len_update(const int32_t* accept_len, const int32_t* pro
 // Keys per work tile of the tcgen05 verify kernel.
 int tc_tile_keys();
 // Dynamic shared memory of the tcgen05 verify kernel.
-int tc_smem_bytes(int D);
+int tc_smem_bytes(int D, bool kv8 = false);
+// bf16 query rows -> f16 rows times a power of two per row, and that power's inverse per row (the e4m3
+// tcgen05 path's query operand).
+cudaError_t launch_q_to_f16(const void* q, void* q16, float* qscale, int64_t rows, int D, cudaStream_t stream);
 cudaError_t launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                              const VerifyParams& p, int dtype, int grid, cudaStream_t stream);
 // Store the message taco_attn_last_error() returns on this thread.

@@ -3,24 +3,24 @@
 // The candidates of one (sequence, KV head) form up to 128 query rows (r = i_local * G + h'), the
 // M = 128 operand of tcgen05.mma; this is how several candidates turn the decode GEMV into a GEMM
 // ("大模型倍速推理引擎 TACO-LLM 的设计与实践", TurboAttention bullets under "整体方案分为两大部分").
-// One CTA per SM, persistent over the same stream-K tile ranges as the mma.sync path:
-//   warps 0, 10 producers: TMA loads of each segment's Q tile (3-D box over [B*C, Hq, D]) and of
-//               every 64-key tile's K chunks (warp 0) and V chunks (warp 10) reached through the block
-//               table, into separate K and V rings (K is released as soon as its Q K^T is done, V
-//               after its P V);
-//   warp 1      Q K^T issuer (one thread): S = Q K^T into one of four tensor-memory S buffers
-//               (64 fp32 columns each), up to four tiles ahead of the P V issuer;
-//   warp 11     P V issuer (one thread): O += P V with P read back from tensor memory (A operand)
-//               and V from shared memory (MN-major B operand). Two issuing threads, each waiting
-//               only for its own inputs in tile order, because issuing one tcgen05.mma or commit
-//               costs a single thread tens of cycles and one thread doing both products plus the
+// One CTA per SM, persistent over the same stream-K tile ranges as the mma.sync path, 128-key tiles:
+//   warps 0, 10 producers: TMA loads of each segment's Q tile (3-D box over [B*C, Hq, D]) and of every
+//               tile's K chunks (warp 0) and V chunks (warp 10) reached through the block table, into
+//               separate K and V rings (K is released as soon as its Q K^T is done, V after its P V).
+//               With e4m3 caches they load raw codes and widen each tile once into the 16-bit layout;
+//   warp 1      Q K^T issuer (one thread): S = Q K^T (M = 128, N = 128) into one of two tensor-memory
+//               S buffers of 128 fp32 columns;
+//   warp 11     P V issuer (one thread): O_w += P_w V_w per 64-key half w, with P read back from tensor
+//               memory (A operand) and V from shared memory (MN-major B operand). Two issuing threads,
+//               each waiting only for its own inputs in tile order, because issuing one tcgen05.mma or
+//               commit costs a single thread tens of cycles and one thread doing both products plus the
 //               polling between them became the bound of the whole kernel;
-//   warps 2..9  two softmax warpgroups; tile k belongs to warpgroup k % 2, which owns its own O
-//               accumulator in tensor memory. Thread r of a warpgroup owns query row r (lane r):
-//               base-2 online softmax in fp32 whose reference max only moves when a row's max grows
-//               by more than 2^8 (so O is rescaled rarely), P written back as bf16/fp16 pairs into
-//               the S buffer. At the end of a segment warpgroup 0 merges the two accumulators
-//               (log-sum-exp weights) and normalises, or writes a split-KV partial.
+//   warps 2..9  two softmax warpgroups; warpgroup w takes keys [64 w, 64 w + 64) of every tile and owns
+//               its own O accumulator in tensor memory. Thread r of a warpgroup owns query row r (lane
+//               r): base-2 online softmax in fp32 whose reference max only moves when a row's max grows
+//               by more than 2^8 (so O is rescaled rarely), P written back as 16-bit pairs into the S
+//               buffer. At the end of a segment both warpgroups combine the two accumulators (each on
+//               half of the head dims) and normalise, or write a split-KV partial.
 // MMA completion is signalled with tcgen05.commit on mbarriers; every wait is bounded.
 #pragma once
 
@@ -38,7 +38,10 @@ namespace taco {
 // every tile.
 constexpr int kTcTileKeys = 128;
 
-template <int D>
+// KV8: e4m3 caches. Their tiles land in rings of raw codes and the producer warps widen each one
+// once (exactly) into a 16-bit stage of the same layout as a 16-bit cache's, so everything downstream
+// is the 16-bit pipeline with f16 operands.
+template <int D, bool KV8 = false>
 struct TcCfg {
   static constexpr int kThreads = 384;
   static constexpr int kTK = kTcTileKeys;
@@ -46,16 +49,18 @@ struct TcCfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = kTK * 128;            // kTK keys x 128 bytes
   static constexpr int kTensorBytes = kPanels * kPanelBytes;
-  static constexpr int kKStages = (D == 128) ? 3 : 6;
-  static constexpr int kVStages = (D == 128) ? 3 : 6;
+  static constexpr int kKStages = KV8 ? ((D == 128) ? 2 : 4) : ((D == 128) ? 3 : 6);
+  static constexpr int kVStages = kKStages;
+  static constexpr int kRawStages = KV8 ? ((D == 128) ? 2 : 3) : 0;  // raw e4m3 tiles per tensor
+  static constexpr int kRawBytes = kTK * D;                // one raw tile: kTK keys x D codes
   static constexpr int kQPanelBytes = 128 * 128;           // 128 rows x 128 bytes
   static constexpr int kQBytes = kPanels * kQPanelBytes;
   static constexpr int kSBufs = 2;                         // S/P buffers of kTK columns at 0, 128
   static constexpr int kTmemCols = 512;
   static constexpr int kOCol = 256;                        // O of warpgroup w at kOCol + w * 128
-  static constexpr int kSharedBytes = 1536;
-  static constexpr int kSmemBytes =
-      1024 + (kKStages + kVStages) * kTensorBytes + kQBytes + kSharedBytes;
+  static constexpr int kSharedBytes = 2048;
+  static constexpr int kSmemBytes = 1024 + (kKStages + kVStages) * kTensorBytes + kQBytes +
+                                    2 * kRawStages * kRawBytes + kSharedBytes;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
@@ -66,11 +71,13 @@ struct TcShared {
   // p_full[2 sb + w]: warpgroup w wrote its half of P into S buffer sb.
   uint64_t k_full[6], k_empty[6], v_full[6], v_empty[6];
   uint64_t q_full, q_empty, s_full[2], p_full[4], o_free;
+  // e4m3 caches: raw tiles of K (index 0) and V (index 1) landed / free again
+  uint64_t raw_full[2][4], raw_empty[2][4];
   uint32_t tmem_base;
   int merge_flag, abort_flag;
   long long W, lo, hi, base_b;
   int nC, b;
-  // per-row values the two softmax warpgroups exchange at a segment's end (log-sum-exp, then scale);
+  // per-row values the two softmax warpgroups exchange at a segment's end (reference max, then weighted sum);
   // the next segment's exchange comes after that segment's last P V, which waits for O to be
   // released, which both warpgroups do only after their reads here.
   float xs[2][128];
@@ -152,16 +159,20 @@ __device__ __forceinline__ void merge_split_row_half(const VerifyParams& p, int 
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool KV8>
 __global__ void __launch_bounds__(384, 1)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const __grid_constant__ CUtensorMap tmap_q, const VerifyParams p) {
-  using Cfg = TcCfg<D>;
-  using Op = MmaOp<T>;
+  using Cfg = TcCfg<D, KV8>;
+  using Op = MmaOp<T>;                       // the output's type
+  // operands of the tensor-core products: the queries' type, or f16 for e4m3 caches (codes widen
+  // exactly to f16; the queries then come as f16 with a power-of-two scale per row)
+  using POp = typename std::conditional<KV8, MmaOp<__half>, MmaOp<T>>::type;
   constexpr int SK = Cfg::kKStages;
   constexpr int SV = Cfg::kVStages;
   constexpr int NS = Cfg::kSBufs;
-  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  constexpr int RS = Cfg::kRawStages;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value && !KV8;
   constexpr int TK = Cfg::kTK;
   constexpr int TH = Cfg::kHalf;
   constexpr uint32_t kIdescQK = tc::idesc_f16(kBf16 ? 1 : 0, 128, TK, 0);
@@ -173,7 +184,8 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* kring = smem;
   uint8_t* vring = kring + SK * Cfg::kTensorBytes;
   uint8_t* qbuf = vring + SV * Cfg::kTensorBytes;
-  TcShared* sh = reinterpret_cast<TcShared*>(qbuf + Cfg::kQBytes);
+  uint8_t* rawring = qbuf + Cfg::kQBytes;  // e4m3: RS raw K tiles, then RS raw V tiles
+  TcShared* sh = reinterpret_cast<TcShared*>(rawring + 2 * RS * Cfg::kRawBytes);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -193,6 +205,11 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; j < NS; ++j) mbar_init(smem_addr(&sh->s_full[j]), 1);
     for (int j = 0; j < 2 * NS; ++j) mbar_init(smem_addr(&sh->p_full[j]), 4);
     mbar_init(smem_addr(&sh->o_free), 8);
+    for (int t = 0; t < 2; ++t)
+      for (int s = 0; s < RS; ++s) {
+        mbar_init(smem_addr(&sh->raw_full[t][s]), 1);
+        mbar_init(smem_addr(&sh->raw_empty[t][s]), 1);
+      }
     sh->merge_flag = 0;
     sh->abort_flag = 0;
     fence_mbar_init();
@@ -238,6 +255,134 @@ __global__ void __launch_bounds__(384, 1)
   const int cpg = p.cands_per_group;
   const int qrows = cpg * p.G;
 
+  if constexpr (KV8) {
+    if (warp == 0 || warp == 10) {
+      // -------------------------------------------------------------- e4m3 producers
+      // Warp 0 streams Q (f16, 3-D box) and K, warp 10 streams V. Each loads raw tiles of codes into a
+      // ring of RS slots up to RS tiles ahead, and widens every landed tile, in tile order, into a
+      // 16-bit stage in the layout a 16-bit cache's TMA load leaves (two 64-column 128-byte-swizzled
+      // panels): cvt.rn.f16x2.e4m3x2 is exact, so the stage holds exactly decode(code); the scale per
+      // KV head is applied to the scores and to O instead.
+      const int t = (warp == 0) ? 0 : 1;
+      const bool is_k = (t == 0);
+      const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
+      prefetch_tensormap(tmap);
+      if (is_k) prefetch_tensormap(&tmap_q);
+      const uint64_t policy = policy_evict_first();
+      const int rpc = p.bs < TK ? p.bs : TK;
+      const uint32_t chunk_bytes = static_cast<uint32_t>(rpc) * D;
+      const uint32_t q_bytes = static_cast<uint32_t>(Cfg::kPanels * qrows * 128);
+      uint8_t* raw = rawring + t * RS * Cfg::kRawBytes;
+      uint8_t* conv = is_k ? kring : vring;
+      uint64_t* conv_full = is_k ? sh->k_full : sh->v_full;
+      uint64_t* conv_empty = is_k ? sh->k_empty : sh->v_empty;
+      constexpr int SC = SK;  // converted stages (SK == SV)
+      TileLoadCursor lc;
+      lc.init(p, sh->b, sh->base_b, lo, hi, is_k);
+      TileWalker cw;  // conversion order (same tiles)
+      cw.init(p, sh->b, sh->base_b, lo, hi);
+      TileInfo ti;
+      bool ok = true;
+      int64_t kc = 0;
+      int q_issued_ui = -1;
+      // raw load of the cursor's current tile into slot lc.k % RS
+      auto issue_raw = [&]() {
+        int row, nload;
+        const bool mine = lc.chunk(p, TK, rpc, &row, &nload);
+        const int rs = static_cast<int>(lc.k % RS);
+        bool go = true;
+        if (lane == 0) {
+          go = ok && (*abort_flag == 0) &&
+               mbar_wait(smem_addr(&sh->raw_empty[t][rs]), static_cast<uint32_t>(((lc.k / RS) & 1) ^ 1), p.error_word);
+          if (!go) *abort_flag = 1;
+          mbar_arrive_expect_tx(smem_addr(&sh->raw_full[t][rs]), go ? static_cast<uint32_t>(nload) * chunk_bytes : 0u);
+        }
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) ok = false;
+        if (go && mine)
+          tma_load_2d(smem_addr(raw + rs * Cfg::kRawBytes) + (threadIdx.x & 31) * chunk_bytes, tmap,
+                      smem_addr(&sh->raw_full[t][rs]), 0, row, policy);
+        __syncwarp();
+        lc.step(p);
+      };
+      while (cw.next(p, ti)) {
+        // keep up to RS raw tiles in flight ahead of the conversion
+        while (lc.have && lc.k < kc + RS) issue_raw();
+        if (is_k && ti.first && q_issued_ui < ti.ui) {
+          // the segment's Q tile: the single Q buffer is free once the previous segment's last Q K^T
+          // is done (that needs only tiles converted already, so this wait always ends)
+          if (lane == 0) {
+            const bool go = ok && (*abort_flag == 0) &&
+                            mbar_wait(smem_addr(&sh->q_empty), static_cast<uint32_t>((ti.ui & 1) ^ 1), p.error_word);
+            if (!go) {
+              ok = false;
+              *abort_flag = 1;
+            }
+            mbar_arrive_expect_tx(smem_addr(&sh->q_full), go ? q_bytes : 0u);
+            if (go) {
+#pragma unroll
+              for (int pn = 0; pn < Cfg::kPanels; ++pn)
+                tma_load_3d(smem_addr(qbuf) + pn * Cfg::kQPanelBytes, &tmap_q, smem_addr(&sh->q_full), pn * 64,
+                            (ti.j / p.row_groups) * p.G, ti.b * p.C + (ti.j % p.row_groups) * cpg);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          q_issued_ui = ti.ui;
+        }
+        const int rs = static_cast<int>(kc % RS);
+        const int cs = static_cast<int>(kc % SC);
+        bool go = true;
+        if (lane == 0) {
+          go = ok && (*abort_flag == 0) &&
+               mbar_wait(smem_addr(&sh->raw_full[t][rs]), static_cast<uint32_t>((kc / RS) & 1), p.error_word) &&
+               mbar_wait(smem_addr(&conv_empty[cs]), static_cast<uint32_t>(((kc / SC) & 1) ^ 1), p.error_word);
+          if (!go) *abort_flag = 1;
+        }
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) ok = false;
+        if (go) {
+          const uint8_t* src = raw + rs * Cfg::kRawBytes;
+          uint8_t* dst = conv + cs * Cfg::kTensorBytes;
+          constexpr int CPR = D / 16;  // 16-code chunks per key row
+#pragma unroll 4
+          for (int idx = lane; idx < TK * CPR; idx += 32) {
+            const int row = idx / CPR;
+            const int c = idx % CPR;
+            const uint4 v = lds_v4(smem_addr(src + row * D + c * 16));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t h[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              h[2 * q] = e4m3x2_to_f16x2(w[q] & 0xffffu);
+              h[2 * q + 1] = e4m3x2_to_f16x2(w[q] >> 16);
+            }
+            // head dims [16c, 16c + 16) = 16-byte chunks 2(c % 4), 2(c % 4) + 1 of panel c / 4, swizzled
+            uint8_t* prow = dst + (c >> 2) * Cfg::kPanelBytes + row * 128;
+            const int j0 = 2 * (c & 3);
+            *reinterpret_cast<uint4*>(prow + ((j0 ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(prow + (((j0 + 1) ^ (row & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_addr(&conv_full[cs]));  // on abort too: nobody waits for a tile forever
+          mbar_arrive(smem_addr(&sh->raw_empty[t][rs]));
+        }
+        ++kc;
+      }
+      // wait (bounded) for our own copies still landing: raw tiles issued but not converted (after an
+      // abort) and the last Q tile
+      if (lane == 0) {
+        for (int64_t kk = kc; kk < lc.k; ++kk)
+          mbar_wait(smem_addr(&sh->raw_full[t][kk % RS]), static_cast<uint32_t>((kk / RS) & 1), p.error_word);
+        if (is_k && q_issued_ui >= 0)
+          mbar_wait(smem_addr(&sh->q_full), static_cast<uint32_t>(q_issued_ui & 1), p.error_word);
+      }
+      if (!ok && lane == 0) *abort_flag = 1;
+      return;
+    }
+  }
   if (warp == 0 || warp == 10) {
     // ------------------------------------------------------------------ producers
     // warp 0 streams Q and K, warp 10 streams V: both walk the same tiles and block table, so each
@@ -479,18 +624,29 @@ __global__ void __launch_bounds__(384, 1)
   bool first_segment = true;
   // a segment's candidate count and this row's mask word, as loaded (the next segment's are loaded
   // at the start of the current one, so that a segment switch does not wait for them)
-  auto load_seg_inputs = [&](int bb, int jj, int& n_raw, uint32_t& mw_raw) {
+  // e4m3 caches: the row's logit scale also takes the KV head's K scale and the row's query scale
+  auto load_seg_inputs = [&](int bb, int jj, int& n_raw, uint32_t& mw_raw, float& sl2) {
     n_raw = 0;
     mw_raw = 0u;
+    sl2 = p.scale_log2;
     if (bb < p.B) {
       n_raw = __ldg(p.num_candidates + bb);
+      const int gg = jj / p.row_groups;
       const int ii = (jj % p.row_groups) * cpg + r / p.G;
-      if (r < qrows && ii < p.C) mw_raw = __ldg(p.tree_mask_bits + static_cast<int64_t>(bb) * p.C + ii);
+      if (r < qrows && ii < p.C) {
+        mw_raw = __ldg(p.tree_mask_bits + static_cast<int64_t>(bb) * p.C + ii);
+        if constexpr (KV8) {
+          sl2 *= __ldg(p.k_scale + gg);
+          if (p.q_scale != nullptr)
+            sl2 *= __ldg(p.q_scale + (static_cast<int64_t>(bb) * p.C + ii) * p.Hq + gg * p.G + r % p.G);
+        }
+      }
     }
   };
   int n_raw_cur;
   uint32_t mw_raw_cur;
-  load_seg_inputs(cur.b, cur.j, n_raw_cur, mw_raw_cur);
+  float sl2_cur;
+  load_seg_inputs(cur.b, cur.j, n_raw_cur, mw_raw_cur, sl2_cur);
   while (cur.valid()) {
     const int b = cur.b;
     const int g = cur.j / p.row_groups;
@@ -507,9 +663,11 @@ __global__ void __launch_bounds__(384, 1)
     const bool row_real = r < qrows && i < p.C;  // a row of the output
     const bool active = row_real && i < n;       // a row with a query
     const uint32_t mw = active ? (mw_raw_cur & nmask) : 0u;
+    const float sl2 = sl2_cur;  // base-2 logit scale of this row
+    const float vsc = KV8 ? __ldg(p.v_scale + g) : 1.f;
     {
       const bool same_b = cur.j + 1 < cur.HR;
-      load_seg_inputs(same_b ? b : b + 1, same_b ? cur.j + 1 : 0, n_raw_cur, mw_raw_cur);
+      load_seg_inputs(same_b ? b : b + 1, same_b ? cur.j + 1 : 0, n_raw_cur, mw_raw_cur, sl2_cur);
     }
 
     float m_ref = -INFINITY;
@@ -531,13 +689,13 @@ __global__ void __launch_bounds__(384, 1)
       // Row max of the raw scores (a positive scale_log2 commutes with max; otherwise the scaled
       // values are used). Masked keys become -inf; only the tiles that reach the candidates mask.
       const bool need_mask = key0 + TH > P;
-      const bool pos_scale = p.scale_log2 > 0.f;
+      const bool pos_scale = sl2 > 0.f;
       float v[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) v[c] = __uint_as_float(sraw[c >> 5][c & 31]);
       if (!pos_scale) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) v[c] *= p.scale_log2;
+        for (int c = 0; c < 64; ++c) v[c] *= sl2;
       }
       if (need_mask) {
 #pragma unroll
@@ -559,7 +717,7 @@ __global__ void __launch_bounds__(384, 1)
       const bool first = (k_mine_last < 0);
       // rows without a query (padding) keep whatever their scores are; they never reach the output,
       // so they are simply kept out of the rescale decision
-      float mx = pos_scale ? mraw * p.scale_log2 : mraw;  // row max of the base-2 logits
+      float mx = pos_scale ? mraw * sl2 : mraw;  // row max of the base-2 logits
       if (!active) mx = first ? 0.f : m_ref;
       bool rescale = false;
       float alpha = 1.f;
@@ -572,8 +730,18 @@ __global__ void __launch_bounds__(384, 1)
         m_ref = mx;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // p = 2^(s * scale_log2 - m) on fp32 pairs; sums in four independent pair accumulators
-      const float sc = pos_scale ? p.scale_log2 : 1.f;
+      // p = 2^(s * scale_log2 - m) on fp32 pairs; sums in four independent pair accumulators. The
+      // fused form leaves every exponent off by the same t_ref - fl(t_ref) (t_ref the exact scaled
+      // reference max), which cancels in the normalisation but reaches 2^(ulp(m) / 2): once a row's
+      // reference max is 2^20 or more, the scores are scaled (rounded) first, so that the reference
+      // key's exponent is exactly 0 (warp-uniform; ordinary logits never take this branch).
+      bool scaled = !pos_scale;
+      if (pos_scale && __any_sync(0xffffffffu, fabsf(m_use) >= 0x1p20f)) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) v[c] *= sl2;
+        scaled = true;
+      }
+      const float sc = scaled ? 1.f : sl2;
       const uint64_t sc2 = tc::f2(sc, sc);
       const uint64_t nm2 = tc::f2(-m_use, -m_use);
       uint64_t acc2[4] = {tc::f2(0.f, 0.f), tc::f2(0.f, 0.f), tc::f2(0.f, 0.f), tc::f2(0.f, 0.f)};
@@ -584,7 +752,7 @@ __global__ void __launch_bounds__(384, 1)
         tc::f2_split(tc::f2_fma(tc::f2(v[2 * c], v[2 * c + 1]), sc2, nm2), a0, a1);
         const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
         acc2[c & 3] = tc::f2_add(acc2[c & 3], tc::f2(p0, p1));
-        pk[c] = Op::pack(p0, p1);
+        pk[c] = POp::pack(p0, p1);
       }
       {
         float s0, s1, s2, s3, s4, s5, s6, s7;
@@ -642,26 +810,32 @@ __global__ void __launch_bounds__(384, 1)
 
     // ---------------------------------------------------------------- segment epilogue
     // Both warpgroups finish the segment together, each on half of the head dims of both O
-    // accumulators: O = s_0 O_0 + s_1 O_1 with s_w = 2^(m_w - LSE) and LSE = log2(l_0 2^m_0 + l_1 2^m_1)
-    // (the base-2 log-sum-exp of the segment; m_w, l_w are warpgroup w's reference max and sum).
-    // Each warpgroup publishes its own log-sum-exp, then its scale, through shared memory; this needs
-    // only the softmax state, so it runs while the segment's last P V is still in flight.
+    // accumulators: O = s_0 O_0 + s_1 O_1 with s_w = 2^(m_w - M) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)),
+    // M = max(m_0, m_1) (m_w, l_w are warpgroup w's reference max and sum). The two exchange their
+    // values through shared memory; this needs only the softmax state, so it runs while the segment's
+    // last P V is still in flight.
     const bool have_keys = k_mine_last >= 0 && l_run > 0.f;
-    const float lse_mine = have_keys ? m_ref + __log2f(l_run) : -INFINITY;
-    sh->xs[wg][r] = lse_mine;
+    // first the reference maxima, then each warpgroup's sum weighted by 2^(m_w - M): no log2(l) is ever
+    // added to a max, which would lose it in rounding once |m| is large (logits of 2^20 and beyond)
+    const float m_mine = have_keys ? m_ref : -INFINITY;
+    sh->xs[wg][r] = m_mine;
     named_bar_sync(3, 256);
-    const float lse_other = sh->xs[wg ^ 1][r];
-    const float lmax = fmaxf(lse_mine, lse_other);
-    const float LSE =
-        lmax == -INFINITY ? -INFINITY : lmax + __log2f(fast_exp2(lse_mine - lmax) + fast_exp2(lse_other - lmax));
-    const float s_mine = have_keys ? fast_exp2(m_ref - LSE) : 0.f;
+    const float m_other = sh->xs[wg ^ 1][r];
+    const float Mx = fmaxf(m_mine, m_other);
+    const float f_mine = m_mine == -INFINITY ? 0.f : fast_exp2(m_mine - Mx);
+    const float f_other = m_other == -INFINITY ? 0.f : fast_exp2(m_other - Mx);
     named_bar_sync(3, 256);
-    sh->xs[wg][r] = s_mine;
+    sh->xs[wg][r] = f_mine * (have_keys ? l_run : 0.f);
     named_bar_sync(3, 256);
-    const float s_other = sh->xs[wg ^ 1][r];
-    const float s0 = wg == 0 ? s_mine : s_other;
-    const float s1 = wg == 0 ? s_other : s_mine;
-    const bool use0 = s0 > 0.f, use1 = s1 > 0.f;
+    const float ltot = f_mine * (have_keys ? l_run : 0.f) + sh->xs[wg ^ 1][r];
+    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+    const float LSE = ltot > 0.f ? Mx + __log2f(ltot) : -INFINITY;  // the segment's base-2 log-sum-exp
+    const float s_mine = f_mine * inv, s_other = f_other * inv;
+    const float s0r = wg == 0 ? s_mine : s_other;
+    const float s1r = wg == 0 ? s_other : s_mine;
+    const bool use0 = s0r > 0.f, use1 = s1r > 0.f;
+    const float s0 = s0r * vsc;  // e4m3 caches: V's scale joins O here
+    const float s1 = s1r * vsc;
     if (k_mine_last >= 0) {
       bool ok = (*abort_flag == 0);
       if (ok) ok = mbar_wait(pv_bar(k_mine_last), pv_par(k_mine_last), p.error_word);

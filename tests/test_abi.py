@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.taco_attn_version() == 6
+    assert lib.taco_attn_version() == 7
 
 
 def _attn_args(**over):
@@ -127,8 +127,8 @@ def _attn8_args(**over):
     (dict(ks=None), _lib.TACO_ERR_INVALID_ARG),
     (dict(vs=None), _lib.TACO_ERR_INVALID_ARG),
     (dict(q=None), _lib.TACO_ERR_INVALID_ARG),
-    (dict(D=64), _lib.TACO_ERR_UNSUPPORTED),          # e4m3 caches: head_dim 128 only
-    (dict(Hq=64, Hkv=2, C=4), _lib.TACO_ERR_UNSUPPORTED),  # 32 * 4 packed rows > 64
+    (dict(D=96), _lib.TACO_ERR_UNSUPPORTED),          # head_dim 64 or 128 only
+    (dict(Hq=129 * 2, Hkv=2, C=1), _lib.TACO_ERR_UNSUPPORTED),  # G > 128: neither kernel takes it
     (dict(dtype=3), _lib.TACO_ERR_INVALID_ARG),
     (dict(k=24), _lib.TACO_ERR_INVALID_ARG),
 ])
@@ -137,10 +137,14 @@ def test_e4m3_attention_rejects_bad_arguments_on_host(lib, over, status):
     assert lib.taco_attn_last_error().decode()
 
 
-def test_e4m3_attention_has_no_tensor_core_kernel(lib):
-    assert lib.taco_attn_set_option(_lib.TACO_OPT_KERNEL, 2) == _lib.TACO_OK
+@pytest.mark.parametrize("over", [dict(D=64), dict(Hq=64, Hkv=2, C=4)])
+def test_e4m3_mma_kernel_rejects_shapes_only_the_tensor_core_kernel_takes(lib, over):
+    """Forcing the mma.sync kernel (head_dim 128, <= 64 packed rows for e4m3) on head_dim 64 or on
+    32 x 4 packed rows is refused on the host; the automatic choice takes the tcgen05 kernel there."""
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_KERNEL, 1) == _lib.TACO_OK
     try:
-        assert lib.paged_tree_attention_e4m3(*_attn8_args()) == _lib.TACO_ERR_UNSUPPORTED
+        assert lib.paged_tree_attention_e4m3(*_attn8_args(**over)) == _lib.TACO_ERR_UNSUPPORTED
+        assert "mma.sync" in lib.taco_attn_last_error().decode()
     finally:
         assert lib.taco_attn_set_option(_lib.TACO_OPT_KERNEL, 0) == _lib.TACO_OK
 

@@ -87,21 +87,37 @@ def test_quantising_append_bit_exact(dtype, D, bs):
         assert codes[7] == 0xFE and codes[11] == 0x00 and codes[12] == 0x80 and codes[16] == 0x7F
 
 
-@pytest.mark.parametrize("grid", [0, 1, 3, 50])
+SHAPES = [
+    # Hq, Hkv, D, C, tree, bs, ctx
+    (32, 8, 128, 1, "chain", 16, ("uniform", 1, 700)),      # decode: 4 packed rows
+    (64, 8, 128, 4, "chain", 64, ("uniform", 100, 900)),    # 32 packed rows
+    (64, 8, 128, 8, "forest", 32, ("uniform", 8, 500)),     # 64 packed rows (tensor-core kernel)
+    (64, 8, 128, 16, "forest", 32, ("uniform", 8, 700)),    # 128 packed rows: the tree shape
+    (8, 1, 128, 5, "forest", 16, ("fixed", [5, 64, 65, 129])),
+    (32, 8, 64, 4, "chain", 16, ("uniform", 1, 600)),       # head_dim 64
+    (64, 8, 64, 16, "forest", 8, ("uniform", 8, 400)),
+]
+
+
+def _mma_possible(shape):
+    Hq, Hkv, D, C = shape[:4]
+    return D == 128 and (Hq // Hkv) * C <= 64
+
+
+@pytest.mark.parametrize("kernel,grid", [(0, 0), (0, 3), (0, 50), (1, 0), (2, 0), (2, 7)])
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
-@pytest.mark.parametrize("shape", [
-    # Hq, Hkv, C, tree, bs, ctx
-    (32, 8, 1, "chain", 16, ("uniform", 1, 700)),        # decode: 4 packed rows
-    (64, 8, 4, "chain", 64, ("uniform", 100, 900)),      # 32 packed rows
-    (64, 8, 8, "forest", 32, ("uniform", 8, 500)),       # 64 packed rows
-    (8, 1, 5, "forest", 16, ("fixed", [5, 64, 65, 129])),
-])
-def test_attention_over_e4m3_cache(shape, dtype, grid):
-    Hq, Hkv, C, tree, bs, ctx = shape
+@pytest.mark.parametrize("shape", SHAPES)
+def test_attention_over_e4m3_cache(shape, dtype, kernel, grid):
+    """Every shape on the automatic choice and on each kernel that takes it (1 = mma.sync with codes
+    widened in registers, 2 = tcgen05 with tiles widened once in shared memory), several grids."""
+    Hq, Hkv, D, C, tree, bs, ctx = shape
+    if kernel == 1 and not _mma_possible(shape):
+        pytest.skip("the mma.sync e4m3 kernel takes head_dim 128 and <= 64 packed rows")
     B = 4
-    spec = dict(dtype=dtype, B=B, Hq=Hq, Hkv=Hkv, D=128, bs=bs, C=C, tree=tree, ctx=ctx)
-    w = wl.make_workload(spec, seed=40 + C + Hq + bs)
+    spec = dict(dtype=dtype, B=B, Hq=Hq, Hkv=Hkv, D=D, bs=bs, C=C, tree=tree, ctx=ctx)
+    w = wl.make_workload(spec, seed=40 + C + Hq + bs + D)
     c8 = wl.make_e4m3_cache(w)
+    taco.set_option(taco.TACO_OPT_KERNEL, kernel)
     taco.set_option(taco.TACO_OPT_GRID_CTAS, grid)
     got = gpu_attention_e4m3(w, c8)
     ref = oracle_attention_e4m3(w, c8)
@@ -117,10 +133,13 @@ def test_empty_contexts_and_padding_rows_are_zero():
     assert_parity(got, oracle_attention_e4m3(w, c8), w)
 
 
-def test_query_magnitudes_far_from_one():
-    """bf16 queries with rows scaled by 2^40 .. 2^-40 and single huge or tiny elements: the kernel
-    rescales each query row into f16 range by a power of two and must still match."""
-    spec = dict(dtype="bf16", B=2, Hq=16, Hkv=2, D=128, bs=16, C=2, tree="chain", ctx=("fixed", [90, 300]))
+@pytest.mark.parametrize("Hq,C", [(16, 2), (64, 8)])
+def test_query_magnitudes_far_from_one(Hq, C):
+    """bf16 queries with rows scaled by 2^40 .. 2^-40 and single huge or tiny elements: the kernels
+    rescale each query row into f16 range by a power of two (in registers on the mma.sync kernel, 16
+    packed rows; in a pre-pass on the tcgen05 kernel, 64 packed rows) and must still match."""
+    spec = dict(dtype="bf16", B=2, Hq=Hq, Hkv=2 if Hq == 16 else 8, D=128, bs=16, C=C, tree="chain",
+                ctx=("fixed", [90, 300]))
     w = wl.make_workload(spec, seed=8)
     q = w.q.float()
     q[0, 0, 0] *= 2.0 ** 40
@@ -154,7 +173,7 @@ def test_append_then_attend_end_to_end():
     assert_parity(out.cpu(), ref, w)
 
 
-@pytest.mark.parametrize("name", ["decode", "chain", "long"])
+@pytest.mark.parametrize("name", ["decode", "chain", "tree", "long"])
 def test_full_size_workloads_sampled_rows(name):
     """The bench's workloads at full size with e4m3 caches, in the default launch configuration:
     24 sampled rows against the oracle."""
@@ -169,3 +188,29 @@ def test_full_size_workloads_sampled_rows(name):
     rows = sorted(rows)
     assert_parity(got, oracle_attention_e4m3(w, c8, rows=rows), w, rows=rows)
     assert torch.isfinite(got.float()).all()
+
+
+@pytest.mark.parametrize("spec", [
+    dict(dtype="bf16", B=3, Hq=64, Hkv=8, D=128, bs=16, C=8, tree="chain", ctx=("uniform", 9, 900)),
+    dict(dtype="fp16", B=3, Hq=32, Hkv=8, D=64, bs=32, C=4, tree="forest", ctx=("uniform", 5, 500)),
+    dict(dtype="bf16", B=4, Hq=32, Hkv=8, D=128, bs=16, C=1, tree="chain", ctx=("uniform", 1, 300)),
+])
+def test_append_and_attend_in_one_call(spec):
+    """paged_tree_attention_append_e4m3: the candidates' rows quantised into slots P_b .. L_b - 1, then
+    the attention, in one call; the caches equal the quantising-append oracle byte for byte and the
+    output the attention oracle over them."""
+    w = wl.make_workload(spec, seed=77, candidates_in_cache=False)
+    c8 = wl.make_e4m3_cache(w)
+    d, g8 = w.to("cuda"), c8.to("cuda")
+    out = torch.full_like(d.q, float("nan"))
+    taco.paged_tree_attention_e4m3(d.q, g8.k_cache, g8.v_cache, g8.k_scale, g8.v_scale, d.block_tables,
+                                   d.context_lens, d.num_candidates, d.tree_mask, w.scale, out=out,
+                                   k_new=d.k_new, v_new=d.v_new)
+    assert taco.check_device() == 0
+    rk, rv = fp8.paged_kv_append_e4m3(wl.to_numpy_bits(w.k_new), wl.to_numpy_bits(w.v_new), w.dtype,
+                                      w.block_tables.numpy(), w.slot_offsets.numpy(), c8.k_scale.numpy(),
+                                      c8.v_scale.numpy(), c8.k_cache.numpy(), c8.v_cache.numpy())
+    assert np.array_equal(g8.k_cache.cpu().numpy(), rk)
+    assert np.array_equal(g8.v_cache.cpu().numpy(), rv)
+    ref = oracle_attention_e4m3(w, c8, k_cache=torch.from_numpy(rk), v_cache=torch.from_numpy(rv))
+    assert_parity(out.cpu(), ref, w)

@@ -80,6 +80,29 @@ def test_split_kv_partitions_agree(grid, kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("grid", [0, 5])
+def test_query_magnitudes_far_from_one(kernel, grid):
+    """Query rows scaled by 2^40 and 2^-40, one huge element, one zero row: logits of 2^40 leave a
+    float32 ulp of 2^16, so any step that adds log2 of a softmax sum to a maximum would lose the sum.
+    The split grid runs the partials and their merge on the same rows."""
+    spec = dict(dtype="bf16", B=2, Hq=64, Hkv=8, D=128, bs=16, C=8, tree="forest", ctx=("fixed", [300, 700]))
+    w = wl.make_workload(spec, seed=8)
+    q = w.q.float()
+    q[0, 0, 0] *= 2.0 ** 40
+    q[0, 0, 1] *= 2.0 ** -40
+    q[0, 1, 2] *= 2.0 ** 20
+    q[1, 0, 3] = 0.0
+    q[1, 0, 4, 7] = 3e4
+    q[1, 2, 9] *= 2.0 ** 30
+    w.q = q.to(torch.bfloat16)
+    ref, _, _ = oracle_step(w, append=False)
+    taco.set_option(taco.TACO_OPT_GRID_CTAS, grid)
+    taco.set_option(taco.TACO_OPT_KERNEL, kernel)
+    out, _, _ = gpu_step(w, append=False)
+    assert_parity(out, ref, w)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 def test_block_permutation_gives_bitwise_identical_output(kernel):
     taco.set_option(taco.TACO_OPT_KERNEL, kernel)
     spec = dict(dtype="bf16", B=4, Hq=32, Hkv=8, D=128, bs=16, C=4, tree="forest", ctx=("uniform", 50, 600))
