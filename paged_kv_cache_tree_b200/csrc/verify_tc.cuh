@@ -343,24 +343,36 @@ __global__ void __launch_bounds__(384, 1)
         if (go) {
           const uint8_t* src = raw + rs * Cfg::kRawBytes;
           uint8_t* dst = conv + cs * Cfg::kTensorBytes;
-          constexpr int CPR = D / 16;  // 16-code chunks per key row
-#pragma unroll 4
-          for (int idx = lane; idx < TK * CPR; idx += 32) {
-            const int row = idx / CPR;
-            const int c = idx % CPR;
-            const uint4 v = lds_v4(smem_addr(src + row * D + c * 16));
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t h[8];
+          constexpr int CPR = D / 16;          // 16-code chunks per key row
+          constexpr int NCH = TK * CPR / 32;   // chunks per lane and tile (32 or 16)
+          constexpr int BATCH = 8;             // chunks whose loads are issued before any is used
+          static_assert(NCH % BATCH == 0, "conversion batches");
+#pragma unroll 1
+          for (int b0 = 0; b0 < NCH; b0 += BATCH) {
+            uint4 v[BATCH];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              h[2 * q] = e4m3x2_to_f16x2(w[q] & 0xffffu);
-              h[2 * q + 1] = e4m3x2_to_f16x2(w[q] >> 16);
+            for (int j = 0; j < BATCH; ++j) {
+              const int idx = (b0 + j) * 32 + lane;
+              v[j] = lds_v4(smem_addr(src + (idx / CPR) * D + (idx % CPR) * 16));
             }
-            // head dims [16c, 16c + 16) = 16-byte chunks 2(c % 4), 2(c % 4) + 1 of panel c / 4, swizzled
-            uint8_t* prow = dst + (c >> 2) * Cfg::kPanelBytes + row * 128;
-            const int j0 = 2 * (c & 3);
-            *reinterpret_cast<uint4*>(prow + ((j0 ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<uint4*>(prow + (((j0 + 1) ^ (row & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+#pragma unroll
+            for (int j = 0; j < BATCH; ++j) {
+              const int idx = (b0 + j) * 32 + lane;
+              const int row = idx / CPR;
+              const int c = idx % CPR;
+              const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+              uint32_t h[8];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                h[2 * q] = e4m3x2_to_f16x2(w[q] & 0xffffu);
+                h[2 * q + 1] = e4m3x2_to_f16x2(w[q] >> 16);
+              }
+              // head dims [16c, 16c + 16) = 16-byte chunks 2(c % 4), 2(c % 4) + 1 of panel c / 4, swizzled
+              uint8_t* prow = dst + (c >> 2) * Cfg::kPanelBytes + row * 128;
+              const int j0 = 2 * (c & 3);
+              *reinterpret_cast<uint4*>(prow + ((j0 ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+              *reinterpret_cast<uint4*>(prow + (((j0 + 1) ^ (row & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+            }
           }
           fence_proxy_async_smem();
         }
