@@ -8,6 +8,7 @@ from ._lib import (  # noqa: F401
     TACO_OPT_GRID_CTAS,
     TACO_OPT_KERNEL,
     TACO_OPT_L2_PREFETCH,
+    TACO_OPT_TEST_STALL,
     TacoError,
     check_device,
     check_noalloc,

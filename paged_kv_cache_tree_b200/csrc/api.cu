@@ -59,6 +59,7 @@ int g_sm_count[kMaxDevices];
 int64_t g_opt_grid = 0;
 int64_t g_opt_kernel = 0;
 int64_t g_opt_prefetch = -1;  // -1 = the kernel's default distance
+int64_t g_opt_stall = 0;      // test knob: 0 = off, t + 1 = CTA 0 leaves tile t unarmed (mma.sync kernel)
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -222,6 +223,11 @@ taco_status taco_attn_set_option(int32_t key, int64_t value) {
     g_opt_kernel = value;
     return TACO_OK;
   }
+  if (key == TACO_OPT_TEST_STALL) {
+    if (value < 0 || value > (1 << 30)) return fail(TACO_ERR_INVALID_ARG, "stall tile must be in [0, 2^30]");
+    g_opt_stall = value;
+    return TACO_OK;
+  }
   if (key == TACO_OPT_L2_PREFETCH) {
     if (value < -1 || value > 64) return fail(TACO_ERR_INVALID_ARG, "prefetch distance must be in [-1, 64]");
     g_opt_prefetch = value;
@@ -353,6 +359,10 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
   p.row_groups = row_groups;
   p.cands_per_group = cands_per_group;
   p.tile_keys = tile;
+  if (g_opt_stall > 0 && !use_tc) {
+    p.stall_tile = static_cast<int>(g_opt_stall);
+    p.wait_limit_ns = 20000000ull;  // 20 ms
+  }
   p.l2_prefetch_tiles = static_cast<int>(
       g_opt_prefetch >= 0 ? g_opt_prefetch : (use_tc ? taco::kTcPrefetchTiles : taco::kMmaPrefetchTiles));
   p.k_scale = k_scale;

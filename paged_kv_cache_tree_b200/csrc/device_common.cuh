@@ -42,6 +42,11 @@ struct VerifyParams {
   const float* k_scale;  // e4m3 caches: per-KV-head scales (K value = code * k_scale[h]); else null
   const float* v_scale;
   const float* q_scale;  // e4m3 caches on the tcgen05 path: the f16 query rows' scale per row, or null
+  // test knobs of the mma.sync kernel (zero = off): a pipeline wait gives up after wait_limit_ns
+  // (0 = kWaitLimitNs); with stall_tile = t + 1, CTA 0's producers leave tile t's stage unarmed, so
+  // that a consumer's bounded wait runs out
+  uint64_t wait_limit_ns;
+  int stall_tile;
   // fused append (16-bit caches, units of <= 16 rows): candidate i's new K/V rows [B, C, Hkv, D] go to
   // logical slot P_b + i of these caches as the verify reads them; null = the caches are complete
   const void* k_new;
@@ -118,14 +123,16 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
   return done != 0;
 }
 
-// Wait for the phase with the given parity to complete. Gives up after kWaitLimitNs, sets the
-// timeout bit in the error word and returns false (the caller then leaves its loop).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* error_word) {
+// Wait for the phase with the given parity to complete. Gives up after limit_ns (kWaitLimitNs when
+// 0), sets the timeout bit in the error word and returns false (the caller then leaves its loop).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* error_word,
+                                          uint64_t limit_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t limit = limit_ns ? limit_ns : kWaitLimitNs;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1; it < (1u << 30); ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) break;
+    if ((it & 255u) == 0u && global_timer_ns() - t0 > limit) break;
   }
   atomicOr(error_word, TACO_DEVERR_WAIT_TIMEOUT);
   return false;

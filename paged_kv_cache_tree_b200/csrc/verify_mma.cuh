@@ -205,12 +205,15 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
         }
         const uint32_t okmask = __ballot_sync(0xffffffffu, ok);
         const uint32_t bytes = __popc(okmask) * chunk_bytes * Cfg::kPanels;
+        // test knob: both producers of CTA 0 leave this stage unarmed (no arrival, no copy)
+        const bool stall = p.stall_tile != 0 && blockIdx.x == 0 && kt == p.stall_tile - 1;
         bool go = true;
         if (lane == 0) {
-          go = (*abort_flag == 0) && mbar_wait(smem_addr(empty_bar + stage), phase ^ 1u, p.error_word);
+          go = (*abort_flag == 0) && mbar_wait(smem_addr(empty_bar + stage), phase ^ 1u, p.error_word, p.wait_limit_ns);
           if (!go) *abort_flag = 1;
-          mbar_arrive_expect_tx(smem_addr(full_bar + stage), go ? bytes : 0u);
+          if (!stall) mbar_arrive_expect_tx(smem_addr(full_bar + stage), go ? bytes : 0u);
         }
+        go = go && !stall;
         go = __shfl_sync(0xffffffffu, go, 0);
         if (go && ok) {
           const uint32_t dst = smem_addr(stages + stage * Cfg::kStageBytes) + (is_k ? 0u : Cfg::kTensorBytes) +
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
         // the most recent use of stage s completed phase (uses-1); waiting for its parity is
         // immediate when it has landed (or when the stage was never used)
         int uses_parity_phase = (s < stage) ? phase : (phase ^ 1u);
-        mbar_wait(smem_addr(full_bar + s), static_cast<uint32_t>(uses_parity_phase), p.error_word);
+        mbar_wait(smem_addr(full_bar + s), static_cast<uint32_t>(uses_parity_phase), p.error_word, p.wait_limit_ns);
       }
     }
     return;
@@ -379,7 +382,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
       const int key0 = tl * Cfg::kTile;
       bool ready = false;
       if (*abort_flag == 0) {
-        ready = mbar_wait(smem_addr(full_bar + stage), phase, p.error_word);
+        ready = mbar_wait(smem_addr(full_bar + stage), phase, p.error_word, p.wait_limit_ns);
         if (!ready) *abort_flag = 1;
       }
       const uint32_t kbase = smem_addr(stages + stage * Cfg::kStageBytes);

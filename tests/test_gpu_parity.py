@@ -252,3 +252,37 @@ def test_two_streams_overlap_without_sharing_a_workspace():
     for k in range(2):
         want, _, _ = oracle_step(ws[k], append=False)
         assert_parity(outs[k].cpu(), want, ws[k])
+
+
+def test_bounded_pipeline_wait_runs_out_and_reports():
+    """The first CTA's producers leave one stage unarmed (TACO_OPT_TEST_STALL, mma.sync kernel), so a
+    consumer's bounded wait on it runs out: the call still returns, the stream's error word carries
+    TACO_DEVERR_WAIT_TIMEOUT (reading it also clears the split-KV counters), and the next clean call
+    gives the same bits as a clean call before the stall."""
+    spec = dict(dtype="bf16", B=4, Hq=32, Hkv=8, D=128, bs=16, C=1, tree="chain", ctx=("uniform", 600, 1500))
+    w = wl.make_workload(spec, seed=12)
+    d = w.to("cuda")
+    taco.set_option(taco.TACO_OPT_KERNEL, 1)
+    taco.set_option(taco.TACO_OPT_GRID_CTAS, 7)   # every unit split: the counters take part too
+
+    def call():
+        out = torch.full_like(d.q, float("nan"))
+        taco.paged_tree_attention(d.q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, d.num_candidates,
+                                  d.tree_mask, w.scale, out=out)
+        return out
+
+    before = call()
+    assert taco.check_device() == 0
+    ref, _, _ = oracle_step(w, append=False)
+    assert_parity(before.cpu(), ref, w)
+    try:
+        taco.set_option(taco.TACO_OPT_TEST_STALL, 2)   # CTA 0's second tile
+        call()
+        with pytest.raises(taco.TacoError) as ei:
+            taco.check_device()
+        assert "pipeline wait timed out" in str(ei.value)
+    finally:
+        taco.set_option(taco.TACO_OPT_TEST_STALL, 0)
+    after = call()
+    assert taco.check_device() == 0
+    assert torch.equal(after.view(torch.int16), before.view(torch.int16))
