@@ -383,6 +383,9 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
       e = kv8 ? taco::launch_append_e4m3(a, k_scale, v_scale, static_cast<cudaStream_t>(stream))
               : taco::launch_append(a, static_cast<cudaStream_t>(stream));
       if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+      // the verify follows the append directly (16-bit caches: no query conversion in between), so
+      // it may read everything but the appended slots before the append ends
+      p.late_wait = kv8 ? 0 : 1;
     }
   }
   // after the append (a plain launch: it starts once the append has finished, and the verify's

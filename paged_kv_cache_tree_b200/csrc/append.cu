@@ -25,7 +25,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   } else {
     const int i = static_cast<int>(bi % a.C);
     const int n = __ldg(a.num_candidates + b), L = __ldg(a.context_lens + b);
-    s = (i < n && n <= L) ? L - n + i : -1;
+    s = (i < n && n <= a.C && n <= L) ? L - n + i : -1;  // slots [L - n, L) with n <= C
   }
   if (s < 0) return;
   if (s >= a.max_blocks * a.bs) {
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(256) append_e4m3_kernel(AppendArgs a, const fl
   } else {
     const int i = static_cast<int>(bi % a.C);
     const int n = __ldg(a.num_candidates + b), L = __ldg(a.context_lens + b);
-    s = (i < n && n <= L) ? L - n + i : -1;
+    s = (i < n && n <= a.C && n <= L) ? L - n + i : -1;  // slots [L - n, L) with n <= C
   }
   if (s < 0) return;
   if (s >= a.max_blocks * a.bs) {

@@ -47,6 +47,11 @@ struct VerifyParams {
   // that a consumer's bounded wait runs out
   uint64_t wait_limit_ns;
   int stall_tile;
+  // 1 when the grid this launch depends on (programmatic launch) is this library's append kernel with
+  // derived slots, launched by the same call: it writes only cache slots [L_b - C, L_b) of each
+  // sequence, and everything else the verify reads was complete before it started. The producers then
+  // wait for it only before loading a tile that reaches key L_b - C, instead of at the start.
+  int late_wait;
   // fused append (16-bit caches, units of <= 16 rows): candidate i's new K/V rows [B, C, Hkv, D] go to
   // logical slot P_b + i of these caches as the verify reads them; null = the caches are complete
   const void* k_new;

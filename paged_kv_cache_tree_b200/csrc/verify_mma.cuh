@@ -133,8 +133,9 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
     }
     fence_mbar_init();
   }
-  // inputs (and the cache an append just wrote) are read only after the grids this launch depends on
-  grid_dependency_wait();
+  // inputs (and the cache an append just wrote) are read only after the grids this launch depends on;
+  // after this library's own append only the producers wait, before the tiles that hold its slots
+  if (!p.late_wait) grid_dependency_wait();
   if (warp == Cfg::kConsumerWarps) {
     SchedStart s = schedule_start(p, blockIdx.x, gridDim.x);
     if (lane == 0) {
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
     TilePrefetcher<Cfg::kPanels, Cfg::kColsPerPanel> pf;
     if (pf_ahead > 0) pf.init(p, b, base_b, lo, hi, Cfg::kStages);
     int64_t kt = 0;  // tile ordinal within the CTA
+    bool dep_done = !p.late_wait;
     while (t < hi) {
       const int g = j / p.row_groups;
       const int tend = static_cast<int>(Tb < tile + (hi - t) ? Tb : tile + (hi - t));
@@ -215,6 +217,10 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
         }
         go = go && !stall;
         go = __shfl_sync(0xffffffffu, go, 0);
+        if (!dep_done && key0 + Cfg::kTile > L - p.C) {  // the tile may hold slots the append wrote
+          grid_dependency_wait();
+          dep_done = true;
+        }
         if (go && ok) {
           const uint32_t dst = smem_addr(stages + stage * Cfg::kStageBytes) + (is_k ? 0u : Cfg::kTensorBytes) +
                                lane * chunk_bytes;

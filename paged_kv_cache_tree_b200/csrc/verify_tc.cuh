@@ -218,8 +218,11 @@ __global__ void __launch_bounds__(384, 1)
     tc::tmem_alloc(smem_addr(&sh->tmem_base), Cfg::kTmemCols);
     tc::tmem_relinquish();
   }
-  // inputs (and the cache an append just wrote) are read only after the grids this launch depends on
-  grid_dependency_wait();
+  // inputs (and the cache an append just wrote) are read only after the grids this launch depends on;
+  // after this library's own append (16-bit caches) only the producers wait, before the tiles that
+  // hold its slots
+  const bool late_wait = !KV8 && p.late_wait;
+  if (!late_wait) grid_dependency_wait();
   if (warp == 0) {
     SchedStart s0 = schedule_start(p, blockIdx.x, gridDim.x);
     if (lane == 0) {
@@ -414,6 +417,7 @@ __global__ void __launch_bounds__(384, 1)
     const int pf_ahead = is_k ? 0 : p.l2_prefetch_tiles;
     TilePrefetcher<Cfg::kPanels, 64> pf;
     if (pf_ahead > 0) pf.init(p, sh->b, sh->base_b, lo, hi, SV);
+    bool dep_done = !late_wait;
     while (cur.valid()) {
       const int g = cur.j / p.row_groups;
       const int rg = cur.j % p.row_groups;
@@ -468,6 +472,10 @@ __global__ void __launch_bounds__(384, 1)
         }
         const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, ok)) * chunk_bytes * Cfg::kPanels;
         const int row = (blk * p.Hkv + g) * p.bs + (key0 + lane * rpc) % p.bs;
+        if (!dep_done && key0 + TK > L - p.C) {  // the tile may hold slots the append wrote
+          grid_dependency_wait();
+          dep_done = true;
+        }
         if (is_k) {  // K
           const int st = static_cast<int>(k % SK);
           bool go = true;

@@ -51,7 +51,7 @@ def test_argmax_full_vocabulary_bit_exact_and_finds_the_planted_index():
 
 
 @pytest.mark.parametrize("dtype,V,offset", [("bf16", 128256, 0), ("fp16", 32000, 0), ("bf16", 1001, 0),
-                                            ("fp16", 4096, 1), ("bf16", 8, 0), ("bf16", 1, 0)])
+                                            ("fp16", 4096, 1), ("bf16", 128256, 1), ("bf16", 8, 0), ("bf16", 1, 0)])
 def test_argmax_ties_nans_and_infinities(dtype, V, offset):
     g = torch.Generator().manual_seed(V + offset)
     rows = 24
@@ -161,3 +161,32 @@ def test_argmax_signed_zeros_tie_and_maxima_anywhere_in_the_row():
     assert got[0] == 0 and got[1] == 3
     # the scratch is left clean: the same call again gives the same answer
     assert np.array_equal(taco.logits_argmax(x.cuda()).cpu().numpy(), got)
+
+
+@pytest.mark.parametrize("rows", [1, 3, 16, 64, 128, 300, 2000])
+def test_argmax_many_row_counts_ties_far_apart(rows):
+    """Random rows of the full vocabulary, from one row to more rows than SMs: equal maxima at two
+    neighbouring positions (spread over the row) or far apart, where the smaller index must win, and
+    single maxima in the last or the first element."""
+    V = 128256
+    nvec = V // 8
+    edges = sorted({k * ((nvec + s - 1) // s) * 8 for s in (2, 4, 8) for k in range(1, s)})
+    g = torch.Generator().manual_seed(rows)
+    x = (torch.rand(rows, V, generator=g) * 2 - 1).to(torch.bfloat16)
+    for r in range(rows):
+        kind = r % 4
+        if kind == 0:
+            e = edges[(r // 4) % len(edges)]
+            x[r, e - 1] = 3.0
+            x[r, e] = 3.0              # the chunk before the edge must win
+        elif kind == 1:
+            x[r, V - 1] = 3.0
+        elif kind == 2:
+            x[r, 0] = 3.0
+        else:
+            e = edges[(r // 4) % len(edges)]
+            x[r, e] = 3.0
+            x[r, V - 1] = 3.0          # the same value later in the row loses
+    got = taco.logits_argmax(x.cuda()).cpu().numpy()
+    want = oracle_argmax(x, "bf16")
+    assert np.array_equal(got, want)

@@ -56,8 +56,11 @@ def test_fused_append_then_attention_matches_oracle(case, grid):
     assert_parity(out, ref, w)
 
 
-def test_full_size_decode_sampled_rows():
-    w = wl.make_workload("decode", candidates_in_cache=False)
+@pytest.mark.parametrize("name", ["decode", "chain", "tree", "long"])
+def test_full_size_sampled_rows(name):
+    """The bench's call at full size: decode fuses the append; chain, tree and long run the append kernel,
+    and the verify waits for it only before the tiles that hold the candidates' slots."""
+    w = wl.make_workload(name, candidates_in_cache=False)
     out, kc, vc = fused_step(w)
     so, bt = w.slot_offsets, w.block_tables
     for b in range(w.B):
@@ -67,8 +70,12 @@ def test_full_size_decode_sampled_rows():
             assert torch.equal(kc[blk, :, s % w.bs].view(torch.int16), w.k_new[b, i].view(torch.int16))
             assert torch.equal(vc[blk, :, s % w.bs].view(torch.int16), w.v_new[b, i].view(torch.int16))
     rng = np.random.default_rng(4)
-    rows = sorted({(int(rng.integers(w.B)), 0, int(rng.integers(w.Hq))) for _ in range(24)} | {(0, 0, 0)})
-    w_after = wl.make_workload("decode", candidates_in_cache=True)
+    rows = set()
+    for _ in range(24):
+        b = int(rng.integers(w.B))
+        rows.add((b, int(rng.integers(max(1, int(w.num_candidates[b])))), int(rng.integers(w.Hq))))
+    rows = sorted(rows | {(0, 0, 0)})
+    w_after = wl.make_workload(name, candidates_in_cache=True)
     ref, _, _ = oracle_step(w_after, append=False, rows=rows)
     assert_parity(out, ref, w, rows=rows)
     assert torch.isfinite(out.float()).all()
