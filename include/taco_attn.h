@@ -411,6 +411,10 @@ void taco_attn_release_workspace(void);
 #define TACO_OPT_KERNEL 2      /* 0 = automatic, 1 = mma.sync path, 2 = tcgen05 path (where built) */
 #define TACO_OPT_L2_PREFETCH 3 /* key tiles of K/V the verify asks L2 to fetch ahead of its shared-memory
                                   loads: -1 = the kernel's default, 0 = none, up to 64 */
+#define TACO_OPT_SEG_COST 5    /* work split of the verify: key tiles each (sequence, KV head, row group)
+                                  unit counts on top of its own, for the cost of starting and finishing
+                                  it, when the units' tiles are divided between CTAs: -1 = the kernel's
+                                  default, 0 = an equal split of the tiles, up to 64 */
 #define TACO_OPT_TEST_STALL 4  /* test knob for the bounded pipeline waits, mma.sync verify kernel only:
                                   0 = off (default); t + 1 = the first CTA's producers never arm the
                                   stage of its tile t, so that a consumer's wait runs out after 20 ms,

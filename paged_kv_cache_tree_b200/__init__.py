@@ -9,6 +9,7 @@ from ._lib import (  # noqa: F401
     TACO_OPT_KERNEL,
     TACO_OPT_L2_PREFETCH,
     TACO_OPT_TEST_STALL,
+    TACO_OPT_SEG_COST,
     TacoError,
     check_device,
     check_noalloc,

@@ -29,6 +29,7 @@ TACO_OPT_GRID_CTAS = 1
 TACO_OPT_KERNEL = 2
 TACO_OPT_L2_PREFETCH = 3
 TACO_OPT_TEST_STALL = 4
+TACO_OPT_SEG_COST = 5
 
 EXPORTED = (
     "paged_tree_attention",

@@ -60,6 +60,7 @@ int64_t g_opt_grid = 0;
 int64_t g_opt_kernel = 0;
 int64_t g_opt_prefetch = -1;  // -1 = the kernel's default distance
 int64_t g_opt_stall = 0;      // test knob: 0 = off, t + 1 = CTA 0 leaves tile t unarmed (mma.sync kernel)
+int64_t g_opt_seg_cost = -1;  // -1 = the kernel's default segment cost of the work split
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -233,6 +234,11 @@ taco_status taco_attn_set_option(int32_t key, int64_t value) {
     g_opt_prefetch = value;
     return TACO_OK;
   }
+  if (key == TACO_OPT_SEG_COST) {
+    if (value < -1 || value > 64) return fail(TACO_ERR_INVALID_ARG, "segment cost must be in [-1, 64]");
+    g_opt_seg_cost = value;
+    return TACO_OK;
+  }
   return fail(TACO_ERR_INVALID_ARG, "unknown option key %d", key);
 }
 
@@ -363,6 +369,8 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
     p.stall_tile = static_cast<int>(g_opt_stall);
     p.wait_limit_ns = 20000000ull;  // 20 ms
   }
+  p.seg_cost = static_cast<int>(g_opt_seg_cost >= 0 ? g_opt_seg_cost
+                                : (use_tc ? taco::tc_seg_cost(cands_per_group * G) : taco::mma_seg_cost(rows)));
   p.l2_prefetch_tiles = static_cast<int>(
       g_opt_prefetch >= 0 ? g_opt_prefetch : (use_tc ? taco::kTcPrefetchTiles : taco::kMmaPrefetchTiles));
   p.k_scale = k_scale;

@@ -20,6 +20,13 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a pipeline wait gives up af
 // default L2 prefetch distances (key tiles past the latest load) of the two verify kernels
 constexpr int kTcPrefetchTiles = 0;
 constexpr int kMmaPrefetchTiles = 0;
+// Default segment cost of the work split (see the schedule below), in key tiles of the kernel, from
+// the packed query rows of a unit: starting and finishing a segment (query load, epilogue, partial
+// write and merge) grows with the rows, a tile's load time does not. Measured best on B200: 2 for
+// 8-row and 5 for 32-row units on the mma.sync kernel (64-key tiles), 2-3 for 64-row and 3-5 for
+// 128-row units on the tcgen05 kernel (128-key tiles).
+inline int mma_seg_cost(int rows) { return 1 + rows / 8; }
+inline int tc_seg_cost(int rows) { return 1 + rows / 64; }
 
 struct VerifyParams {
   const void* q;
@@ -52,6 +59,7 @@ struct VerifyParams {
   // sequence, and everything else the verify reads was complete before it started. The producers then
   // wait for it only before loading a tile that reaches key L_b - C, instead of at the start.
   int late_wait;
+  int seg_cost;          // virtual tiles per unit in the work split (see the schedule below); 0 = equal split
   // fused append (16-bit caches, units of <= 16 rows): candidate i's new K/V rows [B, C, Hkv, D] go to
   // logical slot P_b + i of these caches as the verify reads them; null = the caches are complete
   const void* k_new;
@@ -272,8 +280,14 @@ struct MmaOp<__half> {
 //
 // Work unit u = (b, kv head g, row group rg), ordered u = (b * Hkv + g) * RG + rg. Unit u holds
 // T_b = max(1, ceil(L_b / tile_keys)) key tiles (an empty sequence still gets one tile, which
-// writes its zero rows). All units' tiles are concatenated into one range [0, W); CTA c of the nC
-// working CTAs takes tiles [c*W/nC, (c+1)*W/nC). A unit that falls into several CTAs' ranges is
+// writes its zero rows). All units' tiles are concatenated into one range of real tiles [0, Wr).
+// The split between CTAs is made in a weighted copy of that range: unit u there spans seg_cost
+// virtual tiles (the cost of starting and finishing a segment: loading Q, the epilogue, the arrival)
+// followed by its T_b real tiles, so it starts at weight S_u = (first real tile of u) + seg_cost * u
+// and the total is W = Wr + seg_cost * units. CTA c of the nC working CTAs takes the weights
+// [c*W/nC, (c+1)*W/nC), that is the real tiles from the first one at or after weight c*W/nC up to
+// the first one at or after (c+1)*W/nC. A CTA whose range crosses many unit starts thus gets fewer
+// real tiles; seg_cost = 0 is the plain equal split. A unit that falls into several CTAs' ranges is
 // split: each piece writes a partial (normalised output + log-sum-exp), and the CTA that arrives
 // last on the unit's counter combines them. Since each CTA's range is contiguous, only its first
 // and last piece can be partial, so CTA c owns two partial slots: 2c (its first piece) and 2c+1.
@@ -306,59 +320,109 @@ __device__ __forceinline__ int clamp_candidates(const VerifyParams& p, int b, in
 
 __device__ __forceinline__ int tiles_of(int L, int tile) { return L <= 0 ? 1 : (L + tile - 1) / tile; }
 
-// first CTA (of nC over W tiles) whose range contains tile t
-__device__ __forceinline__ int cta_of_tile(int64_t t, int64_t W, int64_t nC) {
-  return static_cast<int>(((t + 1) * nC - 1) / W);
+// the CTA (of nC over total weight W) whose weight range contains weight w
+__device__ __forceinline__ int cta_of_tile(int64_t w, int64_t W, int64_t nC) {
+  return static_cast<int>(((w + 1) * nC - 1) / W);
+}
+
+// The CTAs holding the first and the last real tile of unit u (global ordinal), whose first real
+// tile is unit_base and which has Tb tiles, and whether the first of them reaches the unit from an
+// earlier unit (then the unit's piece is in its second partial slot).
+struct UnitCtas {
+  int c_first, c_last;
+  bool first_odd;
+};
+__device__ __forceinline__ UnitCtas unit_ctas(const VerifyParams& p, int64_t unit_base, int Tb, int64_t u,
+                                              int64_t W, int nC) {
+  const int64_t S = unit_base + static_cast<int64_t>(p.seg_cost) * u;  // weight where the unit starts
+  UnitCtas r;
+  r.c_first = cta_of_tile(S + p.seg_cost, W, nC);
+  r.c_last = cta_of_tile(S + p.seg_cost + Tb - 1, W, nC);
+  r.first_odd = static_cast<int64_t>(r.c_first) * W / nC < S;
+  return r;
 }
 
 struct SchedStart {
-  int64_t W;        // total tiles
+  int64_t W;        // total weight (real tiles + seg_cost per unit)
   int nC;           // working CTAs
-  int64_t lo, hi;   // this CTA's tile range
+  int64_t lo, hi;   // this CTA's range of real tiles
   int b;            // sequence of the first unit
   int64_t base_b;   // first tile of sequence b's units
 };
+
+// The first real tile at or after weight A (< W), with the sequence holding it and that sequence's
+// first tile. Computed by one full warp; every lane returns the same values.
+struct SchedPoint {
+  int64_t t;
+  int b;
+  int64_t base_b;
+};
+__device__ __forceinline__ SchedPoint schedule_locate(const VerifyParams& p, int64_t A) {
+  const int lane = threadIdx.x & 31;
+  const int HR = p.Hkv * p.row_groups;
+  const int c = p.seg_cost;
+  int64_t run_w = 0, run_r = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    const int Tb = b < p.B ? tiles_of(clamp_context(p, b, false), p.tile_keys) : 0;
+    const int64_t mine_r = static_cast<int64_t>(Tb) * HR;
+    const int64_t mine_w = b < p.B ? static_cast<int64_t>(Tb + c) * HR : 0;
+    int64_t incl_r = mine_r, incl_w = mine_w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t vr = __shfl_up_sync(0xffffffffu, incl_r, o);
+      const int64_t vw = __shfl_up_sync(0xffffffffu, incl_w, o);
+      if (lane >= o) {
+        incl_r += vr;
+        incl_w += vw;
+      }
+    }
+    const int64_t excl_w = run_w + incl_w - mine_w;
+    const int64_t excl_r = run_r + incl_r - mine_r;
+    const bool here = b < p.B && excl_w <= A && A < run_w + incl_w;
+    const uint32_t ball = __ballot_sync(0xffffffffu, here);
+    if (ball) {
+      const int src = __ffs(ball) - 1;
+      SchedPoint r;
+      r.b = b0 + src;
+      r.base_b = __shfl_sync(0xffffffffu, excl_r, src);
+      const int64_t off = A - __shfl_sync(0xffffffffu, excl_w, src);  // weight offset into sequence b
+      const int T = __shfl_sync(0xffffffffu, Tb, src);
+      const int64_t jj = off / (T + c), in = off % (T + c);
+      r.t = r.base_b + jj * T + (in > c ? in - c : 0);
+      return r;
+    }
+    run_w += __shfl_sync(0xffffffffu, incl_w, 31);
+    run_r += __shfl_sync(0xffffffffu, incl_r, 31);
+  }
+  SchedPoint r;  // A at or past the end
+  r.t = run_r;
+  r.b = p.B;
+  r.base_b = run_r;
+  return r;
+}
 
 // Computed by one full warp; every lane returns the same values.
 __device__ __forceinline__ SchedStart schedule_start(const VerifyParams& p, int cta, int grid) {
   const int lane = threadIdx.x & 31;
   const int HR = p.Hkv * p.row_groups;
-  int64_t W = 0;
-  for (int b = lane; b < p.B; b += 32) W += static_cast<int64_t>(tiles_of(clamp_context(p, b, false), p.tile_keys)) * HR;
+  int64_t Wr = 0;
+  for (int b = lane; b < p.B; b += 32) Wr += static_cast<int64_t>(tiles_of(clamp_context(p, b, false), p.tile_keys)) * HR;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+  for (int o = 16; o > 0; o >>= 1) Wr += __shfl_xor_sync(0xffffffffu, Wr, o);
   SchedStart s;
-  s.W = W;
-  s.nC = static_cast<int>(W < grid ? W : grid);
+  s.W = Wr + static_cast<int64_t>(p.seg_cost) * p.B * HR;
+  s.nC = static_cast<int>(Wr < grid ? Wr : grid);
   s.lo = s.hi = 0;
   s.b = 0;
   s.base_b = 0;
   if (cta >= s.nC) return s;
-  s.lo = static_cast<int64_t>(cta) * W / s.nC;
-  s.hi = static_cast<int64_t>(cta + 1) * W / s.nC;
-  // find the sequence whose unit range contains tile lo: scan in chunks of 32 sequences
-  int64_t run = 0;
-  for (int b0 = 0; b0 < p.B; b0 += 32) {
-    const int b = b0 + lane;
-    int64_t mine = b < p.B ? static_cast<int64_t>(tiles_of(clamp_context(p, b, false), p.tile_keys)) * HR : 0;
-    int64_t incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const int64_t excl = run + incl - mine;
-    const bool here = b < p.B && excl <= s.lo && s.lo < run + incl;
-    const uint32_t ball = __ballot_sync(0xffffffffu, here);
-    if (ball) {
-      const int src = __ffs(ball) - 1;
-      s.b = b0 + src;
-      s.base_b = __shfl_sync(0xffffffffu, excl, src);
-      return s;
-    }
-    run += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  return s;  // not reached for lo < W
+  const SchedPoint a = schedule_locate(p, static_cast<int64_t>(cta) * s.W / s.nC);
+  s.lo = a.t;
+  s.b = a.b;
+  s.base_b = a.base_b;
+  s.hi = cta + 1 == s.nC ? Wr : schedule_locate(p, static_cast<int64_t>(cta + 1) * s.W / s.nC).t;
+  return s;
 }
 
 // Destination of merged row r of a unit: dst == nullptr for a padding row (nothing is written),

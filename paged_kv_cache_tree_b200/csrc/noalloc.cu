@@ -208,6 +208,7 @@ extern "C" taco_status paged_tree_attention_noalloc(
   p.row_groups = row_groups;
   p.tile_keys = taco::kTileKeys;
   p.l2_prefetch_tiles = taco::kMmaPrefetchTiles;
+  p.seg_cost = taco::mma_seg_cost(rows);
   e = taco::launch_verify_mma(maps[0], maps[1], p, dtype, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "verify kernel launch: %s", cudaGetErrorString(e));
   return TACO_OK;

@@ -915,9 +915,9 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
     if (!whole_unit) {
       __threadfence();
       named_bar_sync(1, 128);
-      const int c_first = cta_of_tile(unit_base, W, nC);
-      const int c_last = cta_of_tile(unit_base + Tb - 1, W, nC);
       const int u = (b * p.Hkv + g) * p.row_groups + rg;
+      const UnitCtas uc = unit_ctas(p, unit_base, Tb, u, W, nC);
+      const int c_first = uc.c_first, c_last = uc.c_last;
       if (tid == 0) {
         const uint32_t prev = atomicAdd(p.counters + u, 1u);
         const bool last = prev == static_cast<uint32_t>(c_last - c_first);
@@ -929,9 +929,8 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
       }
       named_bar_sync(1, 128);
       if (sched->merge_flag) {
-        const int64_t lo_first = static_cast<int64_t>(c_first) * W / nC;
         const int64_t row0 = static_cast<int64_t>(b) * p.C;
-        merge_split_unit<T, D>(p, ROWS, ROWS, c_first, c_last, lo_first < unit_base, warp, lane,
+        merge_split_unit<T, D>(p, ROWS, ROWS, c_first, c_last, uc.first_odd, warp, lane,
                                [&](int r) -> MergeRow<T> {
                                  const int R = rg * ROWS + r;
                                  if (R >= p.G * p.C) return MergeRow<T>{nullptr, false};

@@ -910,10 +910,9 @@ __global__ void __launch_bounds__(384, 1)
       // the CTA that arrives last on the unit's counter combines every piece's partial
       __threadfence();
       named_bar_sync(1, 256);
-      const int64_t unit_base = cur.unit_base();
-      const int c_first = cta_of_tile(unit_base, W, nC);
-      const int c_last = cta_of_tile(unit_base + Tb - 1, W, nC);
       const int u = (b * p.Hkv + g) * p.row_groups + rg;
+      const UnitCtas uc = unit_ctas(p, cur.unit_base(), Tb, u, W, nC);
+      const int c_first = uc.c_first, c_last = uc.c_last;
       if (warp == 2 && lane == 0) {
         const uint32_t prev = atomicAdd(p.counters + u, 1u);
         const bool last = prev == static_cast<uint32_t>(c_last - c_first);
@@ -925,9 +924,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       named_bar_sync(1, 256);
       if (sh->merge_flag) {
-        const int64_t lo_first = static_cast<int64_t>(c_first) * W / nC;
-        if (row_real)
-          merge_split_row_half<T, D>(p, r, wg, c_first, c_last, lo_first < unit_base, dst, active);
+        if (row_real) merge_split_row_half<T, D>(p, r, wg, c_first, c_last, uc.first_odd, dst, active);
       }
       named_bar_sync(1, 256);
     }

@@ -90,6 +90,10 @@ def test_options(lib):
     assert lib.taco_attn_set_option(_lib.TACO_OPT_GRID_CTAS, 0) == _lib.TACO_OK
     assert lib.taco_attn_set_option(_lib.TACO_OPT_KERNEL, 5) == _lib.TACO_ERR_INVALID_ARG
     assert lib.taco_attn_set_option(99, 1) == _lib.TACO_ERR_INVALID_ARG
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_SEG_COST, 65) == _lib.TACO_ERR_INVALID_ARG
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_SEG_COST, -2) == _lib.TACO_ERR_INVALID_ARG
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_SEG_COST, 0) == _lib.TACO_OK
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_SEG_COST, -1) == _lib.TACO_OK
 
 
 @pytest.mark.parametrize("call,status", [

@@ -19,9 +19,11 @@ pytestmark = pytest.mark.gpu
 def _reset_options():
     taco.set_option(taco.TACO_OPT_GRID_CTAS, 0)
     taco.set_option(taco.TACO_OPT_KERNEL, 0)
+    taco.set_option(taco.TACO_OPT_SEG_COST, -1)
     yield
     taco.set_option(taco.TACO_OPT_GRID_CTAS, 0)
     taco.set_option(taco.TACO_OPT_KERNEL, 0)
+    taco.set_option(taco.TACO_OPT_SEG_COST, -1)
 
 
 def test_tiny_step_append_then_attend():
@@ -73,6 +75,26 @@ def test_split_kv_partitions_agree(grid, kernel):
     ref, _, _ = oracle_step(w, append=False)
     taco.set_option(taco.TACO_OPT_GRID_CTAS, grid)
     taco.set_option(taco.TACO_OPT_KERNEL, kernel)
+    out, _, _ = gpu_step(w, append=False)
+    assert_parity(out, ref, w)
+    again, _, _ = gpu_step(w, append=False)
+    assert torch.equal(out.view(torch.int16), again.view(torch.int16)), "not deterministic run to run"
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("grid", [1, 5, 37, 300])
+@pytest.mark.parametrize("seg_cost", [0, 1, 3, 64])
+def test_weighted_work_split_agrees(seg_cost, grid, kernel):
+    """The work split counts seg_cost extra tiles per unit. Units of one tile next to long ones, and a
+    cost far above the tiles of most units (whole CTA ranges then fall on no real tile), must still give
+    every piece to exactly one CTA and merge it once."""
+    spec = dict(dtype="bf16", B=10, Hq=16, Hkv=2, D=128, bs=16, C=4, tree="chain",
+                ctx=("fixed", [4, 5, 17, 64, 65, 700, 6, 1500, 130, 9]))
+    w = wl.make_workload(spec, seed=17)
+    ref, _, _ = oracle_step(w, append=False)
+    taco.set_option(taco.TACO_OPT_GRID_CTAS, grid)
+    taco.set_option(taco.TACO_OPT_KERNEL, kernel)
+    taco.set_option(taco.TACO_OPT_SEG_COST, seg_cost)
     out, _, _ = gpu_step(w, append=False)
     assert_parity(out, ref, w)
     again, _, _ = gpu_step(w, append=False)
