@@ -370,7 +370,7 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
     p.wait_limit_ns = 20000000ull;  // 20 ms
   }
   p.seg_cost = static_cast<int>(g_opt_seg_cost >= 0 ? g_opt_seg_cost
-                                : (use_tc ? taco::tc_seg_cost(cands_per_group * G) : taco::mma_seg_cost(rows)));
+                                : (use_tc ? taco::tc_seg_cost(cands_per_group * G, kv8) : taco::mma_seg_cost(rows)));
   p.l2_prefetch_tiles = static_cast<int>(
       g_opt_prefetch >= 0 ? g_opt_prefetch : (use_tc ? taco::kTcPrefetchTiles : taco::kMmaPrefetchTiles));
   p.k_scale = k_scale;
