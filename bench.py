@@ -335,6 +335,27 @@ def measure_accept(taco, w, d, dev, stream, args):
     }
 
 
+def measure_append(taco, w, d, dev, stream, args):
+    """Step A1 on its own: paged_kv_append of the step's candidates into their slots, timed with CUDA
+    events on its stream (median of 50 launches). Bytes = read + write of every appended row
+    (2 tensors x 2 x rows x Hkv x D x elt); the rows are a few hundred kB, so the call is launch-bound."""
+    n = 50
+    ts = []
+    for it in range(args.warmup + n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        taco.paged_kv_append(d.k_new, d.v_new, d.block_tables, d.slot_offsets, d.k_cache, d.v_cache, stream=stream)
+        e1.record(stream)
+        if it >= args.warmup:
+            ts.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    taco.check_device(stream)
+    us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in ts)
+    rows = int((w.slot_offsets >= 0).sum().item())
+    nbytes = 2 * 2 * rows * w.Hkv * w.D * 2
+    return {"rows": rows, "bytes": nbytes, "us": us, "GBps": nbytes / (us * 1e-6) / 1e9, "launches": n}
+
+
 def measure_kv8(taco, w, d, dev, stream, args):
     """The same verify step over 8-bit (e4m3) K/V caches with per-KV-head scales: the quantising append
     of the candidates' rows, then the attention. Caches are seeded random codes drawn on the device with
@@ -517,6 +538,7 @@ def measure_config(taco, name, world, rank, dev, stream, args, peak, peak_kind):
     accept = measure_accept(taco, w, d, dev, stream, args)
     accept["argmax_roofline"]["peak"] = peak
     accept["argmax_roofline"]["frac"] = accept["argmax_roofline"]["achieved"] / peak
+    append = measure_append(taco, w, d, dev, stream, args)
     kv8 = measure_kv8(taco, w, d, dev, stream, args)
     if kv8 is not None:
         kv8["attention_frac"] = kv8["attention_GBps"] / peak
@@ -537,6 +559,7 @@ def measure_config(taco, name, world, rank, dev, stream, args, peak, peak_kind):
         "gpu_launches": (1 if fused else 2) * n,
         "clocks": clocks,
         "accept": accept,
+        "append": append,
         "kv8": kv8,
     }
     del d, out
@@ -656,6 +679,7 @@ def run_ours(args, world, rank, local):
     e2e_value = world * nbytes / (e2e_ms * 1e-3) / 1e9
 
     accept = measure_accept(taco, w, d, dev, stream, args)
+    append = measure_append(taco, w, d, dev, stream, args)
     kv8 = measure_kv8(taco, w, d, dev, stream, args)
     prefix = measure_prefix(taco, dev, stream, args)
     lookahead = measure_lookahead(taco, dev, stream, args)
@@ -695,6 +719,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "accept": accept,
+        "append": append,
         "kv8": kv8,
         "prefix_cache": prefix,
         "lookahead_cache": lookahead,
