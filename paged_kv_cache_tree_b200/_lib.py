@@ -185,7 +185,7 @@ def paged_tree_attention_noalloc(q, k_cache, v_cache, block_tables, context_lens
                                  tree_mask_bits, scale: float, out: Optional[torch.Tensor] = None,
                                  stream=None) -> torch.Tensor:
     """Same as paged_tree_attention, through the entry point that allocates no device memory (its
-    scratch is a fixed array in the library; see include/taco_attn.h for its limits)."""
+    scratch is a fixed 24 MiB array in the library; see include/taco_attn.h for its limits)."""
     return paged_tree_attention(q, k_cache, v_cache, block_tables, context_lens, num_candidates, tree_mask_bits,
                                 scale, out=out, stream=stream, _entry="paged_tree_attention_noalloc")
 

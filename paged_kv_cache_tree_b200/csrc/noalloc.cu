@@ -9,18 +9,18 @@
 // result but takes its scratch (split-KV partials, arrival counters, error word) from a fixed array
 // that lives in the library's device image instead of calling cudaMalloc.
 //
-// Kernel: it always runs the mma.sync verify kernel, with at most 64 packed query rows per work unit,
-// and never the tcgen05 kernel that paged_tree_attention picks for wide tiles (G * C >= 48): that
-// kernel's partials (128 rows per slot, two slots per SM) would not fit the fixed array. Wide calls
-// (the chain and tree verify shapes) are therefore slower here than through paged_tree_attention.
+// Kernel: the same choice as paged_tree_attention makes automatically. Wide packed tiles (G * C >= 48,
+// G <= 128) run the tcgen05 kernel (one CTA per SM, 128-row partial slots); the others run the mma.sync
+// kernel.
 //
 // Limits and rules:
-//  - The scratch is kNoAllocScratchBytes = 8 MiB per device. Every GPU that loads the library holds
-//    it until the process exits.
-//  - At most kNoAllocMaxUnits = 65536 work units (batch * num_kv_heads * row groups, where a row group
-//    covers up to 64 packed query rows). Larger calls are rejected with TACO_ERR_UNSUPPORTED before
-//    anything is enqueued. The kernel's grid is capped so that its partials fit in the scratch; for
-//    wide row groups (G * C > 32) this means fewer CTAs than paged_tree_attention uses.
+//  - The scratch is kNoAllocScratchBytes = 24 MiB per device. Every GPU that loads the library holds
+//    it until the process exits. It holds two partial slots per CTA of either kernel's full grid on a
+//    148-SM B200 (the tcgen05 kernel's 128-row slots at head_dim 128 take 19.7 MB).
+//  - At most kNoAllocMaxUnits = 65536 work units (batch * num_kv_heads * row groups). Larger calls are
+//    rejected with TACO_ERR_UNSUPPORTED before anything is enqueued. The grid is capped so that the
+//    partials fit in the scratch (on a GPU with more SMs than that, fewer CTAs than
+//    paged_tree_attention uses).
 //  - All calls on a device share the one array, and it keeps the previous call's contents. Each call
 //    clears the arrival counters it needs on `stream` before its kernel runs. Two calls whose work
 //    overlaps on the GPU (different streams without ordering between them) race on the scratch and
@@ -45,7 +45,7 @@
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+constexpr size_t kNoAllocScratchBytes = size_t(24) << 20;
 constexpr int kNoAllocMaxUnits = 65536;
 constexpr size_t kErrWordBytes = 256;
 constexpr size_t kCounterBytes = size_t(kNoAllocMaxUnits) * 4;
@@ -117,8 +117,11 @@ extern "C" taco_status paged_tree_attention_noalloc(
   if (batch == 0) return TACO_OK;
 
   const int G = num_q_heads / num_kv_heads;
-  const int rows = taco::mma_rows_per_unit(G * max_candidates);
-  const int row_groups = (G * max_candidates + rows - 1) / rows;
+  const int packed = G * max_candidates;
+  const bool use_tc = packed >= 48 && G <= 128;  // as paged_tree_attention chooses for 16-bit caches
+  const int cands_per_group = use_tc ? (max_candidates < 128 / G ? max_candidates : 128 / G) : 0;
+  const int rows = use_tc ? 128 : taco::mma_rows_per_unit(packed);
+  const int row_groups = use_tc ? (max_candidates + cands_per_group - 1) / cands_per_group : (packed + rows - 1) / rows;
   const int64_t units = static_cast<int64_t>(batch) * num_kv_heads * row_groups;
   if (units > kNoAllocMaxUnits)
     return fail(TACO_ERR_UNSUPPORTED,
@@ -142,7 +145,7 @@ extern "C" taco_status paged_tree_attention_noalloc(
   // grid: the kernel's resident CTAs per SM, fewer if the partials (2 slots per CTA) would not fit
   const size_t slot_bytes = static_cast<size_t>(rows) * (head_dim + 1) * 4 + 512;
   const int max_grid = static_cast<int>(kPartialBytes / slot_bytes / 2);
-  int grid = taco::mma_ctas_per_sm(rows) * sms;
+  int grid = (use_tc ? 1 : taco::mma_ctas_per_sm(rows)) * sms;
   if (grid > max_grid) grid = max_grid;
   if (grid < 1) return fail(TACO_ERR_UNSUPPORTED, "scratch too small for one CTA");
   const size_t slots = 2 * static_cast<size_t>(grid);
@@ -156,7 +159,7 @@ extern "C" taco_status paged_tree_attention_noalloc(
   e = cudaMemsetAsync(counters, 0, static_cast<size_t>(units) * 4, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "cudaMemsetAsync(scratch): %s", cudaGetErrorString(e));
 
-  // TMA descriptors of the two caches: rows of D elements, 64-column boxes of min(bs, 64) rows
+  // TMA descriptors of the two caches: rows of D elements, 64-column boxes of min(bs, tile keys) rows
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -168,7 +171,8 @@ extern "C" taco_status paged_tree_attention_noalloc(
       encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(sym);
   });
   if (!encode) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const int rpc = block_size < taco::kTileKeys ? block_size : taco::kTileKeys;
+  const int tile = use_tc ? taco::tc_tile_keys() : taco::kTileKeys;
+  const int rpc = block_size < tile ? block_size : tile;
   CUtensorMap maps[2];
   const void* caches[2] = {k_cache, v_cache};
   for (int m = 0; m < 2; ++m) {
@@ -181,6 +185,20 @@ extern "C" taco_status paged_tree_attention_noalloc(
                         2, const_cast<void*>(caches[m]), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  }
+  // tcgen05 kernel: the query tile view [B*C, Hq, D], one box = 64 columns x G heads x the candidates of
+  // one row group
+  CUtensorMap qmap;
+  if (use_tc) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                          static_cast<cuuint64_t>(batch) * max_candidates};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(cands_per_group)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(&qmap, dtype == TACO_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        3, const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TACO_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", static_cast<int>(r));
   }
 
   taco::VerifyParams p{};
@@ -206,10 +224,12 @@ extern "C" taco_status paged_tree_attention_noalloc(
   p.max_blocks = max_blocks_per_seq;
   p.rows_per_unit = rows;
   p.row_groups = row_groups;
-  p.tile_keys = taco::kTileKeys;
-  p.l2_prefetch_tiles = taco::kMmaPrefetchTiles;
-  p.seg_cost = taco::mma_seg_cost(rows);
-  e = taco::launch_verify_mma(maps[0], maps[1], p, dtype, grid, static_cast<cudaStream_t>(stream));
+  p.cands_per_group = cands_per_group;
+  p.tile_keys = tile;
+  p.l2_prefetch_tiles = use_tc ? taco::kTcPrefetchTiles : taco::kMmaPrefetchTiles;
+  p.seg_cost = use_tc ? taco::tc_seg_cost(cands_per_group * G, false) : taco::mma_seg_cost(rows);
+  e = use_tc ? taco::launch_verify_tc(maps[0], maps[1], qmap, p, dtype, grid, static_cast<cudaStream_t>(stream))
+             : taco::launch_verify_mma(maps[0], maps[1], p, dtype, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(TACO_ERR_CUDA, "verify kernel launch: %s", cudaGetErrorString(e));
   return TACO_OK;
 }

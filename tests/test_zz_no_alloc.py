@@ -44,13 +44,19 @@ def _noalloc_bits():
 
 
 SPECS = [
-    # 16 packed rows, short contexts
+    # 16 packed rows, short contexts: the mma.sync kernel
     dict(dtype="bf16", B=8, Hq=32, Hkv=8, D=128, bs=16, C=4, tree="forest", ctx=("uniform", 200, 3000)),
-    # 64 packed rows (a chain verify): the grid is capped at 121 CTAs for the fixed partials
+    # 64 packed rows (a chain verify): the tcgen05 kernel, as in paged_tree_attention
     dict(dtype="fp16", B=4, Hq=64, Hkv=8, D=128, bs=32, C=8, tree="chain", ctx=("uniform", 100, 2500)),
-    # few long sequences: every unit is split over several CTAs of the capped grid, so the
-    # log-sum-exp merge reads partials from the fixed array
+    # few long sequences: every unit is split over several CTAs, so the log-sum-exp merge reads
+    # 128-row partials from the fixed array
     dict(dtype="bf16", B=2, Hq=64, Hkv=8, D=128, bs=32, C=8, tree="forest", ctx=("uniform", 6000, 9000)),
+    # 128 packed rows (a tree verify) on the tcgen05 kernel
+    dict(dtype="bf16", B=3, Hq=64, Hkv=8, D=128, bs=32, C=16, tree="forest", ctx=("uniform", 500, 4000)),
+    # 32 packed rows, long contexts: mma.sync with split units merged through the fixed array
+    dict(dtype="bf16", B=2, Hq=64, Hkv=8, D=128, bs=64, C=4, tree="chain", ctx=("uniform", 5000, 9000)),
+    # head_dim 64 on the tcgen05 kernel
+    dict(dtype="bf16", B=3, Hq=32, Hkv=4, D=64, bs=16, C=8, tree="forest", ctx=("uniform", 300, 2000)),
 ]
 
 
