@@ -97,7 +97,7 @@ class ClockSampler:
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_power_cap,clocks.mem,temperature.gpu,temperature.memory")
 
     def __init__(self, device_index: int):
         self.proc = None
@@ -119,7 +119,7 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             return None
-        sm, smax, reasons = [], [], set()
+        sm, smax, reasons, mem, power, tgpu, tmem = [], [], set(), [], [], [], []
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for line in out.strip().splitlines():
             parts = [x.strip() for x in line.split(",")]
@@ -133,10 +133,24 @@ class ClockSampler:
             for nm, v in zip(names, parts[4:8]):
                 if v.lower().startswith("active"):
                     reasons.add(nm)
+            for lst, i in ((power, 2), (mem, 8), (tgpu, 9), (tmem, 10)):
+                try:
+                    lst.append(float(parts[i]))
+                except (ValueError, IndexError):
+                    pass
         if not sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        rec = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+               "reasons": sorted(reasons)}
+        if mem:
+            rec["mem_mhz"] = statistics.median(mem)
+        if power:
+            rec["power_w"] = statistics.median(power)
+        if tgpu:
+            rec["temp_gpu_c_max"] = max(tgpu)
+        if tmem:
+            rec["temp_mem_c_max"] = max(tmem)
+        return rec
 
 
 def dist_setup(args):
