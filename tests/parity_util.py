@@ -24,6 +24,23 @@ def gpu_step(w, device="cuda", append=True):
     return out.cpu(), d.k_cache, d.v_cache
 
 
+def full_size_rows(w, seed, extra=24):
+    """Rows (b, i, h) for a full-size parity check: one of every (sequence, KV head) unit (a random live
+    candidate and a random head of the group), so that every unit and every split piece is merged and
+    checked, plus `extra` random rows and the first and last row."""
+    rng = np.random.default_rng(seed)
+    G = w.Hq // w.Hkv
+    rows = {(0, 0, 0), (w.B - 1, max(0, int(w.num_candidates[-1]) - 1), w.Hq - 1)}
+    for b in range(w.B):
+        n = max(1, int(w.num_candidates[b]))
+        for g in range(w.Hkv):
+            rows.add((b, int(rng.integers(n)), g * G + int(rng.integers(G))))
+    for _ in range(extra):
+        b = int(rng.integers(w.B))
+        rows.add((b, int(rng.integers(max(1, int(w.num_candidates[b])))), int(rng.integers(w.Hq))))
+    return sorted(rows)
+
+
 def oracle_inputs(w):
     return dict(q=wl.to_numpy_bits(w.q), k_cache=wl.to_numpy_bits(w.k_cache), v_cache=wl.to_numpy_bits(w.v_cache),
                 block_tables=w.block_tables.numpy(), context_lens=w.context_lens.numpy(),

@@ -9,7 +9,7 @@ import torch
 import oracle
 import paged_kv_cache_tree_b200 as taco
 from paged_kv_cache_tree_b200 import workloads as wl
-from tests.parity_util import assert_parity, oracle_step
+from tests.parity_util import assert_parity, full_size_rows, oracle_step
 
 pytestmark = pytest.mark.gpu
 
@@ -69,12 +69,7 @@ def test_full_size_sampled_rows(name):
             blk = int(bt[b, s // w.bs])
             assert torch.equal(kc[blk, :, s % w.bs].view(torch.int16), w.k_new[b, i].view(torch.int16))
             assert torch.equal(vc[blk, :, s % w.bs].view(torch.int16), w.v_new[b, i].view(torch.int16))
-    rng = np.random.default_rng(4)
-    rows = set()
-    for _ in range(24):
-        b = int(rng.integers(w.B))
-        rows.add((b, int(rng.integers(max(1, int(w.num_candidates[b])))), int(rng.integers(w.Hq))))
-    rows = sorted(rows | {(0, 0, 0)})
+    rows = full_size_rows(w, seed=4)
     w_after = wl.make_workload(name, candidates_in_cache=True)
     ref, _, _ = oracle_step(w_after, append=False, rows=rows)
     assert_parity(out, ref, w, rows=rows)

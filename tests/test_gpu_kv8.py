@@ -12,7 +12,7 @@ import oracle
 from oracle import fp8
 import paged_kv_cache_tree_b200 as taco
 from paged_kv_cache_tree_b200 import workloads as wl
-from tests.parity_util import assert_parity
+from tests.parity_util import assert_parity, full_size_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -175,17 +175,12 @@ def test_append_then_attend_end_to_end():
 
 @pytest.mark.parametrize("name", ["decode", "chain", "tree", "long"])
 def test_full_size_workloads_sampled_rows(name):
-    """The bench's workloads at full size with e4m3 caches, in the default launch configuration:
-    24 sampled rows against the oracle."""
+    """The bench's workloads at full size with e4m3 caches, in the default launch configuration: one row
+    of every (sequence, KV head) unit plus 24 sampled rows against the oracle."""
     w = wl.make_workload(name)
     c8 = wl.make_e4m3_cache(w)
     got = gpu_attention_e4m3(w, c8)
-    rng = np.random.default_rng(1)
-    rows = {(0, 0, 0), (w.B - 1, int(w.num_candidates[-1]) - 1, w.Hq - 1)}
-    while len(rows) < 24:
-        b = int(rng.integers(w.B))
-        rows.add((b, int(rng.integers(max(1, int(w.num_candidates[b])))), int(rng.integers(w.Hq))))
-    rows = sorted(rows)
+    rows = full_size_rows(w, seed=1)
     assert_parity(got, oracle_attention_e4m3(w, c8, rows=rows), w, rows=rows)
     assert torch.isfinite(got.float()).all()
 

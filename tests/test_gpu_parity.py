@@ -10,7 +10,7 @@ import torch
 import oracle
 import paged_kv_cache_tree_b200 as taco
 from paged_kv_cache_tree_b200 import workloads as wl
-from tests.parity_util import as_f64, assert_parity, gpu_step, oracle_inputs, oracle_step
+from tests.parity_util import as_f64, assert_parity, full_size_rows, gpu_step, oracle_inputs, oracle_step
 
 pytestmark = pytest.mark.gpu
 
@@ -185,12 +185,7 @@ def test_full_size_workloads_sampled_rows(name):
             blk = int(bt[b, s // w.bs])
             assert torch.equal(kc_cpu[blk, :, s % w.bs].view(torch.int16), w.k_new[b, i].view(torch.int16))
     del kc_cpu
-    rng = np.random.default_rng(0)
-    rows = {(0, 0, 0), (w.B - 1, int(w.num_candidates[-1]) - 1, w.Hq - 1)}
-    while len(rows) < 24:
-        b = int(rng.integers(w.B))
-        rows.add((b, int(rng.integers(max(1, int(w.num_candidates[b])))), int(rng.integers(w.Hq))))
-    rows = sorted(rows)
+    rows = full_size_rows(w, seed=0)
     w_after = wl.make_workload(name, candidates_in_cache=True)
     ref, _, _ = oracle_step(w_after, append=False, rows=rows)
     assert_parity(out, ref, w, rows=rows)

@@ -23,8 +23,13 @@ def mutant(module_name: str, old: str, new: str) -> types.ModuleType:
     return mod
 
 
-def pins_fail(test_module, mod, names):
-    """Run every test function of test_module with the given names re-bound to mod's; True if any fails."""
+def pins_fail(test_module, mod, names, mutated_file=None):
+    """Run every test function of test_module with the given names re-bound to mod's; True if any fails.
+
+    A pin fails by an assertion. Any other exception counts as a failure only when it was raised while
+    running the mutated oracle source (a frame of mutated_file on its traceback, e.g. an index the
+    mutation pushed out of range); anywhere else it is a fault of the harness or of the pin itself and
+    propagates, so that a broken harness cannot pass for a caught mutant."""
     saved = {n: getattr(test_module, n) for n in names}
     try:
         for n in names:
@@ -52,8 +57,14 @@ def pins_fail(test_module, mod, names):
                     fn(**kwargs)
                 except AssertionError:
                     return True
-                except Exception:
-                    return True
+                except Exception as e:
+                    tb, files = e.__traceback__, set()
+                    while tb is not None:
+                        files.add(tb.tb_frame.f_code.co_filename)
+                        tb = tb.tb_next
+                    if mutated_file is not None and mutated_file in files:
+                        return True
+                    raise
         return False
     finally:
         for n, v in saved.items():
@@ -88,15 +99,16 @@ ACCEPT_MUTATIONS = [
 @pytest.mark.parametrize("old,new", PREFIX_MUTATIONS)
 def test_prefix_pins_catch(old, new):
     import tests.test_oracle_prefix as t
-    assert pins_fail(t, mutant("prefix_cache", old, new),
-                     ["PrefixTree", "batch_insert_choices", "insert_batch", "lookup_batch"])
+    m = mutant("prefix_cache", old, new)
+    assert pins_fail(t, m, ["PrefixTree", "batch_insert_choices", "insert_batch", "lookup_batch"], m.__file__)
 
 
 @pytest.mark.parametrize("old,new", LOOKAHEAD_MUTATIONS)
 def test_lookahead_pins_catch(old, new):
     import tests.test_oracle_lookahead as t
-    assert pins_fail(t, mutant("lookahead_cache", old, new),
-                     ["build_forest", "longest_match", "propose", "propose_batch", "update_copy_len"])
+    m = mutant("lookahead_cache", old, new)
+    assert pins_fail(t, m, ["build_forest", "longest_match", "propose", "propose_batch", "update_copy_len"],
+                     m.__file__)
 
 
 @pytest.mark.parametrize("old,new", ACCEPT_MUTATIONS)
@@ -105,7 +117,7 @@ def test_acceptance_pins_catch(old, new):
     saved = t.ta                       # the pin module calls the oracle through this module alias
     t.ta = mutant("tree_accept", old, new)
     try:
-        assert pins_fail(t, t.ta, [])
+        assert pins_fail(t, t.ta, [], t.ta.__file__)
     finally:
         t.ta = saved
 
@@ -156,9 +168,10 @@ def _oracle_with(mod):
 def test_attention_pins_catch(old, new):
     import tests.test_oracle as t
     saved = t.oracle
-    t.oracle = _oracle_with(mutant("paged_attention", old, new))
+    m = mutant("paged_attention", old, new)
+    t.oracle = _oracle_with(m)
     try:
-        assert pins_fail(t, None, [])
+        assert pins_fail(t, None, [], m.__file__)
     finally:
         t.oracle = saved
 
@@ -169,7 +182,7 @@ def test_fp8_pins_catch(old, new):
     saved = t.fp8
     t.fp8 = mutant("fp8", old, new)
     try:
-        assert pins_fail(t, None, [])
+        assert pins_fail(t, None, [], t.fp8.__file__)
     finally:
         t.fp8 = saved
 
