@@ -55,8 +55,17 @@ __device__ __forceinline__ void chunk_scan(const int32_t* seq, int c0, int count
   a = 0;
   q = 1;
   if (lane < count) {
+    // the block's tokens are loaded eight at a time before they are hashed, so that a block costs one
+    // dependent round trip per eight tokens rather than per token
     const int32_t* t = seq + static_cast<int64_t>(c0 + lane) * bs;
-    for (int i = 0; i < bs; ++i) a = a * kHashBase + (static_cast<uint64_t>(static_cast<uint32_t>(__ldg(t + i))) + 1ull);
+    for (int i0 = 0; i0 < bs; i0 += 8) {
+      uint32_t x[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = i0 + k < bs ? static_cast<uint32_t>(__ldg(t + i0 + k)) : 0u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (i0 + k < bs) a = a * kHashBase + (static_cast<uint64_t>(x[k]) + 1ull);
+    }
     q = base_bs;
   }
 #pragma unroll
@@ -103,6 +112,27 @@ __device__ __forceinline__ bool block_tokens_equal(const int32_t* a, const int32
   }
   bool eq = true;
   for (; i < bs; ++i) eq &= __ldg(a + i) == __ldg(node_tok + i);
+  return eq;
+}
+
+// The same comparison for a node another warp of the running launch may have written: the node's
+// tokens are read through L2 (a read-only-cache line could predate the write).
+__device__ __forceinline__ bool block_tokens_equal_coherent(const int32_t* a, const int32_t* node_tok, int bs) {
+  int i = 0;
+  for (; i + 8 <= bs; i += 8) {
+    int32_t x[8], y[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      x[k] = __ldg(a + i + k);
+      y[k] = __ldcg(node_tok + i + k);
+    }
+    bool eq = true;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) eq &= x[k] == y[k];
+    if (!eq) return false;
+  }
+  bool eq = true;
+  for (; i < bs; ++i) eq &= __ldg(a + i) == __ldcg(node_tok + i);
   return eq;
 }
 
@@ -268,10 +298,73 @@ __global__ void __launch_bounds__(kLookupWarps * 32) prefix_lookup_kernel(Prefix
 }
 
 // --------------------------------------------------------------------------------------------- insert
-// One warp per sequence, its full blocks in order. Probing a block's chain: an empty slot is claimed
-// with a compare-and-swap and the sequence's own block becomes the node (data written, then the slot
-// published); a slot with the same key is waited for until published (bounded) and reused when depth,
-// parent and tokens match. Every other slot is skipped.
+// One block's step of an ordered walk, run by a whole warp (lane 0 does the atomics), with its probe
+// starting at `slot`: an empty slot is claimed with a compare-and-swap and the sequence's own block
+// becomes the node (data written, then the slot published); a slot with the same key is waited for
+// until published (bounded) and reused when depth, parent and tokens match. Every other slot is
+// skipped. Returns the node that holds the block's prefix, or -1 after setting the error bit (no free
+// slot, or the wait ran out).
+__device__ int insert_step(const PrefixArgs& a, uint64_t key, uint64_t slot, int own, int j, const int32_t* tok,
+                           int parent, int lane) {
+  const uint64_t mask = static_cast<uint64_t>(a.cap) - 1;
+  for (int64_t it = 0; it < a.cap; ++it) {
+    uint64_t k = 0;
+    // one compare-and-swap both reads the slot and, when it is empty, claims it (0 comes back)
+    if (lane == 0) k = atomicCAS(reinterpret_cast<unsigned long long*>(a.slot_keys + slot), 0ull, key);
+    k = shfl_u64(k, 0);
+    if (k == 0ull) {
+      for (int i = lane; i < a.bs; i += 32) a.node_tokens[static_cast<int64_t>(own) * a.bs + i] = __ldg(tok + i);
+      if (lane == 0) {
+        a.node_parent[own] = parent;
+        a.node_depth[own] = j;
+      }
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicExch(a.slot_nodes + slot, own);
+      return own;
+    }
+    if (k == key) {
+      int nd = -1;
+      if (lane == 0) {
+        for (int spin = 0; spin < kSpinLimit; ++spin) {
+          nd = atomicAdd(a.slot_nodes + slot, 0);
+          if (nd >= 0) break;
+          __nanosleep(32);
+        }
+      }
+      nd = __shfl_sync(0xffffffffu, nd, 0);
+      if (nd < 0) {
+        if (lane == 0) atomicOr(a.error_word, TACO_DEVERR_WAIT_TIMEOUT);
+        return -1;
+      }
+      __threadfence();
+      bool same = nd < a.num_blocks && __ldcg(a.node_depth + nd) == j && __ldcg(a.node_parent + nd) == parent;
+      if (same) {
+        bool eq = true;
+        for (int i = lane; i < a.bs; i += 32) eq &= (__ldg(tok + i) == __ldcg(a.node_tokens + static_cast<int64_t>(nd) * a.bs + i));
+        same = __all_sync(0xffffffffu, eq);
+      }
+      if (same) return nd;
+    }
+    slot = (slot + 1) & mask;
+  }
+  if (lane == 0) atomicOr(a.error_word, TACO_DEVERR_TABLE_FULL);
+  return -1;
+}
+
+// One warp per sequence, 32 full blocks per round (lane = block):
+//   1. Every block of the round claims an empty slot on its key's probe chain with a compare-and-swap,
+//      or stops at a slot that already holds its key. Nothing waits here, because the holder of that
+//      key (another sequence) may itself still be waiting for this one's earlier blocks.
+//   2. The blocks are then resolved in order. A run of claimed blocks is settled at once: each one's
+//      node is its own block and its parent the block before it, so the run writes its nodes, fences
+//      and publishes them together. A run of blocks that found their keys taken waits for those nodes
+//      together and keeps them up to the first that is not its block's prefix; that block then takes
+//      one step of the ordered walk (insert_step) from the next slot on.
+// The lowest pending block of any sequence can always go on (its parent is settled), so no wait cycle
+// forms. Bad block ids are found before any claim, and the walk ends at the first of them. If the walk
+// ends early (no free slot, a wait that ran out), the round's claims it did not reach are published as
+// node id NB, which no probe accepts, so that nobody waits for them.
 __global__ void __launch_bounds__(256) prefix_insert_kernel(PrefixArgs a) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -285,79 +378,127 @@ __global__ void __launch_bounds__(256) prefix_insert_kernel(PrefixArgs a) {
   const int32_t* table = a.block_tables + static_cast<int64_t>(b) * a.max_blocks;
   int32_t* out = a.out_blocks + static_cast<int64_t>(b) * a.max_blocks;
   uint64_t carry = 0;
-  int parent = -1;
+  int prev = -1;
   int done = 0;
   bool stop = false;
-  uint64_t key_lane = 0;
-  for (int j = 0; j < nfull && !stop; ++j) {
-    if ((j & 31) == 0) {
-      const int count = nfull - j < 32 ? nfull - j : 32;
-      key_lane = chunk_keys(seq, j, count, a.bs, base_bs, carry, lane);
-    }
-    const uint64_t key = shfl_u64(key_lane, j & 31);
-    const int own = __ldg(table + j);
-    if (own < 0 || own >= a.num_blocks) {
+  for (int c0 = 0; c0 < nfull && !stop; c0 += 32) {
+    const int count = nfull - c0 < 32 ? nfull - c0 : 32;
+    const uint64_t key = chunk_keys(seq, c0, count, a.bs, base_bs, carry, lane);
+    const int j = c0 + lane;
+    const int own = lane < count ? __ldg(table + j) : 0;
+    const uint32_t bad = __ballot_sync(0xffffffffu, lane < count && (own < 0 || own >= a.num_blocks));
+    int cnt = count;
+    if (bad) {
+      cnt = __ffs(bad) - 1;
+      stop = true;
       if (lane == 0) atomicOr(a.error_word, TACO_DEVERR_BLOCK_ID);
-      break;
     }
-    const int32_t* tok = seq + static_cast<int64_t>(j) * a.bs;
+    // 1. claims
     uint64_t slot = key & mask;
-    int found = -1;
-    for (int64_t it = 0; it < a.cap && found < 0 && !stop; ++it) {
-      uint64_t k = 0;
-      // one compare-and-swap both reads the slot and, when it is empty, claims it (0 comes back)
-      if (lane == 0) k = atomicCAS(reinterpret_cast<unsigned long long*>(a.slot_keys + slot), 0ull, key);
-      k = shfl_u64(k, 0);
-      if (k == 0ull) {
-        // claimed: write the node, then publish it
-        for (int i = lane; i < a.bs; i += 32) a.node_tokens[static_cast<int64_t>(own) * a.bs + i] = __ldg(tok + i);
-        if (lane == 0) {
-          a.node_parent[own] = parent;
-          a.node_depth[own] = j;
+    int state = 0;  // 1 claimed, 2 found its key in a slot, 3 no free slot on the chain
+    if (lane < cnt) {
+      for (int64_t it = 0; it < a.cap; ++it) {
+        const uint64_t k = atomicCAS(reinterpret_cast<unsigned long long*>(a.slot_keys + slot), 0ull, key);
+        if (k == 0ull) {
+          state = 1;
+          break;
         }
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicExch(a.slot_nodes + slot, own);
-        found = own;
-        break;
+        if (k == key) {
+          state = 2;
+          break;
+        }
+        slot = (slot + 1) & mask;
       }
-      if (k == key) {
-        int nd = -1;
-        if (lane == 0) {
+      if (state == 0) state = 3;
+    }
+    // 2. resolution in block order
+    const uint32_t claimed = __ballot_sync(0xffffffffu, state == 1);
+    const int own_before = __shfl_up_sync(0xffffffffu, own, 1);
+    int r = 0;
+    while (r < cnt) {
+      const uint32_t rest = claimed >> r;
+      int run = rest == 0xffffffffu ? 32 : __ffs(~rest) - 1;
+      if (run > cnt - r) run = cnt - r;
+      if (run > 0) {
+        if (lane >= r && lane < r + run) {
+          const int32_t* tok = seq + static_cast<int64_t>(j) * a.bs;
+          int32_t* dst = a.node_tokens + static_cast<int64_t>(own) * a.bs;
+          for (int i0 = 0; i0 < a.bs; i0 += 8) {  // eight loads in flight before their stores
+            int32_t x[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) x[k] = i0 + k < a.bs ? __ldg(tok + i0 + k) : 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              if (i0 + k < a.bs) dst[i0 + k] = x[k];
+          }
+          a.node_parent[own] = lane == r ? prev : own_before;
+          a.node_depth[own] = j;
+          __threadfence();
+          atomicExch(a.slot_nodes + slot, own);
+          out[j] = own;
+        }
+        prev = __shfl_sync(0xffffffffu, own, r + run - 1);
+        r += run;
+        continue;
+      }
+      // consecutive blocks from r that found their key: each waits for that slot's node (bounded) and
+      // checks it, all at once; a node is this block's prefix when depth, tokens and parent (the node of
+      // the block before) match, and the run is taken up to its first block that does not
+      const uint32_t held = __ballot_sync(0xffffffffu, state == 2) >> r;
+      int hrun = held == 0xffffffffu ? 32 : __ffs(~held) - 1;
+      if (hrun > cnt - r) hrun = cnt - r;
+      uint64_t from = shfl_u64(slot, r);  // where block r's own step starts
+      if (hrun > 0) {
+        const bool in = lane >= r && lane < r + hrun;
+        int nd = -1, par = -2;
+        bool same = false;
+        if (in) {
           for (int spin = 0; spin < kSpinLimit; ++spin) {
             nd = atomicAdd(a.slot_nodes + slot, 0);
             if (nd >= 0) break;
             __nanosleep(32);
           }
+          if (nd >= 0 && nd < a.num_blocks) {
+            __threadfence();
+            same = __ldcg(a.node_depth + nd) == j &&
+                   block_tokens_equal_coherent(seq + static_cast<int64_t>(j) * a.bs,
+                                               a.node_tokens + static_cast<int64_t>(nd) * a.bs, a.bs);
+            par = __ldcg(a.node_parent + nd);
+          }
         }
-        nd = __shfl_sync(0xffffffffu, nd, 0);
-        if (nd < 0) {
+        const int nd_before = __shfl_up_sync(0xffffffffu, nd, 1);
+        same = same && par == (lane == r ? prev : nd_before);
+        const uint32_t ok = __ballot_sync(0xffffffffu, in && same) >> r;
+        int good = ok == 0xffffffffu ? 32 : __ffs(~ok) - 1;
+        if (good > hrun) good = hrun;
+        if (lane >= r && lane < r + good) out[j] = nd;
+        if (good > 0) {
+          prev = __shfl_sync(0xffffffffu, nd, r + good - 1);
+          r += good;
+          continue;
+        }
+        // block r's node is not its prefix (another prefix with the same key) or never came: its own
+        // ordered step, from the slot after (or, after a wait that ran out, at) the one it found
+        const int nd_r = __shfl_sync(0xffffffffu, nd, r);
+        if (nd_r < 0) {
           if (lane == 0) atomicOr(a.error_word, TACO_DEVERR_WAIT_TIMEOUT);
           stop = true;
           break;
         }
-        __threadfence();
-        bool same = nd < a.num_blocks && __ldcg(a.node_depth + nd) == j && __ldcg(a.node_parent + nd) == parent;
-        if (same) {
-          bool eq = true;
-          for (int i = lane; i < a.bs; i += 32) eq &= (__ldg(tok + i) == __ldcg(a.node_tokens + static_cast<int64_t>(nd) * a.bs + i));
-          same = __all_sync(0xffffffffu, eq);
-        }
-        if (same) {
-          found = nd;
-          break;
-        }
+        from = (from + 1) & mask;
       }
-      slot = (slot + 1) & mask;
+      const int found = insert_step(a, shfl_u64(key, r), from, __shfl_sync(0xffffffffu, own, r), c0 + r,
+                                    seq + static_cast<int64_t>(c0 + r) * a.bs, prev, lane);
+      if (found < 0) {
+        stop = true;
+        break;
+      }
+      if (lane == 0) out[c0 + r] = found;
+      prev = found;
+      ++r;
     }
-    if (stop) break;
-    if (found < 0) {
-      if (lane == 0) atomicOr(a.error_word, TACO_DEVERR_TABLE_FULL);
-      break;
-    }
-    if (lane == 0) out[j] = found;
-    parent = found;
-    done = j + 1;
+    if (r < cnt && lane >= r && lane < cnt && state == 1) atomicExch(a.slot_nodes + slot, a.num_blocks);
+    done = c0 + r;
   }
   for (int jj = done + lane; jj < a.max_blocks; jj += 32) out[jj] = -1;
   if (a.out_matched != nullptr && lane == 0) a.out_matched[b] = done;

@@ -163,7 +163,11 @@ def test_device_errors_are_reported_not_faulted():
     with pytest.raises(taco.TacoError) as ei:
         taco.check_device()
     assert "table full" in str(ei.value)
-    assert int(cnt[0]) == 4
+    # the blocks claim slots together, so which of them got the 4 slots is not fixed; the walk ends at
+    # the first block without one, and every block before it is inserted with its own block id
+    n = int(cnt[0])
+    assert 0 <= n <= 4
+    assert got.cpu().tolist()[0] == table[0, :n].tolist() + [-1] * (10 - n)
     # a block id outside the pool, and decreasing seq_starts
     cache = taco.PrefixCache(8, bs, 64)
     bad = torch.tensor([[0, 99, 2]], dtype=torch.int32).cuda()
