@@ -189,6 +189,13 @@ def barrier(world: int):
         dist.barrier()
 
 
+def launch_kernels(launches: int, fused: bool) -> str:
+    """What one paged_tree_attention_append call launched, from the library's own count."""
+    if fused:
+        return "the verify kernel with the append inside" + (" + the combine kernel" if launches == 2 else "")
+    return "the append kernel + the verify kernel" + (" + the combine kernel" if launches == 3 else "")
+
+
 def step_bytes(w) -> int:
     return w.kv_bytes() + w.qo_bytes() + w.append_bytes()
 
@@ -532,6 +539,7 @@ def measure_config(taco, name, world, rank, dev, stream, args, peak, peak_kind):
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize(dev)
+    launches = taco.last_call_launches()
     n = 200
     pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -571,7 +579,8 @@ def measure_config(taco, name, world, rank, dev, stream, args, peak, peak_kind):
                      "peak_source": f"{peak_kind} hbm_gbs",
                      "kernel": "paged_tree_attention_append (append fused into the verify)" if fused else
                                "paged_tree_attention_append (append kernel, then the verify)"},
-        "gpu_launches": (1 if fused else 2) * n,
+        "gpu_launches": launches * n,
+        "launch_kernels": launch_kernels(launches, fused),
         "clocks": clocks,
         "accept": accept,
         "append": append,
@@ -596,9 +605,9 @@ def run_ours(args, world, rank, local):
 
     # one step = the candidates' KV-append and the verify attention, through the fused entry point
     # (append inside the verify kernel for narrow units, the append kernel first otherwise); the
-    # events bracket the whole call, so the attention roofline below counts the append's bytes too
+    # events bracket the whole call, so the attention roofline below counts the append's bytes too;
+    # a call is one to three launches (see launch_kernels below), counted by the library itself
     fused = w.G * w.C <= 16
-    launches_per_step = 1 if fused else 2
 
     def step(ev_pair=None):
         if ev_pair is not None:
@@ -612,6 +621,7 @@ def run_ours(args, world, rank, local):
         step()
     torch.cuda.synchronize(dev)
     taco.check_device(stream)
+    launches_per_step = taco.last_call_launches()
 
     pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -732,6 +742,7 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
+        "launch_kernels": launch_kernels(launches_per_step, fused),
         "clocks": clocks,
         "accept": accept,
         "append": append,

@@ -418,7 +418,17 @@ void taco_attn_release_workspace(void);
                                   0 = off (default); t + 1 = the first CTA's producers never arm the
                                   stage of its tile t, so that a consumer's wait runs out after 20 ms,
                                   the call reports TACO_DEVERR_WAIT_TIMEOUT and its output is undefined */
+#define TACO_OPT_COMBINE 6     /* split-KV combine of the mma.sync verify: 0 = automatic (a separate combine
+                                  kernel when the call has at most a quarter as many work units as
+                                  CTAs, so that units are cut into many pieces; else inside the verify),
+                                  1 = inside the verify, by the last CTA to finish each unit, 2 = the
+                                  separate kernel, one warp per output row */
 taco_status taco_attn_set_option(int32_t key, int64_t value);
+
+/* Kernels the calling thread's last attention call (paged_tree_attention, _append, _e4m3,
+ * _append_e4m3) enqueued: the append or query conversion when it ran, the verify, and the combine when
+ * it ran separately. 0 when that call failed before its first launch. */
+int32_t taco_attn_last_call_launches(void);
 
 /* ABI version of this header (bumped on any signature change). */
 int32_t taco_attn_version(void);

@@ -10,6 +10,7 @@ from ._lib import (  # noqa: F401
     TACO_OPT_L2_PREFETCH,
     TACO_OPT_TEST_STALL,
     TACO_OPT_SEG_COST,
+    TACO_OPT_COMBINE,
     TacoError,
     check_device,
     check_noalloc,
@@ -28,4 +29,5 @@ from ._lib import (  # noqa: F401
     tree_greedy_accept,
     tree_mask_from_parents,
     version,
+    last_call_launches,
 )

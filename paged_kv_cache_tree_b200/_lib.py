@@ -30,6 +30,7 @@ TACO_OPT_KERNEL = 2
 TACO_OPT_L2_PREFETCH = 3
 TACO_OPT_TEST_STALL = 4
 TACO_OPT_SEG_COST = 5
+TACO_OPT_COMBINE = 6
 
 EXPORTED = (
     "paged_tree_attention",
@@ -45,6 +46,7 @@ EXPORTED = (
     "taco_attn_release_workspace",
     "taco_attn_set_option",
     "taco_attn_version",
+    "taco_attn_last_call_launches",
     "tree_mask_from_parents",
     "logits_argmax",
     "tree_greedy_accept",
@@ -98,6 +100,8 @@ def load() -> ctypes.CDLL:
     lib.taco_attn_set_option.restype = i32
     lib.taco_attn_version.argtypes = []
     lib.taco_attn_version.restype = i32
+    lib.taco_attn_last_call_launches.argtypes = []
+    lib.taco_attn_last_call_launches.restype = i32
     lib.tree_mask_from_parents.argtypes = [vp, vp, i32, i32, vp, vp]
     lib.tree_mask_from_parents.restype = i32
     lib.logits_argmax.argtypes = [vp, i32, ctypes.c_int64, i32, vp, vp]
@@ -412,6 +416,11 @@ def release_workspace() -> None:
 
 def version() -> int:
     return int(load().taco_attn_version())
+
+
+def last_call_launches() -> int:
+    """Kernels the calling thread's last attention call enqueued (see include/taco_attn.h)."""
+    return int(load().taco_attn_last_call_launches())
 
 
 class PrefixCache:

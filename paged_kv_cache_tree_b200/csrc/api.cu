@@ -19,7 +19,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAbiVersion = 7;
+constexpr int kAbiVersion = 8;
 
 thread_local std::string g_last_error;
 
@@ -61,6 +61,9 @@ int64_t g_opt_kernel = 0;
 int64_t g_opt_prefetch = -1;  // -1 = the kernel's default distance
 int64_t g_opt_stall = 0;      // test knob: 0 = off, t + 1 = CTA 0 leaves tile t unarmed (mma.sync kernel)
 int64_t g_opt_seg_cost = -1;  // -1 = the kernel's default segment cost of the work split
+int64_t g_opt_combine = 0;    // 0 = automatic, 1 = merge inside the verify, 2 = separate combine kernel
+// kernels the calling thread's last attention call enqueued
+thread_local int g_last_launches = 0;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -210,6 +213,8 @@ extern "C" {
 
 int32_t taco_attn_version(void) { return kAbiVersion; }
 
+int32_t taco_attn_last_call_launches(void) { return g_last_launches; }
+
 const char* taco_attn_last_error(void) { return g_last_error.c_str(); }
 
 taco_status taco_attn_set_option(int32_t key, int64_t value) {
@@ -234,6 +239,11 @@ taco_status taco_attn_set_option(int32_t key, int64_t value) {
     g_opt_prefetch = value;
     return TACO_OK;
   }
+  if (key == TACO_OPT_COMBINE) {
+    if (value < 0 || value > 2) return fail(TACO_ERR_INVALID_ARG, "combine choice must be 0, 1 or 2");
+    g_opt_combine = value;
+    return TACO_OK;
+  }
   if (key == TACO_OPT_SEG_COST) {
     if (value < -1 || value > 64) return fail(TACO_ERR_INVALID_ARG, "segment cost must be in [-1, 64]");
     g_opt_seg_cost = value;
@@ -251,6 +261,7 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                   int32_t num_blocks, int32_t max_blocks_per_seq, void* stream) {
   const bool kv8 = k_scale != nullptr;
+  g_last_launches = 0;
   taco_status st = check_common(dtype, batch, max_candidates, num_kv_heads, head_dim, block_size, num_blocks,
                                 max_blocks_per_seq);
   if (st != TACO_OK) return st;
@@ -369,6 +380,10 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
     p.stall_tile = static_cast<int>(g_opt_stall);
     p.wait_limit_ns = 20000000ull;  // 20 ms
   }
+  // Split units with many pieces (few units against many CTAs, such as a handful of long sequences)
+  // are merged by a separate combine kernel, one warp per output row, instead of serially by the last
+  // CTA to finish each unit at the end of the verify.
+  p.defer_merge = !use_tc && (g_opt_combine == 2 || (g_opt_combine == 0 && units * 4 <= grid)) ? 1 : 0;
   p.seg_cost = static_cast<int>(g_opt_seg_cost >= 0 ? g_opt_seg_cost
                                 : (use_tc ? taco::tc_seg_cost(cands_per_group * G, kv8) : taco::mma_seg_cost(rows)));
   p.l2_prefetch_tiles = static_cast<int>(
@@ -391,6 +406,7 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
       e = kv8 ? taco::launch_append_e4m3(a, k_scale, v_scale, static_cast<cudaStream_t>(stream))
               : taco::launch_append(a, static_cast<cudaStream_t>(stream));
       if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+      ++g_last_launches;
       // the verify follows the append directly (16-bit caches: no query conversion in between), so
       // it may read everything but the appended slots before the append ends
       p.late_wait = kv8 ? 0 : 1;
@@ -402,15 +418,23 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
     e = taco::launch_q_to_f16(q, w.qbuf, reinterpret_cast<float*>(w.qbuf + q16_bytes), q_rows, head_dim,
                               static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "query conversion launch");
+    ++g_last_launches;
   }
 
   if (use_tc) {
     e = taco::launch_verify_tc(tk, tv, tq, p, dtype, grid, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "verify kernel launch");
+    ++g_last_launches;
     return TACO_OK;
   }
   e = taco::launch_verify_mma(tk, tv, p, dtype, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "verify kernel launch");
+  ++g_last_launches;
+  if (p.defer_merge) {
+    e = taco::launch_combine_split(p, dtype, grid, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+    ++g_last_launches;
+  }
   return TACO_OK;
 }
 

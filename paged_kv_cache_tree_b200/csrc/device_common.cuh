@@ -61,6 +61,9 @@ struct VerifyParams {
   // wait for it only before loading a tile that reaches key L_b - C, instead of at the start.
   int late_wait;
   int seg_cost;          // virtual tiles per unit in the work split (see the schedule below); 0 = equal split
+  // 1: split units only write their partials (no arrival counting, no merge); the combine kernel run
+  // after the verify merges them (mma.sync kernel only)
+  int defer_merge;
   // fused append (16-bit caches, units of <= 16 rows): candidate i's new K/V rows [B, C, Hkv, D] go to
   // logical slot P_b + i of these caches as the verify reads them; null = the caches are complete
   const void* k_new;

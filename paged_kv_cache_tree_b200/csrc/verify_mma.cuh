@@ -912,7 +912,7 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
         }
       }
     }
-    if (!whole_unit) {
+    if (!whole_unit && !p.defer_merge) {
       __threadfence();
       named_bar_sync(1, 128);
       const int u = (b * p.Hkv + g) * p.row_groups + rg;

@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.taco_attn_version() == 7
+    assert lib.taco_attn_version() == 8
 
 
 def _attn_args(**over):
@@ -94,6 +94,8 @@ def test_options(lib):
     assert lib.taco_attn_set_option(_lib.TACO_OPT_SEG_COST, -2) == _lib.TACO_ERR_INVALID_ARG
     assert lib.taco_attn_set_option(_lib.TACO_OPT_SEG_COST, 0) == _lib.TACO_OK
     assert lib.taco_attn_set_option(_lib.TACO_OPT_SEG_COST, -1) == _lib.TACO_OK
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_COMBINE, 3) == _lib.TACO_ERR_INVALID_ARG
+    assert lib.taco_attn_set_option(_lib.TACO_OPT_COMBINE, 0) == _lib.TACO_OK
 
 
 @pytest.mark.parametrize("call,status", [

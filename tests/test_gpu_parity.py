@@ -20,10 +20,12 @@ def _reset_options():
     taco.set_option(taco.TACO_OPT_GRID_CTAS, 0)
     taco.set_option(taco.TACO_OPT_KERNEL, 0)
     taco.set_option(taco.TACO_OPT_SEG_COST, -1)
+    taco.set_option(taco.TACO_OPT_COMBINE, 0)
     yield
     taco.set_option(taco.TACO_OPT_GRID_CTAS, 0)
     taco.set_option(taco.TACO_OPT_KERNEL, 0)
     taco.set_option(taco.TACO_OPT_SEG_COST, -1)
+    taco.set_option(taco.TACO_OPT_COMBINE, 0)
 
 
 def test_tiny_step_append_then_attend():
@@ -67,24 +69,27 @@ def test_small_shapes_full_oracle(case, kernel):
     assert_parity(out, ref, w)
 
 
-@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("kernel,combine", [(1, 1), (1, 2), (2, 0)])
 @pytest.mark.parametrize("grid", [1, 3, 7, 64, 500])
-def test_split_kv_partitions_agree(grid, kernel):
+def test_split_kv_partitions_agree(grid, kernel, combine):
+    """Forced grids split the units into 1 to hundreds of pieces; the mma.sync kernel's pieces are merged
+    inside the verify (combine 1) or by the separate combine kernel (combine 2)."""
     spec = dict(dtype="bf16", B=3, Hq=32, Hkv=4, D=128, bs=16, C=6, tree="forest", ctx=("uniform", 100, 900))
     w = wl.make_workload(spec, seed=7)
     ref, _, _ = oracle_step(w, append=False)
     taco.set_option(taco.TACO_OPT_GRID_CTAS, grid)
     taco.set_option(taco.TACO_OPT_KERNEL, kernel)
+    taco.set_option(taco.TACO_OPT_COMBINE, combine)
     out, _, _ = gpu_step(w, append=False)
     assert_parity(out, ref, w)
     again, _, _ = gpu_step(w, append=False)
     assert torch.equal(out.view(torch.int16), again.view(torch.int16)), "not deterministic run to run"
 
 
-@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("kernel,combine", [(1, 1), (1, 2), (2, 0)])
 @pytest.mark.parametrize("grid", [1, 5, 37, 300])
 @pytest.mark.parametrize("seg_cost", [0, 1, 3, 64])
-def test_weighted_work_split_agrees(seg_cost, grid, kernel):
+def test_weighted_work_split_agrees(seg_cost, grid, kernel, combine):
     """The work split counts seg_cost extra tiles per unit. Units of one tile next to long ones, and a
     cost far above the tiles of most units (whole CTA ranges then fall on no real tile), must still give
     every piece to exactly one CTA and merge it once."""
@@ -95,6 +100,7 @@ def test_weighted_work_split_agrees(seg_cost, grid, kernel):
     taco.set_option(taco.TACO_OPT_GRID_CTAS, grid)
     taco.set_option(taco.TACO_OPT_KERNEL, kernel)
     taco.set_option(taco.TACO_OPT_SEG_COST, seg_cost)
+    taco.set_option(taco.TACO_OPT_COMBINE, combine)
     out, _, _ = gpu_step(w, append=False)
     assert_parity(out, ref, w)
     again, _, _ = gpu_step(w, append=False)
@@ -303,3 +309,27 @@ def test_bounded_pipeline_wait_runs_out_and_reports():
     after = call()
     assert taco.check_device() == 0
     assert torch.equal(after.view(torch.int16), before.view(torch.int16))
+
+
+@pytest.mark.parametrize("dtype,D,combine", [("bf16", 128, 2), ("fp16", 64, 2), ("bf16", 128, 0)])
+def test_separate_combine_on_few_long_units_and_launch_count(dtype, D, combine):
+    """Two sequences of thousands of keys on a full grid: every unit is cut into dozens of pieces, which
+    the separate combine kernel merges (chosen automatically for so few units). The call reports its
+    launches: the append kernel, the verify and the combine."""
+    spec = dict(dtype=dtype, B=2, Hq=32, Hkv=4, D=D, bs=64, C=4, tree="chain", ctx=("uniform", 6000, 12000))
+    w = wl.make_workload(spec, seed=21, candidates_in_cache=False)
+    taco.set_option(taco.TACO_OPT_COMBINE, combine)
+    d = w.to("cuda")
+    out = torch.full_like(d.q, float("nan"))
+    taco.paged_tree_attention_append(d.q, d.k_new, d.v_new, d.k_cache, d.v_cache, d.block_tables, d.context_lens,
+                                     d.num_candidates, d.tree_mask, w.scale, out=out)
+    assert taco.last_call_launches() == 3
+    assert taco.check_device() == 0
+    ref, _, _ = oracle_step(w)
+    assert_parity(out.cpu(), ref, w)
+    # the same call twice gives the same bits
+    again = torch.full_like(d.q, float("nan"))
+    taco.paged_tree_attention(d.q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, d.num_candidates,
+                              d.tree_mask, w.scale, out=again)
+    assert taco.last_call_launches() == 2
+    assert torch.equal(out.view(torch.int16), again.view(torch.int16))
