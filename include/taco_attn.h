@@ -418,11 +418,11 @@ void taco_attn_release_workspace(void);
                                   0 = off (default); t + 1 = the first CTA's producers never arm the
                                   stage of its tile t, so that a consumer's wait runs out after 20 ms,
                                   the call reports TACO_DEVERR_WAIT_TIMEOUT and its output is undefined */
-#define TACO_OPT_COMBINE 6     /* split-KV combine of the mma.sync verify: 0 = automatic (a separate combine
+#define TACO_OPT_COMBINE 6     /* split-KV combine: 0 = automatic (mma.sync verify: a separate combine
                                   kernel when the call has at most a quarter as many work units as
-                                  CTAs, so that units are cut into many pieces; else inside the verify),
+                                  CTAs, so that units are cut into many pieces; tcgen05 verify: inside),
                                   1 = inside the verify, by the last CTA to finish each unit, 2 = the
-                                  separate kernel, one warp per output row */
+                                  separate kernel for either verify */
 taco_status taco_attn_set_option(int32_t key, int64_t value);
 
 /* Kernels the calling thread's last attention call (paged_tree_attention, _append, _e4m3,

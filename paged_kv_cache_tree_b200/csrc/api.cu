@@ -383,7 +383,7 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
   // Split units with many pieces (few units against many CTAs, such as a handful of long sequences)
   // are merged by a separate combine kernel, one warp per output row, instead of serially by the last
   // CTA to finish each unit at the end of the verify.
-  p.defer_merge = !use_tc && (g_opt_combine == 2 || (g_opt_combine == 0 && units * 4 <= grid)) ? 1 : 0;
+  p.defer_merge = (g_opt_combine == 2 || (g_opt_combine == 0 && !use_tc && units * 4 <= grid)) ? 1 : 0;
   p.seg_cost = static_cast<int>(g_opt_seg_cost >= 0 ? g_opt_seg_cost
                                 : (use_tc ? taco::tc_seg_cost(cands_per_group * G, kv8) : taco::mma_seg_cost(rows)));
   p.l2_prefetch_tiles = static_cast<int>(
@@ -421,17 +421,14 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
     ++g_last_launches;
   }
 
-  if (use_tc) {
+  if (use_tc)
     e = taco::launch_verify_tc(tk, tv, tq, p, dtype, grid, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "verify kernel launch");
-    ++g_last_launches;
-    return TACO_OK;
-  }
-  e = taco::launch_verify_mma(tk, tv, p, dtype, grid, static_cast<cudaStream_t>(stream));
+  else
+    e = taco::launch_verify_mma(tk, tv, p, dtype, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "verify kernel launch");
   ++g_last_launches;
   if (p.defer_merge) {
-    e = taco::launch_combine_split(p, dtype, grid, static_cast<cudaStream_t>(stream));
+    e = taco::launch_combine_split(p, dtype, grid, use_tc, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
     ++g_last_launches;
   }

@@ -62,9 +62,9 @@ int mma_smem_bytes(int D, int rows_per_unit, bool kv8 = false);
 int mma_tile_keys(int rows_per_unit, bool kv8);
 cudaError_t launch_verify_mma(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p,
                               int dtype, int grid, cudaStream_t stream);
-// The split units' log-sum-exp combine after a verify launched with defer_merge (mma.sync partials),
-// `grid` = that verify's grid.
-cudaError_t launch_combine_split(const VerifyParams& p, int dtype, int grid, cudaStream_t stream);
+// The split units' log-sum-exp combine after a verify launched with defer_merge, `grid` = that
+// verify's grid; transposed = the tcgen05 kernel's partial layout ([slot][D][128]).
+cudaError_t launch_combine_split(const VerifyParams& p, int dtype, int grid, bool transposed, cudaStream_t stream);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 // Quantising append into an e4m3 cache: code = e4m3(x / scale[h]) (round to nearest even, saturating).
 cudaError_t launch_append_e4m3(const AppendArgs& a, const float* k_scale, const float* v_scale, cudaStream_t stream);

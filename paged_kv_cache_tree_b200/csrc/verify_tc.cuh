@@ -906,7 +906,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&sh->o_free));
 
-    if (!whole_unit) {
+    if (!whole_unit && !p.defer_merge) {
       // the CTA that arrives last on the unit's counter combines every piece's partial
       __threadfence();
       named_bar_sync(1, 256);

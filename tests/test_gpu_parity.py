@@ -69,11 +69,11 @@ def test_small_shapes_full_oracle(case, kernel):
     assert_parity(out, ref, w)
 
 
-@pytest.mark.parametrize("kernel,combine", [(1, 1), (1, 2), (2, 0)])
+@pytest.mark.parametrize("kernel,combine", [(1, 1), (1, 2), (2, 1), (2, 2)])
 @pytest.mark.parametrize("grid", [1, 3, 7, 64, 500])
 def test_split_kv_partitions_agree(grid, kernel, combine):
-    """Forced grids split the units into 1 to hundreds of pieces; the mma.sync kernel's pieces are merged
-    inside the verify (combine 1) or by the separate combine kernel (combine 2)."""
+    """Forced grids split the units into 1 to hundreds of pieces; either kernel's pieces are merged inside
+    the verify (combine 1) or by the separate combine kernel (combine 2)."""
     spec = dict(dtype="bf16", B=3, Hq=32, Hkv=4, D=128, bs=16, C=6, tree="forest", ctx=("uniform", 100, 900))
     w = wl.make_workload(spec, seed=7)
     ref, _, _ = oracle_step(w, append=False)
@@ -86,7 +86,7 @@ def test_split_kv_partitions_agree(grid, kernel, combine):
     assert torch.equal(out.view(torch.int16), again.view(torch.int16)), "not deterministic run to run"
 
 
-@pytest.mark.parametrize("kernel,combine", [(1, 1), (1, 2), (2, 0)])
+@pytest.mark.parametrize("kernel,combine", [(1, 1), (1, 2), (2, 1), (2, 2)])
 @pytest.mark.parametrize("grid", [1, 5, 37, 300])
 @pytest.mark.parametrize("seg_cost", [0, 1, 3, 64])
 def test_weighted_work_split_agrees(seg_cost, grid, kernel, combine):
