@@ -50,7 +50,8 @@ DEFAULT_WORKLOAD = "long"
 # the other full-size workloads, each measured in the same run under "per_config"
 PER_CONFIG = ("decode", "chain", "tree", "long")
 CLOCK_WINDOW_S = 1.5
-KERNEL_SOURCES = ("device_common.cuh", "verify_mma.cuh", "verify_mma.cu", "verify_tc.cuh", "verify_tc.cu")
+KERNEL_SOURCES = ("device_common.cuh", "verify_mma.cuh", "verify_mma.cu", "verify_tc.cuh", "verify_tc.cu",
+                  "combine.cu")
 
 
 def time_at_roofline(bytes_moved: float, flops: float, bw_gbs: float, tflops: float):
