@@ -91,6 +91,9 @@ typedef int32_t taco_status;
  * (device, stream); the first call on a stream (or one that needs a larger workspace) allocates it
  * with cudaMalloc and therefore synchronises the device. Calls on different streams use different
  * workspaces and may overlap on the GPU.
+ * Kernels: one verify launch; when a call has few work units against the grid (a handful of long
+ * sequences, whose units are then cut into many split-KV pieces), a second, separate combine kernel
+ * merges the pieces (TACO_OPT_COMBINE; taco_attn_last_call_launches reports what a call enqueued).
  */
 taco_status paged_tree_attention(const void* q, const void* k_cache, const void* v_cache,
                                  const int32_t* block_tables, const int32_t* context_lens,
