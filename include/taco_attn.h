@@ -232,9 +232,14 @@ taco_status paged_tree_attention_e4m3(const void* q, const void* k_cache, const 
 /*
  * paged_tree_attention_append_e4m3: paged_kv_append_e4m3 of each sequence's candidates into logical
  * slots P_b .. L_b - 1 (slot_offsets derived as for paged_tree_attention_append), then
- * paged_tree_attention_e4m3 over the updated caches, in one call: the quantising append kernel runs
- * first on `stream` and the verify waits for it on the device. k_new, v_new: [B, C, Hkv, D] `dtype`.
- * Every other argument, rule and error is that of the two calls.
+ * paged_tree_attention_e4m3 over the updated caches, in one call. k_new, v_new: [B, C, Hkv, D] `dtype`.
+ * On the mma.sync kernel (head_dim 128) with units of at most 16 packed query rows, the verify kernel
+ * quantises the candidates' rows itself: the CTA that loads the tile holding a candidate's key divides
+ * each new value by its head's scale and rounds it to e4m3 exactly as paged_kv_append_e4m3 does, then
+ * writes the codes into its shared-memory copy of the tile and into the cache. One launch, no append
+ * kernel. Otherwise the quantising append kernel runs first on `stream`. The verify then reads all
+ * but the appended slots before the append ends, unless a query conversion runs in between (bf16
+ * queries on the tcgen05 kernel). Every other argument, rule and error is that of the two calls.
  */
 taco_status paged_tree_attention_append_e4m3(const void* q, const void* k_new, const void* v_new, void* k_cache,
                                              void* v_cache, const float* k_scale, const float* v_scale,

@@ -392,9 +392,9 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
   p.v_scale = v_scale;
   p.q_scale = q_convert ? reinterpret_cast<const float*>(w.qbuf + q16_bytes) : nullptr;
   if (k_new) {
-    // fused append where the kernel supports it (mma.sync, <= 16 rows, 16-bit caches); otherwise the
-    // append kernel runs first on the same stream
-    if (!use_tc && rows <= 16 && !kv8) {
+    // fused append where the kernel supports it (mma.sync, <= 16 rows; with e4m3 caches it quantises
+    // as the append kernel does); otherwise the append kernel runs first on the same stream
+    if (!use_tc && rows <= 16) {
       p.k_new = k_new;
       p.v_new = v_new;
       p.k_cache = const_cast<void*>(k_cache);
@@ -407,9 +407,9 @@ static taco_status attention_impl(const void* q, const void* k_cache, const void
               : taco::launch_append(a, static_cast<cudaStream_t>(stream));
       if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
       ++g_last_launches;
-      // the verify follows the append directly (16-bit caches: no query conversion in between), so
-      // it may read everything but the appended slots before the append ends
-      p.late_wait = kv8 ? 0 : 1;
+      // unless a query conversion runs in between, the verify follows the append directly and may
+      // read everything but the appended slots before the append ends
+      p.late_wait = q_convert ? 0 : 1;
     }
   }
   // after the append (a plain launch: it starts once the append has finished, and the verify's

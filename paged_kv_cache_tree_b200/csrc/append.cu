@@ -44,24 +44,6 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   static_cast<uint4*>(a.v_cache)[dst] = vv;
 }
 
-// e4m3 of two floats (first in the low byte), round to nearest even, saturating at +-448
-__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float first, float second) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
-  return r;
-}
-
-template <typename T>
-__device__ __forceinline__ float elt_to_f32(T x);
-template <>
-__device__ __forceinline__ float elt_to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
-  return __bfloat162float(x);
-}
-template <>
-__device__ __forceinline__ float elt_to_f32<__half>(__half x) {
-  return __half2float(x);
-}
-
 // Quantising append into an e4m3 cache [NB, Hkv, bs, D] (one byte per value): one thread per 16-byte
 // piece (8 values) of a (sequence, candidate, KV head) row of k_new / v_new, writing 8 bytes; each
 // value is divided by its KV head's scale (float32, correctly rounded) and rounded to e4m3.
@@ -97,20 +79,10 @@ __global__ void __launch_bounds__(256) append_e4m3_kernel(AppendArgs a, const fl
   const float ks = __ldg(k_scale + h), vs = __ldg(v_scale + h);
   const uint4 kin = __ldg(static_cast<const uint4*>(a.k_new) + row * VEC_PER_ROW + v);
   const uint4 vin = __ldg(static_cast<const uint4*>(a.v_new) + row * VEC_PER_ROW + v);
-  const T* ke = reinterpret_cast<const T*>(&kin);
-  const T* ve = reinterpret_cast<const T*>(&vin);
-  uint16_t kq[4], vq[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    kq[e] = f32x2_to_e4m3x2(__fdiv_rn(elt_to_f32<T>(ke[2 * e]), ks), __fdiv_rn(elt_to_f32<T>(ke[2 * e + 1]), ks));
-    vq[e] = f32x2_to_e4m3x2(__fdiv_rn(elt_to_f32<T>(ve[2 * e]), vs), __fdiv_rn(elt_to_f32<T>(ve[2 * e + 1]), vs));
-  }
   // 8 bytes per thread: cache row (blk, h, slot) is D bytes, this piece starts at byte v * 8
   const int64_t dst = ((static_cast<int64_t>(blk) * a.Hkv + h) * a.bs + s % a.bs) * VEC_PER_ROW + v;
-  static_cast<uint2*>(a.k_cache)[dst] = make_uint2(kq[0] | (static_cast<uint32_t>(kq[1]) << 16),
-                                                   kq[2] | (static_cast<uint32_t>(kq[3]) << 16));
-  static_cast<uint2*>(a.v_cache)[dst] = make_uint2(vq[0] | (static_cast<uint32_t>(vq[1]) << 16),
-                                                   vq[2] | (static_cast<uint32_t>(vq[3]) << 16));
+  static_cast<uint2*>(a.k_cache)[dst] = quantise_e4m3x8<T>(kin, ks);
+  static_cast<uint2*>(a.v_cache)[dst] = quantise_e4m3x8<T>(vin, vs);
 }
 
 cudaError_t launch_append_e4m3(const AppendArgs& a, const float* k_scale, const float* v_scale, cudaStream_t stream) {

@@ -231,6 +231,37 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   return h;
 }
 
+// e4m3 of two floats (first in the low byte), round to nearest even, saturating at +-448
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float first, float second) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
+  return r;
+}
+
+template <typename T>
+__device__ __forceinline__ float elt_to_f32(T x);
+template <>
+__device__ __forceinline__ float elt_to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <>
+__device__ __forceinline__ float elt_to_f32<__half>(__half x) {
+  return __half2float(x);
+}
+
+// The quantising append's arithmetic on 8 values (one 16-byte piece of a 16-bit row): each value
+// divided by the KV head's scale (float32, correctly rounded), then rounded to e4m3; 8 codes, the
+// first value's in the lowest byte.
+template <typename T>
+__device__ __forceinline__ uint2 quantise_e4m3x8(uint4 in, float scale) {
+  const T* e = reinterpret_cast<const T*>(&in);
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    q[i] = f32x2_to_e4m3x2(__fdiv_rn(elt_to_f32<T>(e[2 * i]), scale), __fdiv_rn(elt_to_f32<T>(e[2 * i + 1]), scale));
+  return make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+}
+
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));

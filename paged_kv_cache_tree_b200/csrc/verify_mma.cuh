@@ -441,6 +441,43 @@ __global__ void __launch_bounds__(MmaCfg<D, MT>::kThreads, MmaCfg<D, MT>::kCtasP
           __syncwarp();
         }
       }
+      if constexpr (KV8 && MTS == 1) {
+        // fused quantising append (e4m3 caches), the same division of rows between warps: each new
+        // K/V row is divided by its KV head's scale and rounded to e4m3 as the append kernel does,
+        // 16 codes (two 16-byte pieces of the 16-bit row) per 16-byte chunk of the stage and the cache
+        if (ready && p.k_new != nullptr && key0 + Cfg::kTile > P) {
+          const int p_lo = key0 + wkey0 > P ? key0 + wkey0 : P;
+          const int p_hi = key0 + wkey0 + KW < L ? key0 + wkey0 + KW : L;
+          constexpr int CH = D / 16;  // 16-code chunks per row
+          const float ksc = __ldg(p.k_scale + g), vscl = __ldg(p.v_scale + g);
+          uint8_t* kgen = stages + stage * Cfg::kStageBytes;
+          for (int idx = lane; idx < (p_hi - p_lo) * 2 * CH; idx += 32) {
+            const int pos = p_lo + idx / (2 * CH);
+            const int rem = idx % (2 * CH);
+            const bool is_v = rem >= CH;
+            const int c = rem % CH;
+            const int64_t src_row = (static_cast<int64_t>(b) * p.C + (pos - P)) * p.Hkv + g;
+            const uint4* src =
+                reinterpret_cast<const uint4*>(static_cast<const T*>(is_v ? p.v_new : p.k_new) + src_row * D) + 2 * c;
+            const float sc = is_v ? vscl : ksc;
+            const uint2 lo8 = quantise_e4m3x8<T>(__ldg(src), sc);
+            const uint2 hi8 = quantise_e4m3x8<T>(__ldg(src + 1), sc);
+            const uint4 codes = make_uint4(lo8.x, lo8.y, hi8.x, hi8.y);
+            const int r = pos - key0;
+            *reinterpret_cast<uint4*>(kgen + (is_v ? Cfg::kTensorBytes : 0) + r * 128 + ((c ^ (r & 7)) << 4)) = codes;
+            const int blk = __ldg(p.block_tables + static_cast<int64_t>(b) * p.max_blocks + pos / p.bs);
+            if (blk >= 0 && blk < p.num_blocks) {
+              uint8_t* cache = static_cast<uint8_t*>(is_v ? p.v_cache : p.k_cache);
+              reinterpret_cast<uint4*>(cache + ((static_cast<int64_t>(blk) * p.Hkv + g) * p.bs + pos % p.bs) * D)[c] =
+                  codes;
+            } else if (c == 0 && !is_v) {
+              atomicOr(p.error_word, TACO_DEVERR_BLOCK_ID);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+      }
       if (ready) {
         if constexpr (SW) {
           // ---- swapped form. S^T = K Q^T: m tile m holds keys wkey0 + m*16 .. +15 (rows gq, gq+8 of the

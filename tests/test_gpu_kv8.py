@@ -209,3 +209,68 @@ def test_append_and_attend_in_one_call(spec):
     assert np.array_equal(g8.v_cache.cpu().numpy(), rv)
     ref = oracle_attention_e4m3(w, c8, k_cache=torch.from_numpy(rk), v_cache=torch.from_numpy(rv))
     assert_parity(out.cpu(), ref, w)
+
+
+def _one_call_e4m3(w, c8):
+    d, g8 = w.to("cuda"), c8.to("cuda")
+    out = torch.full_like(d.q, float("nan"))
+    taco.paged_tree_attention_e4m3(d.q, g8.k_cache, g8.v_cache, g8.k_scale, g8.v_scale, d.block_tables,
+                                   d.context_lens, d.num_candidates, d.tree_mask, w.scale, out=out,
+                                   k_new=d.k_new, v_new=d.v_new)
+    assert taco.check_device() == 0
+    launches = taco.last_call_launches()
+    rk, rv = fp8.paged_kv_append_e4m3(wl.to_numpy_bits(w.k_new), wl.to_numpy_bits(w.v_new), w.dtype,
+                                      w.block_tables.numpy(), w.slot_offsets.numpy(), c8.k_scale.numpy(),
+                                      c8.v_scale.numpy(), c8.k_cache.numpy(), c8.v_cache.numpy())
+    assert np.array_equal(g8.k_cache.cpu().numpy(), rk)
+    assert np.array_equal(g8.v_cache.cpu().numpy(), rv)
+    return out.cpu(), rk, rv, launches
+
+
+def _launches_16bit(w):
+    d = w.to("cuda")
+    out = torch.empty_like(d.q)
+    taco.paged_tree_attention_append(d.q, d.k_new, d.v_new, d.k_cache, d.v_cache, d.block_tables, d.context_lens,
+                                     d.num_candidates, d.tree_mask, w.scale, out=out)
+    assert taco.check_device() == 0
+    return taco.last_call_launches()
+
+
+@pytest.mark.parametrize("grid", [0, 5, 300])
+@pytest.mark.parametrize("spec", [
+    # 16 packed rows (one 16-row tile per unit)
+    dict(dtype="bf16", B=5, Hq=32, Hkv=8, D=128, bs=16, C=4, tree="forest", ctx=("uniform", 4, 700)),
+    # 8 and 4 packed rows (the swapped form)
+    dict(dtype="fp16", B=4, Hq=64, Hkv=8, D=128, bs=64, C=1, tree="chain", ctx=("uniform", 1, 900)),
+    dict(dtype="bf16", B=4, Hq=8, Hkv=4, D=128, bs=32, C=2, tree="forest", ctx=("fixed", [2, 31, 129, 600])),
+])
+def test_fused_quantising_append_on_narrow_units(spec, grid):
+    """Units of <= 16 packed rows quantise the candidates' rows inside the verify kernel, as the 16-bit
+    path copies them: the call launches no append kernel (the same launches as the 16-bit one-call
+    path), the caches equal the quantising-append oracle byte for byte (rounding probes included: ties,
+    saturation, infinities, subnormals, signed zeros), and the output the attention oracle over them.
+    Grids of 5 and 300 CTAs cut the units (and the candidates' tiles) into pieces."""
+    w = wl.make_workload(spec, seed=90 + spec["C"] + spec["bs"], candidates_in_cache=False)
+    k, v = special_rows(w)
+    # NaN probes stay with the append-only tests: here every row is attended
+    w.k_new, w.v_new = torch.nan_to_num(k, nan=0.75), torch.nan_to_num(v, nan=-0.75)
+    c8 = wl.make_e4m3_cache(w)
+    taco.set_option(taco.TACO_OPT_GRID_CTAS, grid)
+    got, rk, rv, launches = _one_call_e4m3(w, c8)
+    ref = oracle_attention_e4m3(w, c8, k_cache=torch.from_numpy(rk), v_cache=torch.from_numpy(rv))
+    assert_parity(got, ref, w)
+    assert launches == _launches_16bit(w)
+
+
+@pytest.mark.parametrize("name", ["decode", "long"])
+def test_full_size_one_call_sampled_rows(name):
+    """paged_tree_attention_append_e4m3 on the full decode workload (the append fused into the
+    verify) and on the full long workload (the append kernel, then the verify reading all but the
+    appended slots before the append ends): caches byte-exact, one row of every unit plus 24 sampled
+    rows against the oracle."""
+    w = wl.make_workload(name, candidates_in_cache=False)
+    c8 = wl.make_e4m3_cache(w)
+    got, rk, rv, _ = _one_call_e4m3(w, c8)
+    rows = full_size_rows(w, seed=2)
+    ref = oracle_attention_e4m3(w, c8, rows=rows, k_cache=torch.from_numpy(rk), v_cache=torch.from_numpy(rv))
+    assert_parity(got, ref, w, rows=rows)
