@@ -38,7 +38,7 @@ namespace taco {
 // every tile.
 constexpr int kTcTileKeys = 128;
 
-// KV8: e4m3 caches. Their tiles land in rings of raw codes and the producer warps widen each one
+// KV8: e4m3 caches. Their tiles land in rings of raw codes and the eight softmax warps widen each one
 // once (exactly) into a 16-bit stage of the same layout as a 16-bit cache's, so everything downstream
 // is the 16-bit pipeline with f16 operands.
 template <int D, bool KV8 = false>
@@ -71,7 +71,7 @@ struct TcShared {
   // p_full[2 sb + w]: warpgroup w wrote its half of P into S buffer sb.
   uint64_t k_full[6], k_empty[6], v_full[6], v_empty[6];
   uint64_t q_full, q_empty, s_full[2], p_full[4], o_free;
-  // e4m3 caches: raw tiles of K (index 0) and V (index 1) landed / free again
+  // e4m3 caches: raw tiles of K (index 0) and V (index 1) landed / widened by all eight softmax warps
   uint64_t raw_full[2][4], raw_empty[2][4];
   uint32_t tmem_base;
   int merge_flag, abort_flag;
@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(384, 1)
   constexpr uint32_t kIdescQK = tc::idesc_f16(kBf16 ? 1 : 0, 128, TK, 0);
   constexpr uint32_t kIdescPV = tc::idesc_f16(kBf16 ? 1 : 0, 128, D, 1);
   static_assert(sizeof(TcShared) <= Cfg::kSharedBytes, "shared bookkeeping too large");
+  static_assert(!KV8 || SK == SV, "e4m3 widening indexes K and V stages alike");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -192,12 +193,15 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = tid & 31;
 
   if (tid == 0) {
+    // e4m3 caches: the eight softmax warps complete a stage (each widens sixteen rows of it) and free
+    // a raw slot; 16-bit caches: the producer's TMA completes the stage
+    constexpr uint32_t kFullArrivals = KV8 ? 8u : 1u;
     for (int s = 0; s < SK; ++s) {
-      mbar_init(smem_addr(&sh->k_full[s]), 1);
+      mbar_init(smem_addr(&sh->k_full[s]), kFullArrivals);
       mbar_init(smem_addr(&sh->k_empty[s]), 1);
     }
     for (int s = 0; s < SV; ++s) {
-      mbar_init(smem_addr(&sh->v_full[s]), 1);
+      mbar_init(smem_addr(&sh->v_full[s]), kFullArrivals);
       mbar_init(smem_addr(&sh->v_empty[s]), 1);
     }
     mbar_init(smem_addr(&sh->q_full), 1);
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int t = 0; t < 2; ++t)
       for (int s = 0; s < RS; ++s) {
         mbar_init(smem_addr(&sh->raw_full[t][s]), 1);
-        mbar_init(smem_addr(&sh->raw_empty[t][s]), 1);
+        mbar_init(smem_addr(&sh->raw_empty[t][s]), 8);
       }
     sh->merge_flag = 0;
     sh->abort_flag = 0;
@@ -260,12 +264,11 @@ __global__ void __launch_bounds__(384, 1)
 
   if constexpr (KV8) {
     if (warp == 0 || warp == 10) {
-      // -------------------------------------------------------------- e4m3 producers
-      // Warp 0 streams Q (f16, 3-D box) and K, warp 10 streams V. Each loads raw tiles of codes into a
-      // ring of RS slots up to RS tiles ahead, and widens every landed tile, in tile order, into a
-      // 16-bit stage in the layout a 16-bit cache's TMA load leaves (two 64-column 128-byte-swizzled
-      // panels): cvt.rn.f16x2.e4m3x2 is exact, so the stage holds exactly decode(code); the scale per
-      // KV head is applied to the scores and to O instead.
+      // -------------------------------------------------------------- e4m3 loaders
+      // Warp 0 streams Q (f16, 3-D box) and K, warp 10 streams V: raw tiles of codes into a ring of
+      // RS slots, in tile order, as far ahead as the slots allow. The eight softmax warps widen each
+      // landed tile (sixteen rows each) into the 16-bit stage the tensor cores read and free the slot
+      // (raw_empty counts their eight arrivals).
       const int t = (warp == 0) ? 0 : 1;
       const bool is_k = (t == 0);
       const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
@@ -276,121 +279,62 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t chunk_bytes = static_cast<uint32_t>(rpc) * D;
       const uint32_t q_bytes = static_cast<uint32_t>(Cfg::kPanels * qrows * 128);
       uint8_t* raw = rawring + t * RS * Cfg::kRawBytes;
-      uint8_t* conv = is_k ? kring : vring;
-      uint64_t* conv_full = is_k ? sh->k_full : sh->v_full;
-      uint64_t* conv_empty = is_k ? sh->k_empty : sh->v_empty;
-      constexpr int SC = SK;  // converted stages (SK == SV)
       TileLoadCursor lc;
       lc.init(p, sh->b, sh->base_b, lo, hi, is_k);
-      TileWalker cw;  // conversion order (same tiles)
-      cw.init(p, sh->b, sh->base_b, lo, hi);
-      TileInfo ti;
       bool ok = true;
-      int64_t kc = 0;
       int q_issued_ui = -1;
-      // raw load of the cursor's current tile into slot lc.k % RS
-      auto issue_raw = [&]() {
+      while (lc.have) {
+        const bool seg_first = (lc.tl == lc.c.tile);
+        const int ui = lc.c.ui;
+        const int qb = lc.c.b, qj = lc.c.j;
         int row, nload;
         const bool mine = lc.chunk(p, TK, rpc, &row, &nload);
         const int rs = static_cast<int>(lc.k % RS);
         bool go = true;
         if (lane == 0) {
+          // the slot's previous tile (RS tiles back) has been widened by all eight softmax warps
           go = ok && (*abort_flag == 0) &&
-               mbar_wait(smem_addr(&sh->raw_empty[t][rs]), static_cast<uint32_t>(((lc.k / RS) & 1) ^ 1), p.error_word);
+               (lc.k < RS ||
+                mbar_wait(smem_addr(&sh->raw_empty[t][rs]), static_cast<uint32_t>(((lc.k / RS) - 1) & 1), p.error_word));
           if (!go) *abort_flag = 1;
+          // armed on abort too (with no bytes), so that a widening warp never waits on it forever
           mbar_arrive_expect_tx(smem_addr(&sh->raw_full[t][rs]), go ? static_cast<uint32_t>(nload) * chunk_bytes : 0u);
         }
         go = __shfl_sync(0xffffffffu, go, 0);
         if (!go) ok = false;
         if (go && mine)
-          tma_load_2d(smem_addr(raw + rs * Cfg::kRawBytes) + (threadIdx.x & 31) * chunk_bytes, tmap,
-                      smem_addr(&sh->raw_full[t][rs]), 0, row, policy);
+          tma_load_2d(smem_addr(raw + rs * Cfg::kRawBytes) + lane * chunk_bytes, tmap, smem_addr(&sh->raw_full[t][rs]),
+                      0, row, policy);
         __syncwarp();
-        lc.step(p);
-      };
-      while (cw.next(p, ti)) {
-        // keep up to RS raw tiles in flight ahead of the conversion
-        while (lc.have && lc.k < kc + RS) issue_raw();
-        if (is_k && ti.first && q_issued_ui < ti.ui) {
-          // the segment's Q tile: the single Q buffer is free once the previous segment's last Q K^T
-          // is done (that needs only tiles converted already, so this wait always ends)
+        if (is_k && seg_first && q_issued_ui < ui) {
+          // the segment's Q tile, after its first raw K tile: the single Q buffer is free once the
+          // previous segment's last Q K^T is done, which needs only tiles already loaded
           if (lane == 0) {
-            const bool go = ok && (*abort_flag == 0) &&
-                            mbar_wait(smem_addr(&sh->q_empty), static_cast<uint32_t>((ti.ui & 1) ^ 1), p.error_word);
-            if (!go) {
-              ok = false;
-              *abort_flag = 1;
-            }
-            mbar_arrive_expect_tx(smem_addr(&sh->q_full), go ? q_bytes : 0u);
-            if (go) {
+            bool gq = ok && (*abort_flag == 0) &&
+                      mbar_wait(smem_addr(&sh->q_empty), static_cast<uint32_t>((ui & 1) ^ 1), p.error_word);
+            if (!gq) *abort_flag = 1;
+            mbar_arrive_expect_tx(smem_addr(&sh->q_full), gq ? q_bytes : 0u);
+            if (gq) {
 #pragma unroll
               for (int pn = 0; pn < Cfg::kPanels; ++pn)
                 tma_load_3d(smem_addr(qbuf) + pn * Cfg::kQPanelBytes, &tmap_q, smem_addr(&sh->q_full), pn * 64,
-                            (ti.j / p.row_groups) * p.G, ti.b * p.C + (ti.j % p.row_groups) * cpg);
+                            (qj / p.row_groups) * p.G, qb * p.C + (qj % p.row_groups) * cpg);
             }
+            if (!gq) ok = false;
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
-          q_issued_ui = ti.ui;
+          q_issued_ui = ui;
         }
-        const int rs = static_cast<int>(kc % RS);
-        const int cs = static_cast<int>(kc % SC);
-        bool go = true;
-        if (lane == 0) {
-          go = ok && (*abort_flag == 0) &&
-               mbar_wait(smem_addr(&sh->raw_full[t][rs]), static_cast<uint32_t>((kc / RS) & 1), p.error_word) &&
-               mbar_wait(smem_addr(&conv_empty[cs]), static_cast<uint32_t>(((kc / SC) & 1) ^ 1), p.error_word);
-          if (!go) *abort_flag = 1;
-        }
-        go = __shfl_sync(0xffffffffu, go, 0);
-        if (!go) ok = false;
-        if (go) {
-          const uint8_t* src = raw + rs * Cfg::kRawBytes;
-          uint8_t* dst = conv + cs * Cfg::kTensorBytes;
-          constexpr int CPR = D / 16;          // 16-code chunks per key row
-          constexpr int NCH = TK * CPR / 32;   // chunks per lane and tile (32 or 16)
-          constexpr int BATCH = 8;             // chunks whose loads are issued before any is used
-          static_assert(NCH % BATCH == 0, "conversion batches");
-#pragma unroll 1
-          for (int b0 = 0; b0 < NCH; b0 += BATCH) {
-            uint4 v[BATCH];
-#pragma unroll
-            for (int j = 0; j < BATCH; ++j) {
-              const int idx = (b0 + j) * 32 + lane;
-              v[j] = lds_v4(smem_addr(src + (idx / CPR) * D + (idx % CPR) * 16));
-            }
-#pragma unroll
-            for (int j = 0; j < BATCH; ++j) {
-              const int idx = (b0 + j) * 32 + lane;
-              const int row = idx / CPR;
-              const int c = idx % CPR;
-              const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-              uint32_t h[8];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                h[2 * q] = e4m3x2_to_f16x2(w[q] & 0xffffu);
-                h[2 * q + 1] = e4m3x2_to_f16x2(w[q] >> 16);
-              }
-              // head dims [16c, 16c + 16) = 16-byte chunks 2(c % 4), 2(c % 4) + 1 of panel c / 4, swizzled
-              uint8_t* prow = dst + (c >> 2) * Cfg::kPanelBytes + row * 128;
-              const int j0 = 2 * (c & 3);
-              *reinterpret_cast<uint4*>(prow + ((j0 ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
-              *reinterpret_cast<uint4*>(prow + (((j0 + 1) ^ (row & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
-            }
-          }
-          fence_proxy_async_smem();
-        }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(smem_addr(&conv_full[cs]));  // on abort too: nobody waits for a tile forever
-          mbar_arrive(smem_addr(&sh->raw_empty[t][rs]));
-        }
-        ++kc;
+        lc.step(p);
       }
-      // wait (bounded) for our own copies still landing: raw tiles issued but not converted (after an
-      // abort) and the last Q tile
+      // wait (bounded) for our own copies still landing: the last use of every raw slot, and the
+      // last Q tile
       if (lane == 0) {
-        for (int64_t kk = kc; kk < lc.k; ++kk)
-          mbar_wait(smem_addr(&sh->raw_full[t][kk % RS]), static_cast<uint32_t>((kk / RS) & 1), p.error_word);
+        for (int s = 0; s < RS; ++s) {
+          const int64_t uses = lc.k / RS + (s < lc.k % RS ? 1 : 0);
+          if (uses > 0)
+            mbar_wait(smem_addr(&sh->raw_full[t][s]), static_cast<uint32_t>((uses - 1) & 1), p.error_word);
+        }
         if (is_k && q_issued_ui >= 0)
           mbar_wait(smem_addr(&sh->q_full), static_cast<uint32_t>(q_issued_ui & 1), p.error_word);
       }
@@ -638,6 +582,70 @@ __global__ void __launch_bounds__(384, 1)
   const int r = sub * 32 + lane;              // query row owned by this thread
   const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
   const uint32_t my_o = tmem + lane_base + Cfg::kOCol + static_cast<uint32_t>(wg * 128);
+  // e4m3 caches: softmax warp sw widens rows [16 sw, 16 sw + 16) of tile kk's raw K (t = 0) or V
+  // (t = 1) codes into the tile's 16-bit stage, in the layout a 16-bit cache's TMA load leaves (two
+  // 64-column 128-byte-swizzled panels at D = 128): cvt.rn.f16x2.e4m3x2 is exact, so the stage holds
+  // exactly decode(code); the scales per KV head act on the scores and on O. Rows from zero_from on
+  // (keys past the context) are written as zeros. The stage's previous tile must be done with it (its
+  // Q K^T or P V complete; both needed only tiles widened earlier). Then this warp's arrival on the
+  // stage's full barrier and on the raw slot's empty barrier (eight each); on abort too.
+  auto widen = [&](int t, int64_t kk, int zero_from) {
+    if constexpr (KV8) {
+      const int sw = warp - 2;
+      const int rs = static_cast<int>(kk % RS);
+      const int cs = static_cast<int>(kk % SK);
+      bool okw = (*abort_flag == 0);
+      if (okw) okw = mbar_wait(smem_addr(&sh->raw_full[t][rs]), static_cast<uint32_t>((kk / RS) & 1), p.error_word);
+      if (okw && kk >= SK)
+        okw = mbar_wait(smem_addr(t == 0 ? &sh->k_empty[cs] : &sh->v_empty[cs]),
+                        static_cast<uint32_t>(((kk / SK) - 1) & 1), p.error_word);
+      if (!okw) *abort_flag = 1;
+      if (okw) {
+        const uint8_t* src = rawring + (t * RS + rs) * Cfg::kRawBytes;
+        uint8_t* dst = (t == 0 ? kring : vring) + cs * Cfg::kTensorBytes;
+        constexpr int CPR = D / 16;          // 16-code chunks per key row
+        constexpr int PL = 16 * CPR / 32;    // chunks per lane (4 at D = 128, 2 at D = 64)
+        uint4 v[PL];
+#pragma unroll
+        for (int j = 0; j < PL; ++j) {
+          const int idx = j * 32 + lane;
+          v[j] = lds_v4(smem_addr(src + (16 * sw + idx / CPR) * D + (idx % CPR) * 16));
+        }
+#pragma unroll
+        for (int j = 0; j < PL; ++j) {
+          const int idx = j * 32 + lane;
+          const int row = 16 * sw + idx / CPR;
+          const int c = idx % CPR;
+          const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+          uint32_t h[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            h[2 * q] = e4m3x2_to_f16x2(w[q] & 0xffffu);
+            h[2 * q + 1] = e4m3x2_to_f16x2(w[q] >> 16);
+          }
+          if (row >= zero_from) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) h[e] = 0u;
+          }
+          // head dims [16c, 16c + 16) = 16-byte chunks 2(c % 4), 2(c % 4) + 1 of panel c / 4, swizzled
+          uint8_t* prow = dst + (c >> 2) * Cfg::kPanelBytes + row * 128;
+          const int j0 = 2 * (c & 3);
+          *reinterpret_cast<uint4*>(prow + ((j0 ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(prow + (((j0 + 1) ^ (row & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_addr(t == 0 ? &sh->k_full[cs] : &sh->v_full[cs]));
+        mbar_arrive(smem_addr(&sh->raw_empty[t][rs]));
+      }
+    }
+  };
+  const int64_t n_tiles = hi - lo;  // this CTA's tiles, in the order every role walks them
+  if constexpr (KV8) {
+    if (n_tiles > 0) widen(0, 0, TK);
+  }
   SegCursor cur;
   cur.init(p, sh->b, sh->base_b, lo, hi, false);
   int64_t k = 0;
@@ -696,6 +704,11 @@ __global__ void __launch_bounds__(384, 1)
     for (int tl = tbegin; tl < tend; ++tl, ++k) {
       const int key0 = tl * TK + wg * TH;   // this warpgroup's half of the tile
       const int sb = static_cast<int>(k % NS);
+      if constexpr (KV8) {
+        // the next tile's K (its Q K^T can then run during this tile's softmax), then this tile's V
+        if (k + 1 < n_tiles) widen(0, k + 1, TK);
+        widen(1, k, L - tl * TK);
+      }
       const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(sb * TK + wg * TH);
       bool ok = (*abort_flag == 0);
       if (ok) ok = mbar_wait(s_bar(k), s_par(k), p.error_word);
@@ -783,7 +796,7 @@ __global__ void __launch_bounds__(384, 1)
         l_run += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
       }
       tc::st_32x32b_x32(s_col, pk);
-      if (key0 + TH > L) {
+      if (!KV8 && key0 + TH > L) {
         // keys >= L in this half: their V rows may be stale or NaN-poisoned; zero them once V has
         // landed (after P is written, so that the wait for V overlaps the softmax above; P V reads
         // them only after this warpgroup's p_full arrival below)
