@@ -25,7 +25,8 @@ constexpr int kMmaPrefetchTiles = 0;
 // write and merge) grows with the rows, a tile's load time does not. Measured best on B200: 2 for
 // 8-row and 5 for 32-row units on the mma.sync kernel (64-key tiles), 2-3 for 64-row and 3-5 for
 // 128-row units on the tcgen05 kernel (128-key tiles). With e4m3 caches a tcgen05 tile takes about
-// twice as long (the producers widen it), so a segment costs fewer tiles: 1 measured best on tree.
+// one and a half times as long (the softmax warps widen it), so a segment costs fewer tiles: 1
+// measured best on chain and tree (2 the same, 0 and 3 slower).
 inline int mma_seg_cost(int rows) { return 1 + rows / 8; }
 inline int tc_seg_cost(int rows, bool kv8) { return kv8 ? 1 : 1 + rows / 64; }
 

@@ -7,7 +7,8 @@
 //   warps 0, 10 producers: TMA loads of each segment's Q tile (3-D box over [B*C, Hq, D]) and of every
 //               tile's K chunks (warp 0) and V chunks (warp 10) reached through the block table, into
 //               separate K and V rings (K is released as soon as its Q K^T is done, V after its P V).
-//               With e4m3 caches they load raw codes and widen each tile once into the 16-bit layout;
+//               With e4m3 caches they load raw codes only, and the softmax warps widen each tile once
+//               into the 16-bit layout;
 //   warp 1      Q K^T issuer (one thread): S = Q K^T (M = 128, N = 128) into one of two tensor-memory
 //               S buffers of 128 fp32 columns;
 //   warp 11     P V issuer (one thread): O_w += P_w V_w per 64-key half w, with P read back from tensor
